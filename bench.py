@@ -1,0 +1,382 @@
+"""Per-layer GPTQ throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload q_proj_4096]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = the whole per-layer path on one synthetic layer: Hessian over all
+calibration tokens (H = 2 X^T X), damping + Cholesky factor of the inverse,
+the blocked GPTQ column loop with lazy-batch updates, unpermute and int4
+packing.  Inputs (X 2.15 GB bf16 for q_proj_4096, larger than the 126 MB L2)
+are resident in HBM before the timed region.  With N > 1 (torchrun), every
+rank quantizes its own independent layer (layers are independent, GPTQ
+overview page "Równoległość"): weak scaling, no collective in the data path.
+
+Prints one JSON line (rank 0).  value = quantized weights/s over all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ quantized weights/s per layer; Hessian+update TFLOP/s vs B200 peak"
+UNIT = "weights/s"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "hessian_tc_kernel_q_proj_4096.md")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="q_proj_4096")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ------------------------------------------------------------------ helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return json.load(open(p)), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic(kernel_src: str):
+    """dram read+write bytes per launch of the Hessian kernel from the committed
+    ncu summary, or None when the kernel source changed since the capture."""
+    import hashlib
+    try:
+        text = open(PROFILE_TRAFFIC).read()
+    except OSError:
+        return None
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    val, src_hash = None, None
+    for line in text.splitlines():
+        if line.startswith("traffic_bytes_per_launch:"):
+            val = float(line.split(":", 1)[1].split()[0])
+        if line.startswith("kernel_source_sha256_16:"):
+            src_hash = line.split(":", 1)[1].strip()
+    return val if (val is not None and src_hash == h) else None
+
+
+def cpu_baseline(spec, threads: int):
+    """The float64 checker on a bounded sample of the same workload, each stage
+    extrapolated to the full layer by its own cost law:
+      Hessian      2048 of n_tokens tokens, full d_in     (x n_tokens/2048, O(N d^2))
+      factor       leading 1024 x 1024 block of that H    (x (d_in/1024)^3, O(d^3))
+      column loop  32 rows at d_in = 1024                 (x d_out/32 x (d_in/1024)^2)
+    """
+    import numpy as np
+    import oracle
+    from post_weight_quantization_accumulate_b200 import synth
+    n_s, d_s, r_s = 2048, min(1024, spec.d_in), 32
+    xb = synth.x_bf16(spec, tokens=slice(0, n_s))
+    t0 = time.perf_counter()
+    H = oracle.hessian(xb)
+    t_h = time.perf_counter() - t0
+    Hs = np.ascontiguousarray(H[:d_s, :d_s])
+    t0 = time.perf_counter()
+    perm, U, _, _ = oracle.prepare(Hs, spec.damp, spec.act_order)
+    t_p = time.perf_counter() - t0
+    W = synth.weight_f32(spec, rows=slice(0, r_s))[:, :d_s].astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.quantize(W, U, perm, spec.bits, spec.group_size if spec.group_size <= d_s else -1,
+                    spec.block_size)
+    t_q = time.perf_counter() - t0
+    full = (t_h * spec.n_tokens / n_s + t_p * (spec.d_in / d_s) ** 3 +
+            t_q * (spec.d_out / r_s) * (spec.d_in / d_s) ** 2)
+    sample = (f"Hessian on {n_s}/{spec.n_tokens} tokens (x{spec.n_tokens / n_s:g}); factor at d={d_s} "
+              f"(x{(spec.d_in / d_s) ** 3:g}); column loop {r_s} rows at d_in={d_s} "
+              f"(x{(spec.d_out / r_s) * (spec.d_in / d_s) ** 2:g}); float64, OpenMP")
+    return {"value": spec.d_out * spec.d_in / full, "unit": UNIT, "cores": threads,
+            "kind": "oracle", "sample": sample, "measured_s": t_h + t_p + t_q,
+            "extrapolated_layer_s": full}
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    threads = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+    from post_weight_quantization_accumulate_b200 import synth
+    spec = synth.WORKLOADS[args.workload]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(spec, threads)
+        if i >= args.warmup:
+            vals.append(cb)
+    value = statistics.median(v["value"] for v in vals)
+    layer_s = spec.d_out * spec.d_in / value
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": config_of(spec, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(spec, n):
+    return {"workload": spec.name, "d_out": spec.d_out, "d_in": spec.d_in, "n_tokens": spec.n_tokens,
+            "bits": spec.bits, "group_size": spec.group_size, "block_size": spec.block_size,
+            "damp": spec.damp, "act_order": spec.act_order, "x_dtype": "bf16",
+            "w_dtype": "bf16" if spec.w_bf16 else "f32",
+            "l2": "inputs larger than L2 (X is %.2f GB)" % (spec.n_tokens * spec.d_in * 2 / 1e9),
+            "parallelism": f"independent layer per rank x{n}"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from post_weight_quantization_accumulate_b200 import binding as B
+    from post_weight_quantization_accumulate_b200 import build as build_mod
+    from post_weight_quantization_accumulate_b200 import synth
+    from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
+
+    if rank == 0:
+        build_mod.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=600))
+        dist.barrier()
+        if rank != 0:
+            build_mod.build()
+    B.lib()
+
+    base = synth.WORKLOADS[args.workload]
+    spec = synth.scaled(base, tensor_id=rank)       # an independent layer per rank
+    threads = len(os.sched_getaffinity(0))
+
+    # inputs: generated on the host, pinned, copied to HBM once
+    xb = synth.x_bf16(spec)
+    X_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    del xb
+    wbits = synth.weight_bf16_bits(spec) if spec.w_bf16 else None
+    W_host = (torch.from_numpy(wbits.view(np.int16)).view(torch.bfloat16) if spec.w_bf16
+              else torch.from_numpy(synth.weight_f32(spec))).pin_memory()
+    X = X_host.to(dev, non_blocking=False)
+    Wd = W_host.to(dev)
+    q = LayerQuantizer(spec.d_out, spec.d_in, spec.bits, spec.group_size, spec.block_size,
+                       spec.damp, spec.act_order, device=dev, keep_codes=False)
+    stream = torch.cuda.current_stream(dev)
+
+    ev_h = []   # (start, end) of the Hessian call per timed step
+
+    def step(record=False):
+        q.reset()
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        q.add_batch(X)
+        if record:
+            e1.record(stream)
+            ev_h.append((e0, e1))
+        q.run(Wd)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = B.gptq_launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = B.gptq_launch_count() - launches0
+    ms = t_start.elapsed_time(t_end) / args.steps
+    h_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_h)
+    status = B.gptq_device_status()
+    if world > 1:
+        t = torch.tensor([ms, h_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, h_ms = float(t[0]), float(t[1])
+    clocks = clk.summary()
+
+    # one step broken down by stage (after the timed region)
+    stage = {}
+    if rank == 0:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        evs[0].record(stream)
+        q.reset()
+        q.add_batch(X)
+        evs[1].record(stream)
+        q.prepare()
+        evs[2].record(stream)
+        q.quantize(Wd)
+        evs[3].record(stream)
+        torch.cuda.synchronize()
+        stage = {"hessian_ms": evs[0].elapsed_time(evs[1]), "prepare_ms": evs[1].elapsed_time(evs[2]),
+                 "quantize_ms": evs[2].elapsed_time(evs[3])}
+
+    # end to end through the public API with host buffers: X and W copied in
+    # (overlapped chunked copy of X), packed codes + scales + zeros + g_idx out
+    e2e = None
+    if not args.no_e2e:
+        packed_h = torch.empty_like(q.packed, device="cpu").pin_memory()
+        scales_h = torch.empty_like(q.scales, device="cpu").pin_memory()
+        zeros_h = torch.empty_like(q.zeros, device="cpu").pin_memory()
+        gidx_h = torch.empty_like(q.g_idx, device="cpu").pin_memory()
+        Wd2 = torch.empty_like(Wd)
+
+        def e2e_step():
+            q.reset()
+            q.add_batch_host(X_host, chunk_tokens=16384)
+            Wd2.copy_(W_host, non_blocking=True)
+            res = q.run(Wd2)
+            packed_h.copy_(res.packed, non_blocking=True)
+            scales_h.copy_(res.scales, non_blocking=True)
+            zeros_h.copy_(res.zeros, non_blocking=True)
+            gidx_h.copy_(res.g_idx, non_blocking=True)
+
+        for _ in range(min(args.warmup, 2)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        h2d = X_host.numel() * 2 + W_host.numel() * W_host.element_size()
+        d2h = (packed_h.numel() + scales_h.numel() * 4 + zeros_h.numel() * 4 + gidx_h.numel() * 4)
+        e2e = {"value": world * spec.d_out * spec.d_in / (e2e_ms / 1e3), "unit": UNIT,
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+        cpu = cpu_baseline(spec, threads)
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        alg_flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)   # upper triangle incl. diagonal
+        achieved = alg_flops / (h_ms / 1e3) / 1e12
+        traffic = profiled_traffic(os.path.join(ROOT, "post_weight_quantization_accumulate_b200",
+                                                "csrc", "hessian.cu"))
+        line = {
+            "metric": METRIC, "value": world * spec.d_out * spec.d_in / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_of(spec, world),
+            "roofline": {"kernel": "hessian_tc_kernel (+ mirror copy)", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                         "flops_per_launch": alg_flops, "launch_ms": h_ms},
+            "hessian_tflops_dense_equiv": 2 * spec.n_tokens * spec.d_in ** 2 / (h_ms / 1e3) / 1e12,
+            "stages_ms": stage,
+            "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
+            "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

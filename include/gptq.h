@@ -1,0 +1,180 @@
+/*
+ * gptq.h -- C ABI of libgptq.so, the per-layer GPTQ quantizer for NVIDIA B200
+ * (sm_100a).
+ *
+ * What it computes (GPTQ overview page, robocikowo.com/technologie-ai/gptq):
+ *   "Jak działa"      each linear layer is quantized on its own: H = 2 X X^T
+ *                     from the layer's input activations; weights quantized
+ *                     column by column in a fixed order; after each column the
+ *                     not-yet-quantized weights are corrected by the Optimal
+ *                     Brain Surgeon rule through the inverse Hessian; block
+ *                     updates; 4- or 3-bit weights with a scale per group.
+ *   "Komponenty"      the Cholesky factorisation of the inverse Hessian.
+ *   "Hiperparametry"  bit width, weights per scale, activation order, value
+ *                     added to the Hessian diagonal.
+ * and the calibration flow of the torchao issue "GPTQ implementation with
+ * tensor subclasses" ("Background": gather the activations reaching a linear,
+ * update its weight, use the updated weight for its outputs).
+ *
+ * Conventions shared by every call:
+ *   - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *     owns every buffer; the library allocates no device memory in any call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are stream-ordered and asynchronous unless stated.
+ *   - Matrices are row-major.  W is [d_out, d_in] (PyTorch Linear layout; a
+ *     "column" is an input channel).  X is [n_tokens, d_in].
+ *   - Arguments are validated on the host before any launch; an invalid
+ *     argument returns GPTQ_ERR_INVALID_ARG and launches nothing.
+ *   - A CUDA error returns GPTQ_ERR_CUDA; gptq_last_cuda_error() gives it.
+ *   - Device-side waits are bounded; a wait that runs out records
+ *     GPTQ_ERR_TIMEOUT in the device status word (see gptq_device_status()).
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or option        */
+    GPTQ_ERR_NOT_PD = 2,      /* damped Hessian not positive definite          */
+    GPTQ_ERR_NONFINITE = 3,   /* NaN/Inf met in H                              */
+    GPTQ_ERR_CUDA = 4,        /* a CUDA runtime call failed                    */
+    GPTQ_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up            */
+    GPTQ_ERR_WORKSPACE = 6,   /* workspace pointer NULL/misaligned or too small */
+    GPTQ_ERR_UNSUPPORTED = 7  /* device is not sm_100                          */
+} gptq_status;
+
+/* Static English text for a status code.  Never NULL. */
+const char *gptq_status_string(int status);
+
+/* Text of the last CUDA error seen by this library in this thread ("" if none). */
+const char *gptq_last_cuda_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int gptq_version(void);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all threads).  Lets callers count device work without a profiler. */
+uint64_t gptq_launch_count(void);
+
+/* Reads and clears the device status word of the current device: 0 or the
+ * first gptq_status a kernel recorded (a timed-out wait, an invalid pivot).
+ * Synchronises the current device. */
+int gptq_device_status(void);
+
+/* Bytes of workspace gptq_prepare (d_in) and gptq_quantize (d_out, d_in,
+ * block_size, with or without an activation order) need; the maximum of the
+ * two is safe for both.  The workspace must be 256-byte aligned.  Returns 0
+ * for invalid sizes. */
+size_t gptq_workspace_bytes(int64_t d_out, int64_t d_in, int block_size);
+
+/*
+ * H += 2 * X^T X   ("Jak działa": H = 2 X X^T; "Złożoność obliczeniowa":
+ * O(N_calib d^2)).  Call it once per calibration chunk; H accumulates across
+ * calls, so a saved H is a resumable checkpoint.
+ *
+ *   H         float32 [d_in, d_in], IN/OUT, full symmetric matrix.  The caller
+ *             zero-initialises it before the first chunk.  On return both
+ *             triangles hold the sum (bitwise symmetric).  16-byte aligned.
+ *   X         bfloat16 bit patterns [n_tokens, d_in], row-major, 16-byte
+ *             aligned.  Products of bf16 values are exact; sums are float32
+ *             (tensor cores, tcgen05 kind::f16, accumulating in TMEM).
+ *   n_tokens  >= 0 (0 is a no-op).
+ *   d_in      > 0, multiple of 8 (TMA row pitch), <= 65536.
+ */
+int gptq_hessian_accumulate(float *H, const uint16_t *X, int64_t n_tokens, int64_t d_in,
+                            void *stream);
+
+/*
+ * Same as gptq_hessian_accumulate with X in HOST memory: the rows are copied
+ * in chunks of `chunk_tokens` through two caller-owned device staging buffers
+ * while earlier chunks are accumulated, so the copy overlaps the tensor-core
+ * work.  X_host should be page-locked for the copies to be asynchronous.
+ *
+ *   X_host        host bf16 bit patterns [n_tokens, d_in].
+ *   staging       device buffer of 2 * chunk_tokens * d_in uint16, 16-byte
+ *                 aligned, not used by anything else until the stream reaches
+ *                 the end of this call's work.
+ *   chunk_tokens  > 0.
+ * Returns after all copies and kernels are enqueued; the host buffer must stay
+ * valid until `stream` has finished them.
+ */
+int gptq_hessian_accumulate_host(float *H, const uint16_t *X_host, int64_t n_tokens,
+                                 int64_t d_in, uint16_t *staging, int64_t chunk_tokens,
+                                 void *stream);
+
+/*
+ * Damping, activation order and the Cholesky factor of the inverse Hessian
+ * ("Hiperparametry": value added to the diagonal, quantizing columns in order
+ * of activation importance; "Komponenty": Cholesky of the inverse Hessian).
+ *
+ *   mu = mean(diag H);  H_d = H + damp * mu * I.
+ *   act_order != 0: perm = order of descending diag(H) (undamped), equal keys
+ *                   in increasing column index; otherwise perm = identity.
+ *   U (Hinv_chol) = the upper-triangular factor with U^T U = (P^T H_d P)^{-1},
+ *                   P the permutation, i.e. rows/columns in processing order.
+ *                   Computed as M = chol_lower(J P^T H_d P J), U = J M^{-1} J
+ *                   (J = index reversal), all in float32.
+ *
+ *   H          float32 [d_in, d_in] symmetric, read only.
+ *   damp       >= 0 (0.01 typical).
+ *   perm       int32 [d_in], OUT: perm[k] = original column processed k-th.
+ *   Hinv_chol  float32 [d_in, d_in], OUT: U, entries below the diagonal 0.
+ *   workspace  >= gptq_workspace_bytes(0, d_in, 1) bytes.
+ * Synchronises `stream` once to read the factorisation status.  Returns
+ * GPTQ_ERR_NOT_PD if mean(diag H) <= 0 or a pivot is not positive,
+ * GPTQ_ERR_NONFINITE if H holds NaN/Inf on its diagonal.
+ */
+int gptq_prepare(const float *H, int64_t d_in, float damp, int act_order, int32_t *perm,
+                 float *Hinv_chol, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * GPTQ column loop ("Jak działa"): for columns c in processing order, with a
+ * new per-row (scale, zero) at each group start taken from the row's current
+ * values of the group's columns (range including 0; an all-zero range is
+ * [-1, 1]):
+ *     s = (max - min) / (2^bits - 1),  z = rint(-min / s)
+ *     q = clamp(rint(w_c / s) + z, 0, 2^bits - 1),  w^_c = s (q - z)
+ *     e = (w_c - w^_c) / U[c,c],   w[c+1:] -= e * U[c, c+1:]
+ * with the correction of columns beyond the current block of `block_size`
+ * columns applied once per block as W[:, j+B:] -= E_blk U[j:j+B, j+B:].
+ * Grid choice and rounding are decided in float32; ties round to even.
+ *
+ *   W           float32 [d_out, d_in] IN/OUT, original column order.  On
+ *               return it holds the dequantized weights W^ (original order).
+ *   Hinv_chol   U from gptq_prepare (processing order).
+ *   perm        int32 [d_in] from gptq_prepare, or NULL for identity.
+ *   bits        1..8 (2, 3, 4 are the GPTQ widths; codes are one byte each).
+ *   group_size  > 0 and dividing d_in, or -1 for one (scale, zero) per row
+ *               from the original row.  group_size must divide block_size or
+ *               be a multiple of it.
+ *   block_size  1..128, the lazy-batch width.
+ *   codes       uint8 [d_out, d_in] OUT (original column order) or NULL.
+ *   scales      float32 [d_out, n_groups] OUT, groups in processing order;
+ *               n_groups = d_in / group_size (1 when group_size = -1).
+ *   zeros       float32 [d_out, n_groups] OUT, integer-valued.
+ *   packed_int4 uint8 [d_out, d_in / 2] OUT or NULL; needs bits <= 4 and even
+ *               d_in: column 2i in the low nibble, 2i + 1 in the high nibble.
+ *   g_idx       int32 [d_in] OUT or NULL: group of each original column.
+ *   err_sq      float32 [d_out] OUT or NULL: sum over columns of e^2.
+ *   workspace   >= gptq_workspace_bytes(d_out, d_in, block_size) bytes.
+ */
+int gptq_quantize(float *W, const float *Hinv_chol, const int32_t *perm, int64_t d_out,
+                  int64_t d_in, int bits, int group_size, int block_size, uint8_t *codes,
+                  float *scales, float *zeros, uint8_t *packed_int4, int32_t *g_idx,
+                  float *err_sq, void *workspace, size_t ws_bytes, void *stream);
+
+/* dst[i] = (float) bf16 src[i] (exact widening), n >= 0 elements. */
+int gptq_bf16_to_f32(float *dst, const uint16_t *src, int64_t n, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

@@ -1,0 +1,322 @@
+// hessian.cu -- H += 2 X^T X on the sm_100a tensor cores.
+//
+// GPTQ overview page, "Jak działa": the layer Hessian is H = 2 X X^T from the
+// input activations (X there is d x N; here X is [N, d], so H = 2 X^T X);
+// "Złożoność obliczeniowa": O(N_calib d^2), the dominant cost of the method
+// for calibration sets much larger than d.
+//
+// Design (B200):
+//  * H is symmetric, so only tiles meeting the upper triangle are computed:
+//    128 x 256 output tiles, (ti, tj) with tj >= ti / 2.  The strict lower
+//    triangle is written afterwards by a transpose copy (mirror_upper_kernel),
+//    so H is bitwise symmetric.
+//  * Both operands are slices of the same X rows: A = X[t, 128 i-cols],
+//    B = X[t, 256 j-cols].  Their contraction index (tokens) is the outer
+//    dimension of X, so both are MN-major; TMA brings 64-token x 64-column
+//    boxes with 128-byte swizzle, which is the canonical MN-major SW128
+//    layout tcgen05.mma reads directly.
+//  * Work units = (tile, token split of kSplitTokens).  A persistent grid of
+//    one CTA per SM walks the units split-major, so concurrently running
+//    units read the same token rows of X (L2 reuse).  Each unit accumulates
+//    in TMEM (fp32) and is flushed with fp32 red.add into H, which bounds the
+//    length of any single fp32 accumulation chain.
+//  * Warp roles per CTA (192 threads): warp 0 = TMA producer, warp 1 = MMA
+//    issuer + TMEM owner, warps 2-5 = epilogue (TMEM lanes 0-127).  A 4-stage
+//    shared-memory ring (48 KB per stage) and two TMEM accumulators (2 x 256
+//    columns) let the epilogue of one unit overlap the MMAs of the next.
+//  * Every mbarrier wait is bounded; a time-out records GPTQ_ERR_TIMEOUT,
+//    releases the other roles, and the CTA still frees its TMEM.
+#include "common.cuh"
+
+#include <mutex>
+
+namespace gptq {
+
+namespace {
+
+constexpr int kBM = 128;          // H rows per tile (UMMA M)
+constexpr int kBN = 256;          // H cols per tile (UMMA N)
+constexpr int kBK = 64;           // tokens per pipeline stage
+constexpr int kStages = 4;
+constexpr int kBoxCols = 64;      // 64 bf16 = 128 bytes = one swizzle row
+constexpr int kBoxBytes = kBK * kBoxCols * 2;           // 8 KB
+constexpr int kABytes = kBoxBytes * (kBM / kBoxCols);   // 16 KB
+constexpr int kBBytes = kBoxBytes * (kBN / kBoxCols);   // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;          // 48 KB
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;    // two 256-column fp32 accumulators
+constexpr int kSplitTokens = 8192;
+constexpr uint32_t kIdesc = idesc_f32acc(1 /*bf16*/, 1, 1, kBM, kBN);
+
+struct alignas(1024) HessSmem {
+    uint8_t stage[kStages][kStageBytes];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr size_t kSmemBytes = sizeof(HessSmem) + 1024;
+
+// Upper-triangle tile number -> (ti, tj); row block ti has tiles tj in
+// [ti/2, n_tj).
+__device__ __forceinline__ void tile_coords(int tile, int n_ti, int n_tj, int& ti, int& tj)
+{
+    int idx = tile;
+    for (int i = 0; i < n_ti; ++i) {
+        int cnt = n_tj - (i >> 1);
+        if (idx < cnt) {
+            ti = i;
+            tj = (i >> 1) + idx;
+            return;
+        }
+        idx -= cnt;
+    }
+    ti = n_ti - 1;
+    tj = n_tj - 1;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int d,
+                      int n_tokens, int n_ti, int n_tj, int n_tiles, int n_split, int* status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    HessSmem& S = *reinterpret_cast<HessSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.tfull[b], 1);
+            mbar_init(&S.tempty[b], 4);
+        }
+        S.abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap);
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = S.tmem_base;
+    volatile int* abort = &S.abort;
+    const int n_units = n_tiles * n_split;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+                int ti, tj;
+                tile_coords(u % n_tiles, n_ti, n_tj, ti, tj);
+                const int t0 = (u / n_tiles) * kSplitTokens;
+                const int t1 = min(n_tokens, t0 + kSplitTokens);
+                for (int t = t0; t < t1; t += kBK, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) break;
+                    mbar_arrive_expect_tx(&S.full[s], kStageBytes);
+                    uint8_t* a = S.stage[s];
+                    uint8_t* b = a + kABytes;
+#pragma unroll
+                    for (int m = 0; m < kBM / kBoxCols; ++m)
+                        tma_load_2d(a + m * kBoxBytes, &tmap, &S.full[s], ti * kBM + m * kBoxCols, t);
+#pragma unroll
+                    for (int m = 0; m < kBN / kBoxCols; ++m)
+                        tma_load_2d(b + m * kBoxBytes, &tmap, &S.full[s], tj * kBN + m * kBoxCols, t);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t it = 0, uc = 0;
+            for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++uc) {
+                const int b = uc & 1;
+                const uint32_t uph = (uc >> 1) & 1;
+                if (!mbar_wait_bounded(&S.tempty[b], uph ^ 1, abort, status)) break;
+                tc_fence_after();
+                const uint32_t dt = tbase + b * kBN;
+                const int t0 = (u / n_tiles) * kSplitTokens;
+                const int t1 = min(n_tokens, t0 + kSplitTokens);
+                const int nk = (t1 - t0 + kBK - 1) / kBK;
+                bool ok = true;
+                for (int kk = 0; kk < nk; ++kk, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait_bounded(&S.full[s], ph, abort, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(S.stage[s]);
+                    const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        // 16 tokens = two 8-row swizzle groups = 2048 bytes
+                        const uint64_t ad = sdesc_sw128(a0 + k * 2048, kBoxBytes, 1024);
+                        const uint64_t bd = sdesc_sw128(b0 + k * 2048, kBoxBytes, 1024);
+                        umma_f16(dt, ad, bd, kIdesc, (kk | k) != 0);
+                    }
+                    umma_commit(&S.empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&S.tfull[b]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        uint32_t uc = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uc) {
+            const int b = uc & 1;
+            const uint32_t uph = (uc >> 1) & 1;
+            // every lane waits, so the warp stays converged for tcgen05.ld
+            const bool ok = mbar_wait_bounded(&S.tfull[b], uph, abort, status);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            int ti, tj;
+            tile_coords(u % n_tiles, n_ti, n_tj, ti, tj);
+            const int row = ti * kBM + row_in_tile;
+            const uint32_t taddr = tbase + (static_cast<uint32_t>(q * 32) << 16) + b * kBN;
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                float v[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, v);
+                tmem_ld_wait();
+                const int col0 = tj * kBN + c * 32;
+                if (row < d && col0 < d && col0 + 31 >= row) {
+                    float* dst = H + static_cast<int64_t>(row) * d + col0;
+                    if (col0 + 32 <= d) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m)
+                            atomicAdd(reinterpret_cast<float4*>(dst) + m,
+                                      make_float4(2.f * v[4 * m], 2.f * v[4 * m + 1],
+                                                  2.f * v[4 * m + 2], 2.f * v[4 * m + 3]));
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 32; ++m)
+                            if (m < d - col0) atomicAdd(dst + m, 2.f * v[m]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tempty[b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+// H[j][i] = H[i][j] for i < j: copies the upper triangle into the lower one
+// through a 32 x 32 shared-memory transpose.
+__global__ void mirror_upper_kernel(float* __restrict__ H, int d)
+{
+    __shared__ float t[32][33];
+    const int bx = blockIdx.x, by = blockIdx.y;
+    if (bx > by) return;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const int i = bx * 32 + r, j = by * 32 + threadIdx.x;
+        if (i < d && j < d) t[r][threadIdx.x] = H[static_cast<int64_t>(i) * d + j];
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const int row = by * 32 + r, col = bx * 32 + threadIdx.x;
+        if (row < d && col < d && row > col) H[static_cast<int64_t>(row) * d + col] = t[threadIdx.x][r];
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+// Tensor map over X [n_rows, d] bf16 with 64 x 64 boxes, 128-byte swizzle;
+// rows beyond n_rows read as zero.
+int make_x_tmap(CUtensorMap* map, const uint16_t* X, int64_t n_rows, int64_t d)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n_rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[2] = {kBoxCols, kBK};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return GPTQ_OK;
+}
+
+// Accumulates the upper triangle of 2 X^T X (n_rows < 2^31) into H.
+int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
+                         cudaStream_t stream)
+{
+    if (n_rows <= 0) return GPTQ_OK;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
+    if (dev < 64 && !attr_set[dev]) {
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(hessian_tc_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes)));
+        attr_set[dev] = true;
+    }
+    CUtensorMap map;
+    int rc = make_x_tmap(&map, X, n_rows, d);
+    if (rc) return rc;
+    const int n_ti = static_cast<int>((d + kBM - 1) / kBM);
+    const int n_tj = static_cast<int>((d + kBN - 1) / kBN);
+    int n_tiles = 0;
+    for (int i = 0; i < n_ti; ++i) n_tiles += n_tj - (i >> 1);
+    const int n_split = static_cast<int>((n_rows + kSplitTokens - 1) / kSplitTokens);
+    const int64_t units = static_cast<int64_t>(n_tiles) * n_split;
+    const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
+    hessian_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
+        map, H, static_cast<int>(d), static_cast<int>(n_rows), n_ti, n_tj, n_tiles, n_split,
+        device_status_ptr());
+    GPTQ_LAUNCH_CHECK();
+    return GPTQ_OK;
+}
+
+int launch_mirror(float* H, int64_t d, cudaStream_t stream)
+{
+    const int nb = static_cast<int>((d + 31) / 32);
+    mirror_upper_kernel<<<dim3(nb, nb), dim3(32, 8), 0, stream>>>(H, static_cast<int>(d));
+    GPTQ_LAUNCH_CHECK();
+    return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -1,0 +1,347 @@
+// prepare.cu -- damping, activation order, and the Cholesky factor of the
+// inverse Hessian.
+//
+// GPTQ overview page: "Hiperparametry" (a value added to the Hessian
+// diagonal for numerical stability; columns quantized in order of activation
+// importance) and "Komponenty" / "Jak działa" (a Cholesky decomposition of
+// the inverse Hessian gives stability on large layers).
+//
+// Route: with P the processing order and J the index reversal,
+//   A   = J P^T (H + delta I) P J          (one gather pass, delta = damp * mean diag H)
+//   M   = chol_lower(A)                    (blocked, right-looking, fp32)
+//   U   = J M^{-1} J                       (upper; U^T U = (P^T H_d P)^{-1})
+// which needs one Cholesky and one triangular inverse (2/3 d^3 flops) instead
+// of inverse + Cholesky of the inverse.
+#include "common.cuh"
+#include "gemm.cuh"
+
+#include <algorithm>
+
+namespace gptq {
+
+struct PrepHeader {
+    int status;
+    float mean;
+    float delta;
+    int pad;
+};
+
+constexpr int kNB = 64;  // panel width of the blocked Cholesky / leaf of the inverse
+
+size_t prepare_workspace_bytes(int64_t d)
+{
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t dd = static_cast<size_t>(d) * static_cast<size_t>(d) * sizeof(float);
+    return 256 + up(dd) /*A,M*/ + up(dd) /*Minv*/ + up(dd) /*T*/ +
+           up(static_cast<size_t>(d) * kNB * sizeof(float)) /*Dinv*/;
+}
+
+namespace {
+
+// mean(diag H) in double, delta = damp * mean (float); diagonal sanity.
+__global__ void diag_mean_kernel(const float* __restrict__ H, int d, float damp, PrepHeader* hdr)
+{
+    __shared__ double part[32];
+    __shared__ int bad[1];
+    if (threadIdx.x == 0) bad[0] = 0;
+    __syncthreads();
+    double s = 0.0;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        const float v = H[static_cast<int64_t>(i) * d + i];
+        if (!isfinite(v)) bad[0] = 1;
+        s += v;
+    }
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += part[w];
+        const float mean = static_cast<float>(t / d);
+        hdr->mean = mean;
+        hdr->delta = damp * mean;
+        if (bad[0])
+            hdr->status = GPTQ_ERR_NONFINITE;
+        else if (!(mean > 0.f))
+            hdr->status = GPTQ_ERR_NOT_PD;
+    }
+}
+
+// perm[rank(i)] = i with rank by descending diag(H), ties by lower index.
+__global__ void act_order_kernel(const float* __restrict__ H, int d, int act_order,
+                                 int32_t* __restrict__ perm)
+{
+    __shared__ float key[1024];
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (!act_order) {
+        if (i < d) perm[i] = i;
+        return;
+    }
+    const float ki = (i < d) ? H[static_cast<int64_t>(i) * d + i] : 0.f;
+    int rank = 0;
+    for (int j0 = 0; j0 < d; j0 += 1024) {
+        __syncthreads();
+        for (int t = threadIdx.x; t < 1024; t += blockDim.x) {
+            const int j = j0 + t;
+            key[t] = (j < d) ? H[static_cast<int64_t>(j) * d + j] : 0.f;
+        }
+        __syncthreads();
+        const int jn = min(1024, d - j0);
+        for (int t = 0; t < jn; ++t) {
+            const float kj = key[t];
+            rank += (kj > ki) || (kj == ki && j0 + t < i);
+        }
+    }
+    if (i < d) perm[rank] = i;
+}
+
+// A[a][b] = H[q(a)][q(b)] + (a == b ? delta : 0), q(a) = perm[d-1-a]; one
+// row of H staged in shared memory per CTA (d <= kGatherSmemMax).
+constexpr int kGatherSmemMax = 16384;
+__global__ void gather_rev_kernel(const float* __restrict__ H, int d,
+                                  const int32_t* __restrict__ perm, const PrepHeader* hdr,
+                                  float* __restrict__ A)
+{
+    extern __shared__ float rowbuf[];
+    const float delta = hdr->delta;
+    for (int a = blockIdx.x; a < d; a += gridDim.x) {
+        const int qa = perm[d - 1 - a];
+        __syncthreads();
+        const float* src = H + static_cast<int64_t>(qa) * d;
+        for (int j = threadIdx.x; j < d; j += blockDim.x) rowbuf[j] = src[j];
+        __syncthreads();
+        float* dst = A + static_cast<int64_t>(a) * d;
+        for (int b = threadIdx.x; b < d; b += blockDim.x) {
+            float v = rowbuf[perm[d - 1 - b]];
+            if (b == a) v += delta;
+            dst[b] = v;
+        }
+    }
+}
+
+__global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
+                                         const int32_t* __restrict__ perm, const PrepHeader* hdr,
+                                         float* __restrict__ A)
+{
+    const float delta = hdr->delta;
+    const int64_t n = static_cast<int64_t>(d) * d;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int a = static_cast<int>(idx / d), b = static_cast<int>(idx % d);
+        float v = H[static_cast<int64_t>(perm[d - 1 - a]) * d + perm[d - 1 - b]];
+        if (a == b) v += delta;
+        A[idx] = v;
+    }
+}
+
+// Factor the kb x kb diagonal block at (k0, k0) of A in place (lower) and
+// write its inverse into Dinv[k0 .. k0+kb) (row stride kNB).
+__global__ void __launch_bounds__(256)
+    potrf_block_kernel(float* __restrict__ A, int d, int k0, int kb, float* __restrict__ Dinv,
+                       PrepHeader* hdr)
+{
+    __shared__ float L[kNB][kNB + 1];
+    __shared__ float X[kNB][kNB + 1];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = 0;
+    for (int idx = tid; idx < kNB * kNB; idx += blockDim.x) {
+        const int i = idx / kNB, j = idx % kNB;
+        L[i][j] = (i < kb && j < kb && j <= i) ? A[static_cast<int64_t>(k0 + i) * d + k0 + j]
+                                                 : 0.f;
+    }
+    __syncthreads();
+    for (int c = 0; c < kb; ++c) {
+        if (tid == 0) {
+            const float p = L[c][c];
+            if (!(p > 0.f) || !isfinite(p)) {
+                bad = 1;
+                L[c][c] = 1.f;
+            } else {
+                L[c][c] = sqrtf(p);
+            }
+        }
+        __syncthreads();
+        const float lcc = L[c][c];
+        for (int i = c + 1 + tid; i < kb; i += blockDim.x) L[i][c] = L[i][c] / lcc;
+        __syncthreads();
+        const int rem = kb - c - 1;
+        for (int idx = tid; idx < rem * rem; idx += blockDim.x) {
+            const int i = c + 1 + idx / rem, j = c + 1 + idx % rem;
+            if (j <= i) L[i][j] = fmaf(-L[i][c], L[j][c], L[i][j]);
+        }
+        __syncthreads();
+    }
+    // inverse of the lower factor, one column per thread: L x = e_j
+    if (tid < kb) {
+        const int j = tid;
+        for (int i = 0; i < kb; ++i) {
+            if (i < j) {
+                X[i][j] = 0.f;
+                continue;
+            }
+            float s = (i == j) ? 1.f : 0.f;
+            for (int k = j; k < i; ++k) s = fmaf(-L[i][k], X[k][j], s);
+            X[i][j] = s / L[i][i];
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
+        const int i = idx / kb, j = idx % kb;
+        A[static_cast<int64_t>(k0 + i) * d + k0 + j] = (j <= i) ? L[i][j] : 0.f;
+        Dinv[static_cast<int64_t>(k0 + i) * kNB + j] = X[i][j];
+    }
+    if (tid == 0 && bad) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
+}
+
+// Panel below the diagonal block: L[r][k0:k0+kb] = A[r][k0:k0+kb] * Dinv^T,
+// 64 rows per CTA.
+__global__ void __launch_bounds__(256)
+    trsm_panel_kernel(float* __restrict__ A, int d, int k0, int kb,
+                      const float* __restrict__ Dinv)
+{
+    __shared__ float T[kNB][kNB + 1];
+    __shared__ float Di[kNB][kNB + 1];
+    const int r0 = k0 + kb + blockIdx.x * kNB;
+    const int tid = threadIdx.x;
+    for (int idx = tid; idx < kNB * kNB; idx += blockDim.x) {
+        const int i = idx / kNB, j = idx % kNB;
+        const int r = r0 + i;
+        T[i][j] = (r < d && j < kb) ? A[static_cast<int64_t>(r) * d + k0 + j] : 0.f;
+        Di[i][j] = (i < kb && j < kb) ? Dinv[static_cast<int64_t>(k0 + i) * kNB + j] : 0.f;
+    }
+    __syncthreads();
+    // out[i][j] = sum_{k <= j} T[i][k] * Di[j][k]
+    for (int idx = tid; idx < kNB * kNB; idx += blockDim.x) {
+        const int i = idx / kNB, j = idx % kNB;
+        const int r = r0 + i;
+        if (r >= d || j >= kb) continue;
+        float s = 0.f;
+        for (int k = 0; k <= j; ++k) s = fmaf(T[i][k], Di[j][k], s);
+        A[static_cast<int64_t>(r) * d + k0 + j] = s;
+    }
+}
+
+// Minv diagonal blocks from Dinv.
+__global__ void place_dinv_kernel(float* __restrict__ Minv, int d, const float* __restrict__ Dinv)
+{
+    const int64_t n = static_cast<int64_t>(d) * kNB;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int r = static_cast<int>(idx / kNB), j = static_cast<int>(idx % kNB);
+        const int c = (r / kNB) * kNB + j;
+        if (c < d && j <= r % kNB) Minv[static_cast<int64_t>(r) * d + c] = Dinv[idx];
+    }
+}
+
+// U[i][j] = Minv[d-1-i][d-1-j] for i <= j, 0 below the diagonal.
+__global__ void reverse_upper_kernel(const float* __restrict__ Minv, int d, float* __restrict__ U)
+{
+    const int64_t n = static_cast<int64_t>(d) * d;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int i = static_cast<int>(idx / d), j = static_cast<int>(idx % d);
+        U[idx] = (i <= j) ? Minv[static_cast<int64_t>(d - 1 - i) * d + (d - 1 - j)] : 0.f;
+    }
+}
+
+}  // namespace
+
+int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t* perm, float* U,
+                void* workspace, cudaStream_t stream, int* host_status)
+{
+    const int d = static_cast<int>(d64);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t dd = static_cast<size_t>(d) * d * sizeof(float);
+    PrepHeader* hdr = reinterpret_cast<PrepHeader*>(ws);
+    float* A = reinterpret_cast<float*>(ws + 256);
+    float* Minv = reinterpret_cast<float*>(ws + 256 + up(dd));
+    float* T = reinterpret_cast<float*>(ws + 256 + 2 * up(dd));
+    float* Dinv = reinterpret_cast<float*>(ws + 256 + 3 * up(dd));
+    const int nsm = sm_count();
+
+    GPTQ_CUDA_CHECK(cudaMemsetAsync(hdr, 0, sizeof(PrepHeader), stream));
+    diag_mean_kernel<<<1, 1024, 0, stream>>>(H, d, damp, hdr);
+    GPTQ_LAUNCH_CHECK();
+    act_order_kernel<<<(d + 255) / 256, 256, 0, stream>>>(H, d, act_order, perm);
+    GPTQ_LAUNCH_CHECK();
+    if (d <= kGatherSmemMax) {
+        const size_t sm = static_cast<size_t>(d) * sizeof(float);
+        static bool attr = false;
+        if (!attr) {
+            GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gather_rev_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kGatherSmemMax * static_cast<int>(sizeof(float))));
+            attr = true;
+        }
+        gather_rev_kernel<<<std::min(d, nsm * 8), 256, sm, stream>>>(H, d, perm, hdr, A);
+    } else {
+        gather_rev_direct_kernel<<<nsm * 8, 256, 0, stream>>>(H, d, perm, hdr, A);
+    }
+    GPTQ_LAUNCH_CHECK();
+
+    // blocked right-looking Cholesky, A = M M^T (lower)
+    for (int k0 = 0; k0 < d; k0 += kNB) {
+        const int kb = std::min(kNB, d - k0);
+        potrf_block_kernel<<<1, 256, 0, stream>>>(A, d, k0, kb, Dinv, hdr);
+        GPTQ_LAUNCH_CHECK();
+        const int rest = d - k0 - kb;
+        if (rest <= 0) break;
+        trsm_panel_kernel<<<(rest + kNB - 1) / kNB, 256, 0, stream>>>(A, d, k0, kb, Dinv);
+        GPTQ_LAUNCH_CHECK();
+        float* P = A + static_cast<int64_t>(k0 + kb) * d + k0;
+        float* C = A + static_cast<int64_t>(k0 + kb) * d + k0 + kb;
+        int rc = launch_sgemm(true, rest, rest, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,
+                              kGemmLowerC, stream);
+        if (rc) return rc;
+    }
+
+    // M^{-1}: leaves from Dinv, then recursive doubling
+    //   [A 0; B C]^{-1} = [A^-1 0; -C^-1 B A^-1  C^-1]
+    GPTQ_CUDA_CHECK(cudaMemsetAsync(Minv, 0, dd, stream));
+    place_dinv_kernel<<<nsm * 4, 256, 0, stream>>>(Minv, d, Dinv);
+    GPTQ_LAUNCH_CHECK();
+    for (int s = 2 * kNB; s / 2 < d; s *= 2) {
+        const int h = s / 2;
+        const int nfull = d / s;               // subproblems of full size s
+        // full-size subproblems, batched
+        if (nfull > 0) {
+            const int64_t stride = static_cast<int64_t>(s) * d + s;  // diagonal step
+            int rc = launch_sgemm(false, h, h, h, 1.f, A + static_cast<int64_t>(h) * d, d, stride,
+                                  Minv, d, stride, 0.f, T, h, static_cast<int64_t>(h) * h, nfull,
+                                  kGemmLowerB, stream);
+            if (rc) return rc;
+            rc = launch_sgemm(false, h, h, h, -1.f, Minv + static_cast<int64_t>(h) * d + h, d,
+                              stride, T, h, static_cast<int64_t>(h) * h, 0.f,
+                              Minv + static_cast<int64_t>(h) * d, d, stride, nfull, kGemmLowerA,
+                              stream);
+            if (rc) return rc;
+        }
+        // ragged tail subproblem: offset o = nfull * s, size d - o > h
+        const int o = nfull * s;
+        const int m2 = d - o - h;
+        if (m2 > 0) {
+            const float* Bo = A + static_cast<int64_t>(o + h) * d + o;
+            const float* Ai = Minv + static_cast<int64_t>(o) * d + o;
+            int rc = launch_sgemm(false, m2, h, h, 1.f, Bo, d, 0, Ai, d, 0, 0.f, T, h, 0, 1,
+                                  kGemmLowerB, stream);
+            if (rc) return rc;
+            const float* Ci = Minv + static_cast<int64_t>(o + h) * d + o + h;
+            rc = launch_sgemm(false, m2, h, m2, -1.f, Ci, d, 0, T, h, 0, 0.f,
+                              Minv + static_cast<int64_t>(o + h) * d + o, d, 0, 1, kGemmLowerA,
+                              stream);
+            if (rc) return rc;
+        }
+    }
+    reverse_upper_kernel<<<nsm * 8, 256, 0, stream>>>(Minv, d, U);
+    GPTQ_LAUNCH_CHECK();
+
+    int st = 0;
+    GPTQ_CUDA_CHECK(cudaMemcpyAsync(&st, &hdr->status, sizeof(int), cudaMemcpyDeviceToHost, stream));
+    GPTQ_CUDA_CHECK(cudaStreamSynchronize(stream));
+    *host_status = st;
+    return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects invalid arguments on the host before touching a device (no GPU
+needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_accumulate_b200 import binding as B
+from post_weight_quantization_accumulate_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_all_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the binding covers exactly the header
+    assert sorted(s[0] for s in B.SIGNATURES) == names
+
+
+def test_version_status_strings(lib):
+    assert B.gptq_version() >= 100
+    assert B.gptq_status_string(0) == "ok"
+    for s in range(1, 8):
+        assert B.gptq_status_string(s) not in ("", "unknown status")
+    assert B.gptq_status_string(99) == "unknown status"
+    assert isinstance(B.gptq_launch_count(), int)
+
+
+def test_workspace_bytes(lib):
+    w = B.gptq_workspace_bytes(4096, 4096, 128)
+    assert w >= 3 * 4096 * 4096 * 4          # factorisation buffers
+    assert w >= 4096 * 4096 * 5              # working weights + codes
+    assert B.gptq_workspace_bytes(4096, 0, 128) == 0
+    assert B.gptq_workspace_bytes(4096, -5, 128) == 0
+
+
+def _call(lib, name, *args):
+    return getattr(lib, name)(*args)
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: validation fails first
+    # H NULL
+    assert lib.gptq_hessian_accumulate(None, fake, 16, 64, None) == 1
+    # d_in not a multiple of 8
+    assert lib.gptq_hessian_accumulate(fake, fake, 16, 60, None) == 1
+    # negative tokens
+    assert lib.gptq_hessian_accumulate(fake, fake, -1, 64, None) == 1
+    # misaligned
+    assert lib.gptq_hessian_accumulate(P((1 << 20) + 4), fake, 16, 64, None) == 1
+    # prepare: negative damp, null outputs, missing workspace
+    assert lib.gptq_prepare(fake, 64, ctypes.c_float(-1.0), 0, fake, fake, fake, 1 << 30, None) == 1
+    assert lib.gptq_prepare(fake, 64, ctypes.c_float(0.01), 0, None, fake, fake, 1 << 30, None) == 1
+    assert lib.gptq_prepare(fake, 64, ctypes.c_float(0.01), 0, fake, fake, None, 0, None) == 6
+    assert lib.gptq_prepare(fake, 64, ctypes.c_float(0.01), 0, fake, fake, fake, 10, None) == 6
+
+    def q(bits=4, gs=128, block=128, d_in=256, packed=None, ws=fake, ws_bytes=1 << 40):
+        return lib.gptq_quantize(fake, fake, None, 64, d_in, bits, gs, block, None, fake, fake,
+                                 packed, None, None, ws, ws_bytes, None)
+    assert q(bits=0) == 1
+    assert q(bits=9) == 1
+    assert q(gs=100) == 1            # does not divide d_in
+    assert q(gs=0) == 1
+    assert q(block=12) == 1          # not a multiple of 8
+    assert q(block=256) == 1         # above the fused kernel's width
+    assert q(gs=64, block=96) == 1   # neither divides the other
+    assert q(bits=5, packed=fake) == 1
+    assert q(d_in=100) == 1          # not a multiple of 8
+    assert q(ws=None) == 6
+    assert q(ws_bytes=100) == 6
+    assert lib.gptq_bf16_to_f32(None, fake, 10, None) == 1
+    assert lib.gptq_hessian_accumulate_host(fake, fake, 16, 64, None, 8, None) == 1
+    assert lib.gptq_hessian_accumulate_host(fake, fake, 16, 64, fake, 0, None) == 1

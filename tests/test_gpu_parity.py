@@ -1,0 +1,262 @@
+"""GPU path vs the float64 checker, element by element, on seeded inputs.
+
+Staged as in the design notes: the Hessian against the checker's H from the
+same bf16 bytes; the factor U against the checker's OBS elimination of the
+GPU's own H; the column loop against the checker given the GPU's U and order;
+and the whole path from scratch against the checker's own H, U and order.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_accumulate_b200 import binding as B
+from post_weight_quantization_accumulate_b200 import synth
+from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
+
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _x_dev(xb: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(xb.view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+def _gpu_hessian(xb: np.ndarray) -> np.ndarray:
+    d = xb.shape[1]
+    H = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    B.gptq_hessian_accumulate(H, _x_dev(xb))
+    torch.cuda.synchronize()
+    return H.cpu().numpy()
+
+
+def _rand_x(seed, n, d, outliers=0):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((n, d)).astype(np.float32)
+    if outliers:
+        idx = g.choice(d, outliers, replace=False)
+        x[:, idx] *= 20
+    return synth.f32_to_bf16_bits(x)
+
+
+# --------------------------------------------------------------------- Hessian
+
+@pytest.mark.parametrize("n,d", [(2048, 256), (1000, 200), (4097, 392), (63, 8), (64, 64),
+                                 (8192 + 77, 520), (20000, 1024)])
+def test_hessian_matches_checker(n, d):
+    xb = _rand_x(n * 7 + d, n, d, outliers=min(4, d // 8))
+    Hg = _gpu_hessian(xb)
+    Hr = oracle.hessian(xb)
+    assert np.array_equal(Hg, Hg.T), "H must be bitwise symmetric"
+    assert P.rel_fro(Hg, Hr) <= P.H_RTOL
+    # every entry, relative to the scale of its row/column
+    scale = np.sqrt(np.outer(np.diag(Hr), np.diag(Hr))) + 1e-30
+    assert np.max(np.abs(Hg - Hr) / scale) < 1e-5
+
+
+def test_hessian_tiny_workload_and_chunked_accumulation():
+    spec = synth.WORKLOADS["tiny"]
+    xb = synth.x_bf16(spec)
+    Hr = oracle.hessian(xb)
+    H = torch.zeros(256, 256, dtype=torch.float32, device=DEV)
+    for a, b in [(0, 700), (700, 701), (701, 2048)]:
+        B.gptq_hessian_accumulate(H, _x_dev(xb[a:b]))
+    torch.cuda.synchronize()
+    Hg = H.cpu().numpy()
+    assert np.array_equal(Hg, Hg.T)
+    assert P.rel_fro(Hg, Hr) <= P.H_RTOL
+
+
+def test_hessian_host_streaming_matches_device():
+    xb = _rand_x(5, 5000, 256, 4)
+    Hd = _gpu_hessian(xb)
+    H = torch.zeros(256, 256, dtype=torch.float32, device=DEV)
+    Xh = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    staging = torch.empty(2 * 1024 * 256, dtype=torch.bfloat16, device=DEV)
+    B.gptq_hessian_accumulate_host(H, Xh, staging, 1024)
+    torch.cuda.synchronize()
+    Hh = H.cpu().numpy()
+    assert np.array_equal(Hh, Hh.T)
+    assert P.rel_fro(Hh, Hd) <= 1e-6
+    assert P.rel_fro(Hh, oracle.hessian(xb)) <= P.H_RTOL
+
+
+def test_hessian_zero_tokens_is_noop():
+    H = torch.ones(64, 64, dtype=torch.float32, device=DEV)
+    X = torch.empty(0, 64, dtype=torch.bfloat16, device=DEV)
+    B.gptq_hessian_accumulate(H, X)
+    torch.cuda.synchronize()
+    assert torch.all(H == 1)
+
+
+# ---------------------------------------------------------------- factorisation
+
+def _gpu_prepare(Hg: np.ndarray, act_order: bool, damp=0.01):
+    d = Hg.shape[0]
+    H = torch.from_numpy(Hg).to(DEV)
+    U = torch.empty(d, d, dtype=torch.float32, device=DEV)
+    perm = torch.empty(d, dtype=torch.int32, device=DEV)
+    ws = B.workspace(1, d, 128)
+    B.gptq_prepare(H, damp, act_order, perm, U, ws)
+    torch.cuda.synchronize()
+    return perm.cpu().numpy(), U.cpu().numpy()
+
+
+@pytest.mark.parametrize("d", [8, 64, 200, 256, 392, 1000, 1024])
+@pytest.mark.parametrize("act_order", [False, True])
+def test_prepare_matches_checker(d, act_order):
+    xb = _rand_x(d + 3, max(4 * d, 512), d, outliers=max(1, d // 64))
+    Hg = _gpu_hessian(xb)
+    perm_g, Ug = _gpu_prepare(Hg, act_order)
+    H64 = Hg.astype(np.float64)
+    perm_r, Ur, Hp, _ = oracle.prepare(H64, 0.01, act_order)
+    np.testing.assert_array_equal(perm_g, perm_r)
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert P.rel_fro(Ug, Ur) <= P.U_RTOL
+    # U^T U H_d = I (property at any size)
+    I = Ug.astype(np.float64).T @ Ug.astype(np.float64) @ Hp
+    assert np.abs(I - np.eye(d)).max() < 1e-3
+
+
+def test_prepare_rejects_singular_and_nonfinite():
+    d = 64
+    with pytest.raises(B.GptqError) as e:
+        _gpu_prepare(np.zeros((d, d), np.float32), False)
+    assert e.value.status == 2
+    H = np.eye(d, dtype=np.float32)
+    H[3, 3] = np.nan
+    with pytest.raises(B.GptqError) as e:
+        _gpu_prepare(H, False)
+    assert e.value.status == 3
+    # indefinite even after damping
+    H = np.eye(d, dtype=np.float32)
+    H[0, 1] = H[1, 0] = 5.0
+    with pytest.raises(B.GptqError) as e:
+        _gpu_prepare(H, False, damp=0.0)
+    assert e.value.status == 2
+
+
+# ------------------------------------------------------------------ column loop
+
+def _gpu_quantize(W: np.ndarray, Ug: np.ndarray, perm: np.ndarray | None, bits, gs, block):
+    d_out, d_in = W.shape
+    Wt = torch.from_numpy(W.astype(np.float32)).to(DEV)
+    U = torch.from_numpy(Ug).to(DEV)
+    pm = torch.from_numpy(perm.astype(np.int32)).to(DEV) if perm is not None else None
+    ng = d_in // gs if gs > 0 else 1
+    scales = torch.empty(d_out, ng, dtype=torch.float32, device=DEV)
+    zeros = torch.empty_like(scales)
+    codes = torch.empty(d_out, d_in, dtype=torch.uint8, device=DEV)
+    packed = torch.empty(d_out, d_in // 2, dtype=torch.uint8, device=DEV) if bits <= 4 else None
+    g_idx = torch.empty(d_in, dtype=torch.int32, device=DEV)
+    err = torch.empty(d_out, dtype=torch.float32, device=DEV)
+    ws = B.workspace(d_out, d_in, block)
+    B.gptq_quantize(Wt, U, pm, bits, gs, block, scales, zeros, ws, codes=codes,
+                    packed_int4=packed, g_idx=g_idx, err_sq=err)
+    torch.cuda.synchronize()
+    return dict(W_hat=Wt.cpu().numpy(), scales=scales.cpu().numpy(), zeros=zeros.cpu().numpy(),
+                codes=codes.cpu().numpy(), packed=None if packed is None else packed.cpu().numpy(),
+                g_idx=g_idx.cpu().numpy(), err_sq=err.cpu().numpy())
+
+
+def _staged_check(W, xb, bits, gs, block, act_order, where):
+    """GPU column loop vs checker given the GPU's own H, U and order."""
+    Hg = _gpu_hessian(xb)
+    perm, Ug = _gpu_prepare(Hg, act_order)
+    g = _gpu_quantize(W, Ug, perm if act_order else None, bits, gs, block)
+    r = oracle.quantize(W.astype(np.float64), Ug.astype(np.float64), perm, bits, gs, block)
+    P.check_codes(g["codes"], r["codes"], where)
+    P.check_scales_zeros(g["scales"], g["zeros"], r["scales"], r["zeros"],
+                         g["codes"][:, perm], r["codes_perm"], gs, where)
+    H64 = Hg.astype(np.float64)
+    mse_g = oracle.output_mse(W, g["W_hat"], H64, xb.shape[0])
+    mse_r = oracle.output_mse(W, r["W_hat"], H64, xb.shape[0])
+    P.check_mse(mse_g, mse_r, where)
+    # W^ is exactly s (q - z) of the GPU's own codes and grid
+    gi = g["g_idx"]
+    np.testing.assert_array_equal(gi, oracle.g_idx(perm, gs))
+    s = g["scales"][:, gi] if gs > 0 else np.repeat(g["scales"], W.shape[1], axis=1)
+    z = g["zeros"][:, gi] if gs > 0 else np.repeat(g["zeros"], W.shape[1], axis=1)
+    deq = s * (g["codes"].astype(np.float32) - z)
+    np.testing.assert_array_equal(g["W_hat"], deq)
+    if g["packed"] is not None:
+        np.testing.assert_array_equal(g["packed"], oracle.pack_int4(g["codes"]))
+    # |e|^2 per row equals (w - w^) H_d (w - w^)^T in processing order
+    Hd, _ = oracle.damp(H64, 0.01)
+    Hp = Hd[np.ix_(perm, perm)]
+    dW = (W - g["W_hat"].astype(np.float64))[:, perm]
+    lhs = np.einsum("ij,jk,ik->i", dW, Hp, dW)
+    np.testing.assert_allclose(g["err_sq"], lhs, rtol=2e-3, atol=1e-12 * lhs.max())
+    return g, r
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("gs", [-1, 32, 64, 128, 256])
+@pytest.mark.parametrize("act_order", [False, True])
+def test_quantize_matches_checker(bits, gs, act_order):
+    d_out, d_in, n = 96, 512, 2048
+    W, xb = synth.random_layer(bits * 31 + gs, d_out, d_in, n, correlated=True)
+    _staged_check(W, xb, bits, gs, 128, act_order, f"b{bits} g{gs} ao{act_order}")
+
+
+@pytest.mark.parametrize("d_out,d_in,gs,block", [(33, 200, 8, 64), (1, 392, 56, 8), (130, 264, 24, 24),
+                                                 (257, 136, -1, 128), (64, 1000, 40, 40),
+                                                 (40, 8, -1, 8)])
+def test_quantize_ragged_shapes(d_out, d_in, gs, block):
+    W, xb = synth.random_layer(d_out + d_in, d_out, d_in, max(512, 2 * d_in), correlated=True)
+    _staged_check(W, xb, 4, gs, block, True, f"{d_out}x{d_in} g{gs} B{block}")
+
+
+def test_tiny_workload_end_to_end_from_scratch():
+    """S4: the checker computes its own H, U and order."""
+    spec = synth.WORKLOADS["tiny"]
+    xb = synth.x_bf16(spec)
+    W = synth.weight_f32(spec)
+    q = LayerQuantizer(spec.d_out, spec.d_in, spec.bits, spec.group_size, spec.block_size,
+                       spec.damp, spec.act_order, keep_err=True)
+    q.reset()
+    q.add_batch(_x_dev(xb))
+    res = q.run(torch.from_numpy(W).to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle.layer(W.astype(np.float64), xb, spec.bits, spec.group_size)
+    mse_g = oracle.output_mse(W, res.W_hat.cpu().numpy(), ref["H"], spec.n_tokens)
+    P.check_mse(mse_g, ref["mse"], "tiny")
+    codes = res.codes.cpu().numpy()
+    rate = 1.0 - np.mean(codes != ref["codes"])
+    assert rate >= P.CODE_MATCH
+    rtn = oracle.rtn(W.astype(np.float64), spec.bits, spec.group_size)
+    assert mse_g < oracle.output_mse(W, rtn["W_hat"], ref["H"], spec.n_tokens)
+
+
+def test_quantize_is_deterministic():
+    W, xb = synth.random_layer(77, 64, 256, 1024)
+    Hg = _gpu_hessian(xb)
+    perm, Ug = _gpu_prepare(Hg, True)
+    a = _gpu_quantize(W, Ug, perm, 4, 64, 64)
+    b = _gpu_quantize(W, Ug, perm, 4, 64, 64)
+    for k in ("codes", "scales", "zeros", "W_hat", "packed"):
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_diagonal_hessian_gives_rtn_on_gpu():
+    """With a diagonal H no error is carried: codes equal round-to-nearest."""
+    d_out, d_in = 64, 256
+    g = np.random.default_rng(3)
+    W = (g.standard_normal((d_out, d_in)) * 0.02).astype(np.float32)
+    H = np.diag(g.uniform(0.5, 5.0, d_in)).astype(np.float32)
+    perm, Ug = _gpu_prepare(H, False)
+    gq = _gpu_quantize(W, Ug, None, 4, 64, 128)
+    rt = oracle.rtn(W.astype(np.float64), 4, 64)
+    np.testing.assert_array_equal(gq["codes"], rt["codes"])
+    np.testing.assert_array_equal(gq["scales"], rt["scales"])
+    np.testing.assert_array_equal(gq["zeros"], rt["zeros"])
+
+
+def test_launch_count_increases():
+    before = B.gptq_launch_count()
+    _gpu_hessian(_rand_x(1, 128, 64))
+    assert B.gptq_launch_count() >= before + 2
+    assert B.gptq_device_status() == 0
