@@ -15,15 +15,23 @@
 //    dimension of X, so both are MN-major; TMA brings 64-token x 64-column
 //    boxes with 128-byte swizzle, which is the canonical MN-major SW128
 //    layout tcgen05.mma reads directly.
-//  * Work units = (tile, token split of kSplitTokens).  A persistent grid of
-//    one CTA per SM walks the units split-major, so concurrently running
-//    units read the same token rows of X (L2 reuse).  Each unit accumulates
-//    in TMEM (fp32) and is flushed with fp32 red.add into H, which bounds the
-//    length of any single fp32 accumulation chain.
-//  * Warp roles per CTA (192 threads): warp 0 = TMA producer, warp 1 = MMA
-//    issuer + TMEM owner, warps 2-5 = epilogue (TMEM lanes 0-127).  A 4-stage
-//    shared-memory ring (48 KB per stage) and two TMEM accumulators (2 x 256
-//    columns) let the epilogue of one unit overlap the MMAs of the next.
+//  * Work units = (tile, token span of kSpanTokens).  A persistent grid of
+//    one CTA per SM walks the units span-major, so concurrently running
+//    units read the same token rows of X (L2 reuse).
+//  * Accumulation precision: the tensor core adds each MMA's result into the
+//    fp32 TMEM accumulator with a rounding that is biased for long chains
+//    (measured: sums of squares come out ~0.25 ulp low per MMA).  So a TMEM
+//    chain covers only kChainTokens tokens (32 MMAs); the epilogue promotes
+//    each chain into fp32 registers with round-to-nearest adds, and flushes
+//    the span's sum into H with one fp32 red.add per element.
+//  * Warp roles per CTA (384 threads, three warpgroups): warp 0 = TMA
+//    producer, warp 1 = MMA issuer + TMEM owner (warpgroup 0 gives its
+//    registers up to 56); warps 4-11 = epilogue (raised to 224 registers);
+//    warps w and w+4 share TMEM lanes 32*(w%4)..+31 and split the 256 columns
+//    in halves, 128 fp32 registers of running sum each.  The launch budget
+//    384 x 168 equals 128 x 56 + 256 x 224.  A 4-stage shared-memory ring (48 KB per
+//    stage) and two TMEM chain buffers (2 x 256 columns) let the promotion of
+//    one chain overlap the MMAs of the next.
 //  * Every mbarrier wait is bounded; a time-out records GPTQ_ERR_TIMEOUT,
 //    releases the other roles, and the CTA still frees its TMEM.
 #include "common.cuh"
@@ -43,9 +51,11 @@ constexpr int kBoxBytes = kBK * kBoxCols * 2;           // 8 KB
 constexpr int kABytes = kBoxBytes * (kBM / kBoxCols);   // 16 KB
 constexpr int kBBytes = kBoxBytes * (kBN / kBoxCols);   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;          // 48 KB
-constexpr int kThreads = 192;
-constexpr int kTmemCols = 512;    // two 256-column fp32 accumulators
-constexpr int kSplitTokens = 8192;
+constexpr int kThreads = 384;
+constexpr int kEpiWarps = 8;
+constexpr int kTmemCols = 512;    // two 256-column fp32 chain buffers
+constexpr int kChainTokens = 512; // tokens per TMEM accumulation chain
+constexpr int kSpanTokens = 16384;  // tokens per work unit (one flush into H)
 constexpr uint32_t kIdesc = idesc_f32acc(1 /*bf16*/, 1, 1, kBM, kBN);
 
 struct alignas(1024) HessSmem {
@@ -94,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&S.tfull[b], 1);
-            mbar_init(&S.tempty[b], 4);
+            mbar_init(&S.tempty[b], kEpiWarps);
         }
         S.abort = 0;
         fence_mbar_init();
@@ -111,18 +121,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort = &S.abort;
     const int n_units = n_tiles * n_split;
 
-    if (warp == 0) {
-        if (lane == 0) {
+    if (warp < 4) {
+        regs_dealloc<56>();
+        if (warp == 0 && lane == 0) {
             uint32_t it = 0;
             for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
                 int ti, tj;
                 tile_coords(u % n_tiles, n_ti, n_tj, ti, tj);
-                const int t0 = (u / n_tiles) * kSplitTokens;
-                const int t1 = min(n_tokens, t0 + kSplitTokens);
-                for (int t = t0; t < t1; t += kBK, ++it) {
+                const int t0 = (u / n_tiles) * kSpanTokens;
+                const int t1 = min(n_tokens, t0 + kSpanTokens);
+                bool ok = true;
+                for (int t = t0; t < t1 && ok; t += kBK, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) break;
+                    if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&S.full[s], kStageBytes);
                     uint8_t* a = S.stage[s];
                     uint8_t* b = a + kABytes;
@@ -133,84 +145,100 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int m = 0; m < kBN / kBoxCols; ++m)
                         tma_load_2d(b + m * kBoxBytes, &tmap, &S.full[s], tj * kBN + m * kBoxCols, t);
                 }
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0) {
-            uint32_t it = 0, uc = 0;
-            for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++uc) {
-                const int b = uc & 1;
-                const uint32_t uph = (uc >> 1) & 1;
-                if (!mbar_wait_bounded(&S.tempty[b], uph ^ 1, abort, status)) break;
-                tc_fence_after();
-                const uint32_t dt = tbase + b * kBN;
-                const int t0 = (u / n_tiles) * kSplitTokens;
-                const int t1 = min(n_tokens, t0 + kSplitTokens);
-                const int nk = (t1 - t0 + kBK - 1) / kBK;
-                bool ok = true;
-                for (int kk = 0; kk < nk; ++kk, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait_bounded(&S.full[s], ph, abort, status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(S.stage[s]);
-                    const uint32_t b0 = a0 + kABytes;
-#pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        // 16 tokens = two 8-row swizzle groups = 2048 bytes
-                        const uint64_t ad = sdesc_sw128(a0 + k * 2048, kBoxBytes, 1024);
-                        const uint64_t bd = sdesc_sw128(b0 + k * 2048, kBoxBytes, 1024);
-                        umma_f16(dt, ad, bd, kIdesc, (kk | k) != 0);
-                    }
-                    umma_commit(&S.empty[s]);
-                }
                 if (!ok) break;
-                umma_commit(&S.tfull[b]);
+            }
+        } else if (warp == 1 && lane == 0) {
+            uint32_t it = 0, ch = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok && !*abort; u += gridDim.x) {
+                const int t0 = (u / n_tiles) * kSpanTokens;
+                const int t1 = min(n_tokens, t0 + kSpanTokens);
+                for (int c0 = t0; c0 < t1 && ok; c0 += kChainTokens, ++ch) {
+                    const int b = ch & 1;
+                    const uint32_t cph = (ch >> 1) & 1;
+                    if (!mbar_wait_bounded(&S.tempty[b], cph ^ 1, abort, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t dt = tbase + b * kBN;
+                    const int nk = (min(t1, c0 + kChainTokens) - c0 + kBK - 1) / kBK;
+                    for (int kk = 0; kk < nk; ++kk, ++it) {
+                        const int s = it % kStages;
+                        const uint32_t ph = (it / kStages) & 1;
+                        if (!mbar_wait_bounded(&S.full[s], ph, abort, status)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(S.stage[s]);
+                        const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+                        for (int k = 0; k < kBK / 16; ++k) {
+                            // 16 tokens = two 8-row swizzle groups = 2048 bytes
+                            const uint64_t ad = sdesc_sw128(a0 + k * 2048, kBoxBytes, 1024);
+                            const uint64_t bd = sdesc_sw128(b0 + k * 2048, kBoxBytes, 1024);
+                            umma_f16(dt, ad, bd, kIdesc, (kk | k) != 0);
+                        }
+                        umma_commit(&S.empty[s]);
+                    }
+                    if (ok) umma_commit(&S.tfull[b]);
+                }
             }
         }
         __syncwarp();
     } else {
-        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
+        regs_alloc<224>();
+        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31, column half h
         const int q = warp & 3;
+        const int h = (warp - 4) / 4;
         const int row_in_tile = q * 32 + lane;
-        uint32_t uc = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uc) {
-            const int b = uc & 1;
-            const uint32_t uph = (uc >> 1) & 1;
-            // every lane waits, so the warp stays converged for tcgen05.ld
-            const bool ok = mbar_wait_bounded(&S.tfull[b], uph, abort, status);
-            __syncwarp();
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        uint32_t ch = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            const int t0 = (u / n_tiles) * kSpanTokens;
+            const int t1 = min(n_tokens, t0 + kSpanTokens);
+            float acc[kBN / 2];
+#pragma unroll
+            for (int i = 0; i < kBN / 2; ++i) acc[i] = 0.f;
+            for (int c0 = t0; c0 < t1; c0 += kChainTokens, ++ch) {
+                const int b = ch & 1;
+                const uint32_t cph = (ch >> 1) & 1;
+                // every lane waits, then the warp reconverges for tcgen05.ld
+                const bool got = mbar_wait_bounded(&S.tfull[b], cph, abort, status);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tbase + lane_addr + b * kBN + h * (kBN / 2);
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
+                    float v[16];
+                    tmem_ld_32x32b_x16(taddr + c * 16, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[c * 16 + i] += v[i];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.tempty[b]);
+            }
+            if (!ok) break;
             int ti, tj;
             tile_coords(u % n_tiles, n_ti, n_tj, ti, tj);
             const int row = ti * kBM + row_in_tile;
-            const uint32_t taddr = tbase + (static_cast<uint32_t>(q * 32) << 16) + b * kBN;
-#pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                float v[32];
-                tmem_ld_32x32b_x32(taddr + c * 32, v);
-                tmem_ld_wait();
-                const int col0 = tj * kBN + c * 32;
+#pragma unroll
+            for (int c = 0; c < kBN / 64; ++c) {
+                const int col0 = tj * kBN + h * (kBN / 2) + c * 32;
                 if (row < d && col0 < d && col0 + 31 >= row) {
                     float* dst = H + static_cast<int64_t>(row) * d + col0;
                     if (col0 + 32 <= d) {
 #pragma unroll
                         for (int m = 0; m < 8; ++m)
                             atomicAdd(reinterpret_cast<float4*>(dst) + m,
-                                      make_float4(2.f * v[4 * m], 2.f * v[4 * m + 1],
-                                                  2.f * v[4 * m + 2], 2.f * v[4 * m + 3]));
+                                      make_float4(2.f * acc[c * 32 + 4 * m], 2.f * acc[c * 32 + 4 * m + 1],
+                                                  2.f * acc[c * 32 + 4 * m + 2], 2.f * acc[c * 32 + 4 * m + 3]));
                     } else {
 #pragma unroll
                         for (int m = 0; m < 32; ++m)
-                            if (m < d - col0) atomicAdd(dst + m, 2.f * v[m]);
+                            if (m < d - col0) atomicAdd(dst + m, 2.f * acc[c * 32 + m]);
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.tempty[b]);
         }
     }
 
@@ -301,7 +329,7 @@ int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
     const int n_tj = static_cast<int>((d + kBN - 1) / kBN);
     int n_tiles = 0;
     for (int i = 0; i < n_ti; ++i) n_tiles += n_tj - (i >> 1);
-    const int n_split = static_cast<int>((n_rows + kSplitTokens - 1) / kSplitTokens);
+    const int n_split = static_cast<int>((n_rows + kSpanTokens - 1) / kSpanTokens);
     const int64_t units = static_cast<int64_t>(n_tiles) * n_split;
     const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
     hessian_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(

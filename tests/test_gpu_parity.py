@@ -168,7 +168,7 @@ def _staged_check(W, xb, bits, gs, block, act_order, where):
     perm, Ug = _gpu_prepare(Hg, act_order)
     g = _gpu_quantize(W, Ug, perm if act_order else None, bits, gs, block)
     r = oracle.quantize(W.astype(np.float64), Ug.astype(np.float64), perm, bits, gs, block)
-    P.check_codes(g["codes"], r["codes"], where)
+    P.check_codes(g["codes"], r["codes"], where, bits, perm)
     P.check_scales_zeros(g["scales"], g["zeros"], r["scales"], r["zeros"],
                          g["codes"][:, perm], r["codes_perm"], gs, where)
     H64 = Hg.astype(np.float64)
