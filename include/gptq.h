@@ -170,6 +170,41 @@ int gptq_quantize(float *W, const float *Hinv_chol, const int32_t *perm, int64_t
                   float *scales, float *zeros, uint8_t *packed_int4, int32_t *g_idx,
                   float *err_sq, void *workspace, size_t ws_bytes, void *stream);
 
+/* Size of the fixed device array that gptq_quantize_static_scratch works in:
+ * 96 MiB.  Every GPU on which the library's device code is loaded holds it
+ * from then until the process exits. */
+#define GPTQ_STATIC_SCRATCH_BYTES ((size_t)96 << 20)
+
+/*
+ * gptq_quantize with no workspace argument, for callers that cannot allocate
+ * device memory: a plugin inside another engine that is handed only input and
+ * output pointers and has no allocator to ask; a serving loop that must not
+ * pay cudaMalloc's implicit device-wide synchronisation; a process that has
+ * reserved the GPU's memory up front for its own pool.  The paper has no
+ * counterpart to this call; it exists only for such callers.
+ *
+ * Arguments, outputs and results are those of gptq_quantize.  The scratch is
+ * a fixed array inside the library (GPTQ_STATIC_SCRATCH_BYTES), so the call
+ * allocates nothing.  Limits and rules:
+ *   - A layer whose working set exceeds the array (about 5 bytes per weight
+ *     plus 512 bytes per output row: 4096 x 4096 needs about 82 MiB and fits,
+ *     4096 x 11008 does not) is refused with GPTQ_ERR_WORKSPACE before the
+ *     device is touched.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (a one-time set-up); make that first call before any
+ *     stream capture begins.
+ *   - All calls share the one array, and it keeps whatever the last call left
+ *     in it.  Nothing in it needs to start at zero (each call writes every byte
+ *     it later reads), but two calls whose work overlaps on the GPU (different
+ *     streams, or different host threads) race on it: order them on one stream
+ *     or otherwise make sure one finishes before the next starts.
+ */
+int gptq_quantize_static_scratch(float *W, const float *Hinv_chol, const int32_t *perm,
+                                 int64_t d_out, int64_t d_in, int bits, int group_size,
+                                 int block_size, uint8_t *codes, float *scales, float *zeros,
+                                 uint8_t *packed_int4, int32_t *g_idx, float *err_sq,
+                                 void *stream);
+
 /* dst[i] = (float) bf16 src[i] (exact widening), n >= 0 elements. */
 int gptq_bf16_to_f32(float *dst, const uint16_t *src, int64_t n, void *stream);
 

@@ -35,6 +35,7 @@ SIGNATURES = [
     ("gptq_hessian_accumulate_host", _I, [_P, _P, _I64, _I64, _P, _I64, _P]),
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    ("gptq_quantize_static_scratch", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     ("gptq_bf16_to_f32", _I, [_P, _P, _I64, _P]),
 ]
 
@@ -175,6 +176,22 @@ def gptq_quantize(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor |
                                group_size, block_size, _ptr(codes), _ptr(scales), _ptr(zeros),
                                _ptr(packed_int4), _ptr(g_idx), _ptr(err_sq), _ptr(ws),
                                ws.numel(), _stream(W, stream)))
+
+
+def gptq_quantize_static_scratch(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor | None,
+                                 bits: int, group_size: int, block_size: int, scales: torch.Tensor,
+                                 zeros: torch.Tensor, codes: torch.Tensor | None = None,
+                                 packed_int4: torch.Tensor | None = None,
+                                 g_idx: torch.Tensor | None = None,
+                                 err_sq: torch.Tensor | None = None, stream=None):
+    """gptq_quantize using the library's fixed scratch array (no workspace)."""
+    _need(W, torch.float32, "W")
+    d_out, d_in = W.shape
+    _check("gptq_quantize_static_scratch",
+           lib().gptq_quantize_static_scratch(_ptr(W), _ptr(Hinv_chol), _ptr(perm), d_out, d_in,
+                                              bits, group_size, block_size, _ptr(codes),
+                                              _ptr(scales), _ptr(zeros), _ptr(packed_int4),
+                                              _ptr(g_idx), _ptr(err_sq), _stream(W, stream)))
 
 
 def gptq_bf16_to_f32(dst: torch.Tensor, src: torch.Tensor, stream=None):
