@@ -1,0 +1,72 @@
+"""Runs one library call on a synthetic layer, a few times, for profiling.
+
+    python -m post_weight_quantization_accumulate_b200.kernel_case \
+        --call hessian|prepare|quantize|layer --workload q_proj_4096 [--tokens N] [--reps R]
+
+The inputs follow the workload's recipe (see synth.py) with `--tokens`
+overriding the calibration size, so a profiler can capture a launch on a case
+that is larger than L2 but small in device memory.  Prints the mean CUDA-event
+time of the call.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import numpy as np
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+from post_weight_quantization_accumulate_b200 import binding as B  # noqa: E402
+from post_weight_quantization_accumulate_b200 import synth  # noqa: E402
+from post_weight_quantization_accumulate_b200.layer import LayerQuantizer  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--call", default="hessian", choices=["hessian", "prepare", "quantize", "layer"])
+    ap.add_argument("--workload", default="q_proj_4096")
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args()
+    spec = synth.WORKLOADS[a.workload]
+    if a.tokens:
+        spec = synth.scaled(spec, n_tokens=a.tokens)
+    dev = torch.device("cuda", 0)
+    X = torch.from_numpy(synth.x_bf16(spec).view(np.int16)).to(dev).view(torch.bfloat16)
+    W = torch.from_numpy(synth.weight_f32(spec)).to(dev)
+    q = LayerQuantizer(spec.d_out, spec.d_in, spec.bits, spec.group_size, spec.block_size,
+                       spec.damp, spec.act_order, device=dev)
+    q.reset()
+    q.add_batch(X)
+    q.prepare()
+
+    def once():
+        if a.call == "hessian":
+            q.reset()
+            q.add_batch(X)
+        elif a.call == "prepare":
+            q.prepare()
+        elif a.call == "quantize":
+            q.quantize(W)
+        else:
+            q.reset()
+            q.add_batch(X)
+            q.run(W)
+
+    once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    print(f"{a.call} {spec.name} tokens={spec.n_tokens}: {e0.elapsed_time(e1) / a.reps:.3f} ms/call, "
+          f"status {B.gptq_device_status()}")
+
+
+if __name__ == "__main__":
+    main()
