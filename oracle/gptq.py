@@ -70,7 +70,7 @@ def _load():
             lib.orc_hessian_block.argtypes = [P, P, I64, I64, P, I64, P, I64]
             lib.orc_inverse_gauss_jordan.argtypes = [P, I64]
             lib.orc_obs_upper.argtypes = [P, I64, P]
-            lib.orc_gptq_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64, I64, P, P, P, P]
+            lib.orc_gptq_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64, I64, P, P, P, P, P, P]
             for f in (lib.orc_hessian_accumulate, lib.orc_hessian_block,
                       lib.orc_inverse_gauss_jordan, lib.orc_obs_upper, lib.orc_gptq_rows):
                 f.restype = ctypes.c_int
@@ -165,9 +165,12 @@ def prepare(H: np.ndarray, lam: float = 0.01, act_order: bool = False):
 
 # --- 5. the column loop ------------------------------------------------------
 
-def gptq_rows(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, block: int = 0):
+def gptq_rows(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, block: int = 0,
+              raw: dict | None = None):
     """Column loop on W already in processing order.  Returns
-    (W_hat, codes, scales, zeros, E) all in processing order."""
+    (W_hat, codes, scales, zeros, E) all in processing order.  With `raw` (a
+    dict), also fills raw["qraw"] = w / s and raw["zraw"] = -min / s before
+    rounding (how close each integer decision was to a tie)."""
     W = np.array(Wp, dtype=np.float64, copy=True, order="C")
     d_out, d_in = W.shape
     U = np.ascontiguousarray(U, dtype=np.float64)
@@ -177,8 +180,15 @@ def gptq_rows(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, block: 
     scales = np.empty((d_out, ng), dtype=np.float32)
     zeros = np.empty((d_out, ng), dtype=np.float32)
     E = np.empty((d_out, d_in), dtype=np.float64)
+    qraw = zraw = None
+    if raw is not None:
+        qraw = np.empty((d_out, d_in), dtype=np.float32)
+        zraw = np.empty((d_out, ng), dtype=np.float32)
+        raw["qraw"], raw["zraw"] = qraw, zraw
     _check(_load().orc_gptq_rows(_ptr(W), _ptr(U), d_out, d_in, bits, group_size, block,
-                                 _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(E)), "gptq_rows")
+                                 _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(E),
+                                 _ptr(qraw) if qraw is not None else None,
+                                 _ptr(zraw) if zraw is not None else None), "gptq_rows")
     return W, codes, scales, zeros, E
 
 
@@ -210,13 +220,15 @@ def quantize(W: np.ndarray, U: np.ndarray, perm: np.ndarray | None, bits: int,
     if perm is None:
         perm = np.arange(d_in, dtype=np.int32)
     perm = np.asarray(perm, dtype=np.int64)
-    What_p, codes_p, scales, zeros, E_p = gptq_rows(W[:, perm], U, bits, group_size, block)
+    raw = {}
+    What_p, codes_p, scales, zeros, E_p = gptq_rows(W[:, perm], U, bits, group_size, block, raw)
     codes = np.empty_like(codes_p)
     codes[:, perm] = codes_p
     What = np.empty_like(What_p)
     What[:, perm] = What_p
     out = dict(codes=codes, scales=scales, zeros=zeros, W_hat=What, E_perm=E_p,
-               codes_perm=codes_p, g_idx=g_idx(perm, group_size), perm=perm.astype(np.int32))
+               codes_perm=codes_p, g_idx=g_idx(perm, group_size), perm=perm.astype(np.int32),
+               qraw_perm=raw["qraw"], zraw=raw["zraw"])
     if bits <= 4 and d_in % 2 == 0:
         out["packed"] = pack_int4(codes)
     return out

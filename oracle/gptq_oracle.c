@@ -171,7 +171,7 @@ int orc_obs_upper(const double *Hinv, int64_t d, double *U)
 
 /* Grid of the asymmetric min/max quantizer on the values v[0..n): the range
  * always contains 0; an all-zero range becomes [-1, 1].  Decided in binary32. */
-static void qgrid(const double *v, int64_t n, int maxq, float *s_out, float *z_out)
+static void qgrid(const double *v, int64_t n, int maxq, float *s_out, float *z_out, float *zraw)
 {
     float xmin = 0.0f, xmax = 0.0f;
     for (int64_t k = 0; k < n; k++) {
@@ -181,14 +181,18 @@ static void qgrid(const double *v, int64_t n, int maxq, float *s_out, float *z_o
     }
     if (xmin == xmax) { xmin = -1.0f; xmax = 1.0f; }
     float s = (xmax - xmin) / (float)maxq;
-    float z = rintf(-xmin / s);
+    float zr = -xmin / s;
+    float z = rintf(zr);
     *s_out = s;
     *z_out = z;
+    if (zraw) *zraw = zr;
 }
 
-static int qcode(double w, float s, float z, int maxq)
+static int qcode(double w, float s, float z, int maxq, float *qraw)
 {
-    float q = rintf((float)w / s) + z;
+    float r = (float)w / s;
+    if (qraw) *qraw = r;
+    float q = rintf(r) + z;
     if (q < 0.0f) q = 0.0f;
     if (q > (float)maxq) q = (float)maxq;
     return (int)q;
@@ -209,10 +213,13 @@ static int qcode(double w, float s, float z, int maxq)
  * Per column: q = clamp(rint(w/s) + z, 0, maxq); w^ = s (q - z);
  *             e = (w - w^) / U[c][c].
  * Outputs: codes [d_out][d_in], scales/zeros [d_out][n_groups],
- *          E [d_out][d_in] (optional, the scaled errors e). */
+ *          E [d_out][d_in] (optional, the scaled errors e).
+ * Optional diagnostics (NULL to skip): qraw [d_out][d_in] = w / s before
+ * rounding, zraw [d_out][n_groups] = -min / s before rounding; they tell how
+ * close each integer decision was to a rounding tie. */
 int orc_gptq_rows(double *W, const double *U, int64_t d_out, int64_t d_in, int bits,
                   int64_t group_size, int64_t block, uint8_t *codes, float *scales,
-                  float *zeros, double *E)
+                  float *zeros, double *E, float *qraw, float *zraw)
 {
     if (!W || !U || !codes || !scales || !zeros || d_out < 0 || d_in <= 0 || bits < 1 ||
         bits > 8 || group_size == 0)
@@ -227,18 +234,19 @@ int orc_gptq_rows(double *W, const double *U, int64_t d_out, int64_t d_in, int b
         if (!e_row) { status = ORC_ERR_ARG; continue; }
         float s = 0.0f, z = 0.0f;
         if (group_size < 0) {
-            qgrid(w, d_in, maxq, &s, &z);
+            qgrid(w, d_in, maxq, &s, &z, zraw ? zraw + r : NULL);
             scales[r] = s;
             zeros[r] = z;
         }
         for (int64_t c = 0; c < d_in; c++) {
             if (group_size > 0 && c % group_size == 0) {
                 int64_t len = (d_in - c < group_size) ? d_in - c : group_size;
-                qgrid(w + c, len, maxq, &s, &z);
+                qgrid(w + c, len, maxq, &s, &z,
+                      zraw ? zraw + r * n_groups + c / group_size : NULL);
                 scales[r * n_groups + c / group_size] = s;
                 zeros[r * n_groups + c / group_size] = z;
             }
-            int q = qcode(w[c], s, z, maxq);
+            int q = qcode(w[c], s, z, maxq, qraw ? qraw + r * d_in + c : NULL);
             double what = (double)s * ((double)q - (double)z);
             double e = (w[c] - what) / U[c * d_in + c];
             codes[r * d_in + c] = (uint8_t)q;

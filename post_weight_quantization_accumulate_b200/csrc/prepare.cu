@@ -134,92 +134,170 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
     }
 }
 
-// Factor the kb x kb diagonal block at (k0, k0) of A in place (lower) and
-// write its inverse into Dinv[k0 .. k0+kb) (row stride kNB).
-__global__ void __launch_bounds__(256)
-    potrf_block_kernel(float* __restrict__ A, int d, int k0, int kb, float* __restrict__ Dinv,
-                       PrepHeader* hdr)
+// Element r (0..3) of four register values, without dynamic indexing.
+__device__ __forceinline__ float pick4(float v0, float v1, float v2, float v3, int r)
 {
-    __shared__ float L[kNB][kNB + 1];
-    __shared__ float X[kNB][kNB + 1];
-    __shared__ int bad;
-    const int tid = threadIdx.x;
-    if (tid == 0) bad = 0;
-    for (int idx = tid; idx < kNB * kNB; idx += blockDim.x) {
-        const int i = idx / kNB, j = idx % kNB;
-        L[i][j] = (i < kb && j < kb && j <= i) ? A[static_cast<int64_t>(k0 + i) * d + k0 + j]
-                                                 : 0.f;
-    }
-    __syncthreads();
-    for (int c = 0; c < kb; ++c) {
-        if (tid == 0) {
-            const float p = L[c][c];
-            if (!(p > 0.f) || !isfinite(p)) {
-                bad = 1;
-                L[c][c] = 1.f;
-            } else {
-                L[c][c] = sqrtf(p);
-            }
-        }
-        __syncthreads();
-        const float lcc = L[c][c];
-        for (int i = c + 1 + tid; i < kb; i += blockDim.x) L[i][c] = L[i][c] / lcc;
-        __syncthreads();
-        const int rem = kb - c - 1;
-        for (int idx = tid; idx < rem * rem; idx += blockDim.x) {
-            const int i = c + 1 + idx / rem, j = c + 1 + idx % rem;
-            if (j <= i) L[i][j] = fmaf(-L[i][c], L[j][c], L[i][j]);
-        }
-        __syncthreads();
-    }
-    // inverse of the lower factor, one column per thread: L x = e_j
-    if (tid < kb) {
-        const int j = tid;
-        for (int i = 0; i < kb; ++i) {
-            if (i < j) {
-                X[i][j] = 0.f;
-                continue;
-            }
-            float s = (i == j) ? 1.f : 0.f;
-            for (int k = j; k < i; ++k) s = fmaf(-L[i][k], X[k][j], s);
-            X[i][j] = s / L[i][i];
-        }
-    }
-    __syncthreads();
-    for (int idx = tid; idx < kb * kb; idx += blockDim.x) {
-        const int i = idx / kb, j = idx % kb;
-        A[static_cast<int64_t>(k0 + i) * d + k0 + j] = (j <= i) ? L[i][j] : 0.f;
-        Dinv[static_cast<int64_t>(k0 + i) * kNB + j] = X[i][j];
-    }
-    if (tid == 0 && bad) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
+    return r == 0 ? v0 : r == 1 ? v1 : r == 2 ? v2 : v3;
 }
 
-// Panel below the diagonal block: L[r][k0:k0+kb] = A[r][k0:k0+kb] * Dinv^T,
-// 64 rows per CTA.
+// One panel step of the blocked Cholesky, fused:
+//   every CTA factors the kb x kb diagonal block at (k0, k0) (redundantly, so
+//   no other launch has to wait for it) and inverts the factor; CTA 0 writes
+//   L_kk^{-1} into Dinv[k0 .. k0+kb); CTA b >= 1 solves the
+//   panel rows k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T}.
+// 256 threads as 16 x 16; thread (ty, tx) keeps the 4 x 4 sub-block rows
+// 4ty.., cols 4tx.. in registers.  Each column (row) step needs one barrier:
+// the column (row) for step c+1 is published to shared memory during step c.
 __global__ void __launch_bounds__(256)
-    trsm_panel_kernel(float* __restrict__ A, int d, int k0, int kb,
-                      const float* __restrict__ Dinv)
+    chol_panel_kernel(float* __restrict__ A, int d, int k0, int kb, float* __restrict__ Dinv,
+                      PrepHeader* hdr)
 {
-    __shared__ float T[kNB][kNB + 1];
-    __shared__ float Di[kNB][kNB + 1];
-    const int r0 = k0 + kb + blockIdx.x * kNB;
-    const int tid = threadIdx.x;
-    for (int idx = tid; idx < kNB * kNB; idx += blockDim.x) {
-        const int i = idx / kNB, j = idx % kNB;
-        const int r = r0 + i;
-        T[i][j] = (r < d && j < kb) ? A[static_cast<int64_t>(r) * d + k0 + j] : 0.f;
-        Di[i][j] = (i < kb && j < kb) ? Dinv[static_cast<int64_t>(k0 + i) * kNB + j] : 0.f;
+    __shared__ float Ls[kNB][kNB + 1];
+    __shared__ float Xs[kNB][kNB + 1];
+    __shared__ float vec[2][kNB];
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    const int r0 = 4 * ty, c0 = 4 * tx;
+
+    // diagonal block (lower part); padding beyond kb is the identity
+    float a[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int gi = r0 + i, gj = c0 + j;
+            float v = (gi == gj) ? 1.f : 0.f;
+            if (gi < kb && gj < kb && gj <= gi) v = A[static_cast<int64_t>(k0 + gi) * d + k0 + gj];
+            a[i][j] = v;
+        }
+    if (tx == 0)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) vec[0][r0 + i] = a[i][0];
+    __syncthreads();
+
+    bool bad = false;
+    for (int c = 0; c < kNB; ++c) {
+        const float* col = vec[c & 1];
+        float piv = col[c];
+        if (!(piv > 0.f) || !isfinite(piv)) {
+            bad = true;
+            piv = 1.f;
+        }
+        const float rs = 1.f / sqrtf(piv);
+        float li[4], lj[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) li[i] = col[r0 + i] * rs;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) lj[j] = col[c0 + j] * rs;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int gi = r0 + i, gj = c0 + j;
+                if (gj == c && gi >= c) a[i][j] = li[i];
+                else if (gj > c && gi >= gj) a[i][j] = fmaf(-li[i], lj[j], a[i][j]);
+            }
+        const int cn = c + 1;
+        if (cn < kNB && tx == (cn >> 2)) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) vec[cn & 1][r0 + i] = pick4(a[i][0], a[i][1], a[i][2], a[i][3], cn & 3);
+        }
+        __syncthreads();
+    }
+    if (bad && tid == 0 && blockIdx.x == 0) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Ls[r0 + i][c0 + j] = (c0 + j <= r0 + i) ? a[i][j] : 0.f;
+    __syncthreads();
+
+    // X = L^{-1}: row c of X is final once divided by L[c][c]; then rows > c
+    // subtract L[i][c] X[c][:].
+    float x[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[i][j] = (r0 + i == c0 + j) ? 1.f : 0.f;
+    if (ty == 0) {
+        const float inv = 1.f / Ls[0][0];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[0][j] *= inv;
+            vec[0][c0 + j] = x[0][j];
+        }
     }
     __syncthreads();
-    // out[i][j] = sum_{k <= j} T[i][k] * Di[j][k]
-    for (int idx = tid; idx < kNB * kNB; idx += blockDim.x) {
-        const int i = idx / kNB, j = idx % kNB;
-        const int r = r0 + i;
-        if (r >= d || j >= kb) continue;
-        float s = 0.f;
-        for (int k = 0; k <= j; ++k) s = fmaf(T[i][k], Di[j][k], s);
-        A[static_cast<int64_t>(r) * d + k0 + j] = s;
+    for (int c = 0; c < kNB; ++c) {
+        float rv[4], lc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) rv[j] = vec[c & 1][c0 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) lc[i] = Ls[r0 + i][c];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (r0 + i > c)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[i][j] = fmaf(-lc[i], rv[j], x[i][j]);
+        const int cn = c + 1;
+        if (cn < kNB && ty == (cn >> 2)) {
+            const float inv = 1.f / Ls[cn][cn];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i == (cn & 3))
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        x[i][j] *= inv;
+                        vec[cn & 1][c0 + j] = x[i][j];
+                    }
+        }
+        __syncthreads();
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Xs[r0 + i][c0 + j] = x[i][j];
+
+    if (blockIdx.x == 0) {
+        // L_kk itself is not needed later (the inverse uses L_kk^{-1} and the
+        // off-diagonal panels), and the other CTAs of this launch may still be
+        // reading the diagonal block of A, so only Dinv is written.
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int gi = r0 + i, gj = c0 + j;
+                if (gi < kb && gj < kb) Dinv[static_cast<int64_t>(k0 + gi) * kNB + gj] = x[i][j];
+            }
+        return;
+    }
+
+    // panel rows: P[i][j] = sum_{k <= j} T[i][k] X[j][k]
+    const int pr0 = k0 + kb + (blockIdx.x - 1) * kNB;
+    __syncthreads();
+    for (int idx = tid; idx < kNB * kNB; idx += 256) {
+        const int i = idx / kNB, j = idx % kNB;
+        const int r = pr0 + i;
+        Ls[i][j] = (r < d && j < kb) ? A[static_cast<int64_t>(r) * d + k0 + j] : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4] = {};
+    for (int k = 0; k < kNB; ++k) {
+        float t[4], xv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = Ls[r0 + i][k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xv[j] = Xs[c0 + j][k];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(t[i], xv[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = pr0 + r0 + i, cj = c0 + j;
+            if (r < d && cj < kb) A[static_cast<int64_t>(r) * d + k0 + cj] = acc[i][j];
+        }
 }
 
 // Minv diagonal blocks from Dinv.
@@ -284,12 +362,10 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     // blocked right-looking Cholesky, A = M M^T (lower)
     for (int k0 = 0; k0 < d; k0 += kNB) {
         const int kb = std::min(kNB, d - k0);
-        potrf_block_kernel<<<1, 256, 0, stream>>>(A, d, k0, kb, Dinv, hdr);
-        GPTQ_LAUNCH_CHECK();
         const int rest = d - k0 - kb;
-        if (rest <= 0) break;
-        trsm_panel_kernel<<<(rest + kNB - 1) / kNB, 256, 0, stream>>>(A, d, k0, kb, Dinv);
+        chol_panel_kernel<<<1 + (rest + kNB - 1) / kNB, 256, 0, stream>>>(A, d, k0, kb, Dinv, hdr);
         GPTQ_LAUNCH_CHECK();
+        if (rest <= 0) break;
         float* P = A + static_cast<int64_t>(k0 + kb) * d + k0;
         float* C = A + static_cast<int64_t>(k0 + kb) * d + k0 + kb;
         int rc = launch_sgemm(true, rest, rest, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,

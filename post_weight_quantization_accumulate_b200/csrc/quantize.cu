@@ -26,11 +26,12 @@ namespace {
 
 constexpr int QB = 128;           // largest block width
 constexpr int QTPR = 4;           // threads per row
-constexpr int QCPT = 32;          // columns per thread
+constexpr int QCPT = QB / QTPR;   // columns per thread (column 4m + p belongs to part p)
 constexpr int QROWS = 32;         // rows per CTA
 constexpr int QTHREADS = QROWS * QTPR;
-constexpr int US_LD = QTPR * (QCPT + 4);   // padded so the 4 column parts hit distinct banks
-constexpr size_t kBlockSmem = (static_cast<size_t>(QB) * US_LD + QB) * sizeof(float);
+constexpr int UT_PART = QCPT + 4; // padded part stride: the 4 parts of a U row hit distinct banks
+constexpr int UT_LD = QTPR * UT_PART;
+constexpr size_t kBlockSmem = (static_cast<size_t>(QB) * UT_LD + QB) * sizeof(float);
 
 struct QArgs {
     float* Wp;            // [d_out][d_in] working weights, processing order
@@ -53,22 +54,49 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, 
     z = rintf(__fdiv_rn(-mn, s));
 }
 
+// One lazy-batch block [j0, j0 + bw) of the column loop for QROWS rows.
+// Part p of a row holds columns 4m + p (m = 0..31) of the block in registers.
+// Per column c the row's value is known to all four parts through `nxt`
+// (a look-ahead copy of column c+1 fetched one step early), so the shuffle is
+// off the dependency chain  w_c -> q -> e -> w_{c+1}.  Only registers m >=
+// c/4 can still change, so step c updates 32 - c/4 of them.
 __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
 {
     extern __shared__ __align__(16) float qsm[];
-    float* Us = qsm;
-    float* udiag = qsm + QB * US_LD;
+    float* Ut = qsm;                  // Ut[c][p][m] = U[j0+c][j0+4m+p] for 4m+p > c
+    float* rdiag = qsm + QB * UT_LD;  // 1 / U[c][c]
     const int tid = threadIdx.x;
     const int j0 = a.j0, bw = a.bw, d_in = a.d_in;
 
-    for (int idx = tid; idx < QB * QB; idx += QTHREADS) {
-        const int c = idx / QB, k = idx % QB;
-        float v = 0.f;
-        if (c < bw && k < bw && k > c) v = a.U[static_cast<int64_t>(j0 + c) * d_in + j0 + k];
-        Us[c * US_LD + (k >> 5) * (QCPT + 4) + (k & 31)] = v;
+    // U block: 128 rows x 32 float4 = 4096 float4 loads, 32 per thread, 8 in flight
+#pragma unroll 1
+    for (int base = 0; base < QB * (QB / 4); base += QTHREADS * 8) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int idx = base + i * QTHREADS + tid;
+            const int c = idx / (QB / 4), k = (idx % (QB / 4)) * 4;
+            v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c < bw && k < bw)
+                v[i] = *reinterpret_cast<const float4*>(a.U + static_cast<int64_t>(j0 + c) * d_in + j0 + k);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int idx = base + i * QTHREADS + tid;
+            const int c = idx / (QB / 4), k = (idx % (QB / 4)) * 4;
+            const float e4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int kk = k + t;  // column kk = 4m + p with m = kk/4, p = kk%4 = t
+                Ut[c * UT_LD + t * UT_PART + (kk >> 2)] = (kk > c && kk < bw) ? e4[t] : 0.f;
+            }
+            if (k <= c && c < k + 4 && c < bw) {
+                const int t = c - k;
+                const float dv = t == 0 ? v[i].x : t == 1 ? v[i].y : t == 2 ? v[i].z : v[i].w;
+                rdiag[c] = 1.f / dv;
+            }
+        }
     }
-    for (int c = tid; c < QB; c += QTHREADS)
-        udiag[c] = (c < bw) ? a.U[static_cast<int64_t>(j0 + c) * (d_in + 1)] : 1.f;
     __syncthreads();
 
     const int lrow = tid / QTPR, part = tid % QTPR;
@@ -78,20 +106,11 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
     const int lane_base = lane & ~(QTPR - 1);
     const float maxq = static_cast<float>((1 << a.bits) - 1);
     const int64_t rowoff = static_cast<int64_t>(r) * d_in;
+    const float* wsrc = a.Wp + rowoff + j0 + part;
 
     float w[QCPT];
-    {
-        const int c0 = part * QCPT;
 #pragma unroll
-        for (int m = 0; m < QCPT; m += 4) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (valid && c0 + m < bw) v = *reinterpret_cast<const float4*>(a.Wp + rowoff + j0 + c0 + m);
-            w[m] = v.x;
-            w[m + 1] = v.y;
-            w[m + 2] = v.z;
-            w[m + 3] = v.w;
-        }
-    }
+    for (int m = 0; m < QCPT; ++m) w[m] = (valid && 4 * m + part < bw) ? wsrc[4 * m] : 0.f;
 
     // grid of the group in effect at the block start
     float s = 1.f, z = 0.f;
@@ -123,77 +142,75 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
             z = a.zeros[static_cast<int64_t>(r) * a.n_groups + g];
         }
     }
-    const bool inblock_groups = a.gs > 0 && a.gs <= a.block;
+    const int gs_in = (a.gs > 0 && a.gs <= a.block) ? a.gs : 0;
+    int next_group = gs_in ? 0 : 1 << 30;
 
-    uint32_t cq[QCPT / 4];
-#pragma unroll
-    for (int i = 0; i < QCPT / 4; ++i) cq[i] = 0u;
     float ereg[QCPT];
+    uint32_t qreg[QCPT / 4];
 #pragma unroll
     for (int i = 0; i < QCPT; ++i) ereg[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < QCPT / 4; ++i) qreg[i] = 0u;
     float errsum = 0.f;
+    float nxt = __shfl_sync(0xffffffffu, w[0], lane_base | 0);   // column 0
 
-    for (int po = 0; po < QTPR; ++po) {
 #pragma unroll
-        for (int m = 0; m < QCPT; ++m) {
-            const int c = po * QCPT + m;
-            if (c >= bw) break;
-            if (inblock_groups && (c % a.gs) == 0) {
-                float mn = 0.f, mx = 0.f;
+    for (int c = 0; c < QB; ++c) {
+        if (c >= bw) continue;   // uniform: the ragged last block of a row
+        const int m = c >> 2, po = c & 3;
+        // value of column c+1 after the updates of steps < c (owner's register)
+        const float pre = (c + 1 < QB) ? __shfl_sync(0xffffffffu, w[(c + 1) >> 2], lane_base | ((c + 1) & 3)) : 0.f;
+        if (c == next_group) {
+            float mn = 0.f, mx = 0.f;
 #pragma unroll
-                for (int mm = 0; mm < QCPT; ++mm) {
-                    const int col = part * QCPT + mm;
-                    const bool in = col >= c && col < c + a.gs && col < bw;
-                    const float v = in ? w[mm] : 0.f;
-                    mn = fminf(mn, v);
-                    mx = fmaxf(mx, v);
-                }
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                grid_from_range(mn, mx, maxq, s, z);
-                if (valid && part == 0) {
-                    const int g = (j0 + c) / a.gs;
-                    a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
-                    a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
-                }
+            for (int mm = m; mm < QCPT; ++mm) {
+                const int col = 4 * mm + part;
+                const bool in = col >= c && col < c + gs_in && col < bw;
+                const float v = in ? w[mm] : 0.f;
+                mn = fminf(mn, v);
+                mx = fmaxf(mx, v);
             }
-            const float wc = __shfl_sync(0xffffffffu, w[m], lane_base | po);
-            float q = rintf(__fdiv_rn(wc, s)) + z;
-            q = fminf(fmaxf(q, 0.f), maxq);
-            const float what = s * (q - z);
-            const float e = __fdiv_rn(wc - what, udiag[c]);
-            if (part == po) {
-                w[m] = what;
-                ereg[m] = e;
-                cq[m >> 2] |= static_cast<uint32_t>(q) << (8 * (m & 3));
-                errsum = fmaf(e, e, errsum);
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            grid_from_range(mn, mx, maxq, s, z);
+            if (valid && part == 0) {
+                const int g = (j0 + c) / gs_in;
+                a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
+                a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
             }
-            const float* urow = Us + c * US_LD + part * (QCPT + 4);
-#pragma unroll
-            for (int mm = 0; mm < QCPT; mm += 4) {
-                const float4 u4 = *reinterpret_cast<const float4*>(urow + mm);
-                w[mm] = fmaf(-e, u4.x, w[mm]);
-                w[mm + 1] = fmaf(-e, u4.y, w[mm + 1]);
-                w[mm + 2] = fmaf(-e, u4.z, w[mm + 2]);
-                w[mm + 3] = fmaf(-e, u4.w, w[mm + 3]);
-            }
+            next_group += gs_in;
         }
+        const float wc = nxt;
+        float q = rintf(__fdiv_rn(wc, s)) + z;
+        q = fminf(fmaxf(q, 0.f), maxq);
+        const float what = s * (q - z);
+        const float e = (wc - what) * rdiag[c];
+        if (part == po) {
+            w[m] = what;
+            ereg[m] = e;
+            qreg[m >> 2] |= static_cast<uint32_t>(q) << (8 * (m & 3));
+            errsum = fmaf(e, e, errsum);
+        }
+        const float* urow = Ut + c * UT_LD + part * UT_PART;
+        if (c + 1 < QB) nxt = fmaf(-e, Ut[c * UT_LD + ((c + 1) & 3) * UT_PART + ((c + 1) >> 2)], pre);
+#pragma unroll
+        for (int mm = m; mm < QCPT; ++mm) w[mm] = fmaf(-e, urow[mm], w[mm]);
     }
 
     errsum += __shfl_xor_sync(0xffffffffu, errsum, 1);
     errsum += __shfl_xor_sync(0xffffffffu, errsum, 2);
     if (!valid) return;
-    const int c0 = part * QCPT;
+    float* wdst = a.Wp + rowoff + j0 + part;
+    float* edst = a.E + static_cast<int64_t>(r) * QB + part;
+    uint8_t* cdst = a.codes_p + rowoff + j0 + part;
 #pragma unroll
-    for (int m = 0; m < QCPT; m += 4) {
-        if (c0 + m < bw) {
-            *reinterpret_cast<float4*>(a.Wp + rowoff + j0 + c0 + m) =
-                make_float4(w[m], w[m + 1], w[m + 2], w[m + 3]);
-            *reinterpret_cast<float4*>(a.E + static_cast<int64_t>(r) * QB + c0 + m) =
-                make_float4(ereg[m], ereg[m + 1], ereg[m + 2], ereg[m + 3]);
-            *reinterpret_cast<uint32_t*>(a.codes_p + rowoff + j0 + c0 + m) = cq[m >> 2];
+    for (int m = 0; m < QCPT; ++m) {
+        if (4 * m + part < bw) {
+            wdst[4 * m] = w[m];
+            edst[4 * m] = ereg[m];
+            cdst[4 * m] = static_cast<uint8_t>(qreg[m >> 2] >> (8 * (m & 3)));
         }
     }
     if (a.err_sq && part == 0) a.err_sq[r] += errsum;

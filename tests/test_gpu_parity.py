@@ -168,9 +168,7 @@ def _staged_check(W, xb, bits, gs, block, act_order, where):
     perm, Ug = _gpu_prepare(Hg, act_order)
     g = _gpu_quantize(W, Ug, perm if act_order else None, bits, gs, block)
     r = oracle.quantize(W.astype(np.float64), Ug.astype(np.float64), perm, bits, gs, block)
-    P.check_codes(g["codes"], r["codes"], where, bits, perm)
-    P.check_scales_zeros(g["scales"], g["zeros"], r["scales"], r["zeros"],
-                         g["codes"][:, perm], r["codes_perm"], gs, where)
+    P.check_quantized(g["codes"], g["scales"], g["zeros"], r, bits, gs, perm, where)
     H64 = Hg.astype(np.float64)
     mse_g = oracle.output_mse(W, g["W_hat"], H64, xb.shape[0])
     mse_r = oracle.output_mse(W, r["W_hat"], H64, xb.shape[0])
@@ -197,7 +195,7 @@ def _staged_check(W, xb, bits, gs, block, act_order, where):
 @pytest.mark.parametrize("gs", [-1, 32, 64, 128, 256])
 @pytest.mark.parametrize("act_order", [False, True])
 def test_quantize_matches_checker(bits, gs, act_order):
-    d_out, d_in, n = 96, 512, 2048
+    d_out, d_in, n = 256, 512, 2048
     W, xb = synth.random_layer(bits * 31 + gs, d_out, d_in, n, correlated=True)
     _staged_check(W, xb, bits, gs, 128, act_order, f"b{bits} g{gs} ao{act_order}")
 

@@ -50,11 +50,11 @@ def _outputs(d_out, d_in, bits, gs):
 
 def _compare(ref_W, ref, W, out, bits, gs, perm, where):
     torch.cuda.synchronize()
-    p = np.arange(ref_W.shape[1]) if perm is None else perm.cpu().numpy()
-    P.check_codes(out["codes"].cpu().numpy(), ref["codes"].cpu().numpy(), where, bits, p)
-    P.check_scales_zeros(out["scales"].cpu().numpy(), out["zeros"].cpu().numpy(),
-                         ref["scales"].cpu().numpy(), ref["zeros"].cpu().numpy(),
-                         out["codes"].cpu().numpy()[:, p], ref["codes"].cpu().numpy()[:, p], gs, where)
+    # the same kernels run behind both entry points: results agree exactly,
+    # which is inside every tolerance of the parity tests
+    np.testing.assert_array_equal(out["codes"].cpu().numpy(), ref["codes"].cpu().numpy())
+    np.testing.assert_allclose(out["scales"].cpu().numpy(), ref["scales"].cpu().numpy(), rtol=P.SZ_RTOL)
+    np.testing.assert_array_equal(out["zeros"].cpu().numpy(), ref["zeros"].cpu().numpy())
     np.testing.assert_allclose(W.cpu().numpy(), ref_W.cpu().numpy(), rtol=1e-5, atol=1e-7)
     np.testing.assert_array_equal(out["packed_int4"].cpu().numpy(), ref["packed_int4"].cpu().numpy())
     np.testing.assert_array_equal(out["g_idx"].cpu().numpy(), ref["g_idx"].cpu().numpy())
