@@ -242,6 +242,22 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// Shared-memory descriptor for an MN-major 32-bit (tf32) operand, the
+// SWIZZLE_128B_BASE32B layout (32-byte chunks swizzled within 128-byte rows,
+// period 4 rows) that TMA writes with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B:
+// lbo = bytes between consecutive 32-element MN chunks, sbo = bytes between
+// consecutive 4-row K groups.
+__device__ __forceinline__ uint64_t sdesc_sw128_base32b(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+    d |= static_cast<uint64_t>(1) << 61;  // SWIZZLE_128B_BASE32B
+    return d;
+}
+
 // Instruction descriptor for kind::f16 / kind::tf32 with f32 accumulation.
 // fmt: 0 = f16, 1 = bf16, 2 = tf32 (both operands); a_mn/b_mn: operand is
 // MN-major (1) or K-major (0).

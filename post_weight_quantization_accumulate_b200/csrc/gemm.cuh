@@ -13,9 +13,21 @@ enum GemmFlags : int {
 
 // C = alpha * A * B + beta * C (row-major; beta == 0 ignores C's contents).
 // trans_b: B is stored as [N, K] (ldb) instead of [K, N].
-// batch > 1: blockIdx.z selects A + z*sA, B + z*sB, C + z*sC.
+// batch > 1: matrix z of the batch is A + z*sA, B + z*sB, C + z*sC.
+// Runs on the tensor cores (3xTF32, gemm_tc.cu) whenever A and B are 16-byte
+// aligned with leading dimensions and batch strides that are multiples of 4
+// floats (the TMA rules), else on the SIMT kernel (gemm_simt.cu).
 int launch_sgemm(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                  int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                  int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream);
+
+int launch_sgemm_simt(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
+                      int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
+                      int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream);
+int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
+                   int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
+                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream);
+bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, int64_t ldb,
+                       int64_t sB, int batch);
 
 }  // namespace gptq

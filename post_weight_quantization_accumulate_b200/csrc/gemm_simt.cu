@@ -120,6 +120,17 @@ int launch_sgemm(bool trans_b, int M, int N, int K, float alpha, const float* A,
                  int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                  int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream)
 {
+    if (gemm_tc_supported(A, lda, sA, B, ldb, sB, batch))
+        return launch_gemm_tc(trans_b, M, N, K, alpha, A, lda, sA, B, ldb, sB, beta, C, ldc, sC,
+                              batch, flags, stream);
+    return launch_sgemm_simt(trans_b, M, N, K, alpha, A, lda, sA, B, ldb, sB, beta, C, ldc, sC,
+                             batch, flags, stream);
+}
+
+int launch_sgemm_simt(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
+                      int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
+                      int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream)
+{
     if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, batch);
     if (trans_b)

@@ -1,0 +1,411 @@
+// gemm_tc.cu -- fp32-accurate matrix product on the sm_100a tensor cores.
+//
+// C = alpha * A * B + beta * C with float32 operands, computed as three
+// tcgen05 kind::tf32 products (3xTF32): every operand x is split in shared
+// memory into hi = rna_tf32(x) and lo = x - hi (exact), and
+//     A B ~= A_hi B_hi + A_hi B_lo + A_lo B_hi
+// which keeps about 2^-22 relative error per product, close to float32.
+//
+// Used for the lazy-batch update of the column loop (W[:, j+B:] -= E U_blk),
+// the trailing update of the blocked Cholesky (A22 -= L21 L21^T) and the
+// recursive triangular inverse.
+//
+// Per CTA (384 threads, persistent over 128 x 128 output tiles x batch):
+//   warp 0       TMA producer: fp32 tiles of A (K-major) and B (MN- or K-major)
+//   warp 1       MMA issuer + TMEM owner (two 128-column fp32 accumulators)
+//   warps 4-7    converters: hi/lo split of each stage in shared memory
+//   warps 8-11   epilogue: TMEM -> registers -> alpha acc + beta C -> global
+// Three 64 KB stages (A_hi, A_lo, B_hi, B_lo of 16 KB each).  All waits are
+// bounded (see mbar_wait_bounded).
+#include "gemm.cuh"
+
+#include <mutex>
+
+namespace gptq {
+namespace {
+
+constexpr int TBM = 128, TBN = 128, TBK = 32;   // 32 fp32 = 128 bytes = one swizzle row
+constexpr int TSTAGES = 3;
+constexpr int TILE_BYTES = TBM * TBK * 4;        // 16 KB (A tile; also B tile: 128 x 32)
+constexpr int STAGE_BYTES = 4 * TILE_BYTES;      // A_hi, A_lo, B_hi, B_lo
+constexpr int TTHREADS = 384;
+constexpr int TMEM_COLS = 2 * TBN;
+
+struct alignas(1024) GemmSmem {
+    uint8_t stage[TSTAGES][STAGE_BYTES];
+    uint64_t full[TSTAGES];    // TMA landed
+    uint64_t conv[TSTAGES];    // hi/lo split done
+    uint64_t empty[TSTAGES];   // MMAs done reading
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr size_t GEMM_SMEM = sizeof(GemmSmem) + 1024;
+
+struct GemmArgs {
+    int M, N, K, batch, flags, trans_b;
+    float alpha, beta;
+    float* C;
+    int64_t ldc, sC;
+    int n_mt, n_nt;
+    int* status;
+};
+
+__device__ __forceinline__ uint32_t tf32_rna(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// Unit u -> (batch, m-tile, n-tile) and its K range [k0, k1) (multiples of TBK);
+// returns false for a tile the lower-triangular output flag skips.
+__device__ __forceinline__ bool unit_info(const GemmArgs& g, int u, int& b, int& mt, int& nt, int& k0,
+                                          int& k1)
+{
+    const int per = g.n_mt * g.n_nt;
+    b = u / per;
+    const int t = u % per;
+    mt = t / g.n_nt;
+    nt = t % g.n_nt;
+    const int m0 = mt * TBM, n0 = nt * TBN;
+    if ((g.flags & kGemmLowerC) && n0 > m0 + TBM - 1) return false;
+    k0 = 0;
+    k1 = g.K;
+    if (g.flags & kGemmLowerB) k0 = (n0 / TBK) * TBK;
+    if (g.flags & kGemmLowerA) k1 = min(g.K, m0 + TBM);
+    return true;
+}
+
+__global__ void __launch_bounds__(TTHREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   const GemmArgs g)
+{
+    extern __shared__ uint8_t smem_raw[];
+    GemmSmem& S = *reinterpret_cast<GemmSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TSTAGES; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.conv[s], 4);
+            mbar_init(&S.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&S.tfull[a], 1);
+            mbar_init(&S.tempty[a], 4);
+        }
+        S.abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&mapA);
+        prefetch_tmap(&mapB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = S.tmem_base;
+    volatile int* abort = &S.abort;
+    int* status = g.status;
+    const int n_units = g.n_mt * g.n_nt * g.batch;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                int b, mt, nt, k0, k1;
+                if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
+                for (int k = k0; k < k1; k += TBK, ++it) {
+                    const int s = it % TSTAGES;
+                    const uint32_t ph = (it / TSTAGES) & 1;
+                    if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&S.full[s], 2 * TILE_BYTES);
+                    uint8_t* st = S.stage[s];
+                    tma_load_3d(st, &mapA, &S.full[s], k, mt * TBM, b);
+                    uint8_t* bh = st + 2 * TILE_BYTES;
+                    if (g.trans_b) {
+                        tma_load_3d(bh, &mapB, &S.full[s], k, nt * TBN, b);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < TBN / 32; ++q)   // 32-column x 32-row boxes
+                            tma_load_3d(bh + q * (TBK * 32 * 4), &mapB, &S.full[s], nt * TBN + q * 32, k, b);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, g.trans_b ? 0u : 1u, TBM, TBN);
+            uint32_t it = 0, uc = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                int b, mt, nt, k0, k1;
+                if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
+                const int acc = uc & 1;
+                const uint32_t aph = (uc >> 1) & 1;
+                ++uc;
+                if (!mbar_wait_bounded(&S.tempty[acc], aph ^ 1, abort, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t dt = tbase + acc * TBN;
+                bool first = true;
+                for (int k = k0; k < k1; k += TBK, ++it) {
+                    const int s = it % TSTAGES;
+                    const uint32_t ph = (it / TSTAGES) & 1;
+                    if (!mbar_wait_bounded(&S.conv[s], ph, abort, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t ahi = smem_u32(S.stage[s]);
+                    const uint32_t alo = ahi + TILE_BYTES;
+                    const uint32_t bhi = ahi + 2 * TILE_BYTES;
+                    const uint32_t blo = ahi + 3 * TILE_BYTES;
+#pragma unroll
+                    for (int k8 = 0; k8 < TBK / 8; ++k8) {
+                        // A: K-major, 8 fp32 = 32 bytes further along the swizzled row
+                        const uint64_t dah = sdesc_sw128(ahi + k8 * 32, 16, 1024);
+                        const uint64_t dal = sdesc_sw128(alo + k8 * 32, 16, 1024);
+                        uint64_t dbh, dbl;
+                        if (g.trans_b) {
+                            dbh = sdesc_sw128(bhi + k8 * 32, 16, 1024);
+                            dbl = sdesc_sw128(blo + k8 * 32, 16, 1024);
+                        } else {
+                            // B: MN-major tf32 (128B swizzle, 32-byte atoms): 8 K-rows are
+                            // 1024 bytes on, 4-row K groups 512 bytes apart, 32-column
+                            // chunks TBK * 128 bytes apart
+                            dbh = sdesc_sw128_base32b(bhi + k8 * 1024, TBK * 128, 512);
+                            dbl = sdesc_sw128_base32b(blo + k8 * 1024, TBK * 128, 512);
+                        }
+                        umma_tf32(dt, dal, dbh, idesc, first ? 0u : 1u);
+                        umma_tf32(dt, dah, dbl, idesc, 1u);
+                        umma_tf32(dt, dah, dbh, idesc, 1u);
+                        first = false;
+                    }
+                    umma_commit(&S.empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&S.tfull[acc]);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // converters: x -> hi = rna_tf32(x) in place, lo = x - hi
+        const int ct = threadIdx.x - 128;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            int b, mt, nt, k0, k1;
+            if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
+            for (int k = k0; k < k1; k += TBK, ++it) {
+                const int s = it % TSTAGES;
+                const uint32_t ph = (it / TSTAGES) & 1;
+                const bool got = mbar_wait_bounded(&S.full[s], ph, abort, status);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                float4* ah = reinterpret_cast<float4*>(S.stage[s]);
+                float4* al = reinterpret_cast<float4*>(S.stage[s] + TILE_BYTES);
+                float4* bh = reinterpret_cast<float4*>(S.stage[s] + 2 * TILE_BYTES);
+                float4* bl = reinterpret_cast<float4*>(S.stage[s] + 3 * TILE_BYTES);
+#pragma unroll 4
+                for (int i = ct; i < TILE_BYTES / 16; i += 128) {
+                    float4 x = ah[i], h, l;
+                    h.x = __uint_as_float(tf32_rna(x.x)); l.x = x.x - h.x;
+                    h.y = __uint_as_float(tf32_rna(x.y)); l.y = x.y - h.y;
+                    h.z = __uint_as_float(tf32_rna(x.z)); l.z = x.z - h.z;
+                    h.w = __uint_as_float(tf32_rna(x.w)); l.w = x.w - h.w;
+                    ah[i] = h;
+                    al[i] = l;
+                    x = bh[i];
+                    h.x = __uint_as_float(tf32_rna(x.x)); l.x = x.x - h.x;
+                    h.y = __uint_as_float(tf32_rna(x.y)); l.y = x.y - h.y;
+                    h.z = __uint_as_float(tf32_rna(x.z)); l.z = x.z - h.z;
+                    h.w = __uint_as_float(tf32_rna(x.w)); l.w = x.w - h.w;
+                    bh[i] = h;
+                    bl[i] = l;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.conv[s]);
+            }
+        }
+    } else if (warp >= 8) {
+        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (= tile rows)
+        const int q = warp & 3;
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        uint32_t uc = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            int b, mt, nt, k0, k1;
+            if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
+            const int acc = uc & 1;
+            const uint32_t aph = (uc >> 1) & 1;
+            ++uc;
+            const bool got = mbar_wait_bounded(&S.tfull[acc], aph, abort, status);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const bool have = k1 > k0;   // an empty K range leaves the accumulator unwritten
+            const int row = mt * TBM + q * 32 + lane;
+            float* crow = g.C + b * g.sC + static_cast<int64_t>(row) * g.ldc;
+#pragma unroll 1
+            for (int c = 0; c < TBN / 32; ++c) {
+                float v[32];
+                tmem_ld_32x32b_x32(tbase + lane_addr + acc * TBN + c * 32, v);
+                tmem_ld_wait();
+                const int col0 = nt * TBN + c * 32;
+                if (row >= g.M || col0 >= g.N) continue;
+                const bool lower = (g.flags & kGemmLowerC) != 0;
+                if (col0 + 32 <= g.N && !(lower && col0 + 31 > row) &&
+                    (reinterpret_cast<uintptr_t>(crow + col0) & 15) == 0) {
+                    float4* p = reinterpret_cast<float4*>(crow + col0);
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (g.beta != 0.f) o = p[m];
+                        const float a0 = have ? v[4 * m] : 0.f, a1 = have ? v[4 * m + 1] : 0.f;
+                        const float a2 = have ? v[4 * m + 2] : 0.f, a3 = have ? v[4 * m + 3] : 0.f;
+                        o.x = fmaf(g.alpha, a0, g.beta * o.x);
+                        o.y = fmaf(g.alpha, a1, g.beta * o.y);
+                        o.z = fmaf(g.alpha, a2, g.beta * o.z);
+                        o.w = fmaf(g.alpha, a3, g.beta * o.w);
+                        p[m] = o;
+                    }
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 32; ++m) {
+                        const int col = col0 + m;
+                        if (col >= g.N || (lower && col > row)) continue;
+                        const float a = have ? v[m] : 0.f;
+                        const float old = (g.beta != 0.f) ? crow[col] : 0.f;
+                        crow[col] = fmaf(g.alpha, a, g.beta * old);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tempty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, TMEM_COLS);
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D fp32 tensor map: inner dimension `cols` (contiguous), `rows` rows of
+// pitch ld, `batch` matrices `bstride` elements apart; box box_c x box_r x 1.
+int make_map_f32(CUtensorMap* map, const float* base, int64_t cols, int64_t rows, int64_t ld,
+                 int batch, int64_t bstride, int box_c, int box_r, CUtensorMapSwizzle swz)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(batch)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 4,
+                             static_cast<cuuint64_t>(batch > 1 ? bstride : ld * rows) * 4};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_c), static_cast<cuuint32_t>(box_r), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return GPTQ_OK;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, int64_t ldb,
+                       int64_t sB, int batch)
+{
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    if (!al16(A) || !al16(B) || (lda & 3) || (ldb & 3)) return false;
+    if (batch > 1 && ((sA & 3) || (sB & 3))) return false;
+    return true;
+}
+
+int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
+                   int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
+                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream)
+{
+    if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
+    if (dev < 64 && !attr_set[dev]) {
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(GEMM_SMEM)));
+        attr_set[dev] = true;
+    }
+    const int Kp = K > 0 ? K : 1;
+    CUtensorMap mA, mB;
+    int rc = make_map_f32(&mA, A, Kp, M, lda, batch, sA, TBK, TBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    if (trans_b)
+        rc = make_map_f32(&mB, B, Kp, N, ldb, batch, sB, TBK, TBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        rc = make_map_f32(&mB, B, N, Kp, ldb, batch, sB, 32, TBK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+    if (rc) return rc;
+    GemmArgs g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.batch = batch;
+    g.flags = flags;
+    g.trans_b = trans_b ? 1 : 0;
+    g.alpha = alpha;
+    g.beta = beta;
+    g.C = C;
+    g.ldc = ldc;
+    g.sC = sC;
+    g.n_mt = (M + TBM - 1) / TBM;
+    g.n_nt = (N + TBN - 1) / TBN;
+    g.status = device_status_ptr();
+    const int64_t units = static_cast<int64_t>(g.n_mt) * g.n_nt * batch;
+    const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
+    gemm_tc_kernel<<<grid, TTHREADS, GEMM_SMEM, stream>>>(mA, mB, g);
+    GPTQ_LAUNCH_CHECK();
+    return GPTQ_OK;
+}
+
+}  // namespace gptq

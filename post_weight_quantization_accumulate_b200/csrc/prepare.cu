@@ -182,20 +182,30 @@ __global__ void __launch_bounds__(256)
             bad = true;
             piv = 1.f;
         }
-        const float rs = 1.f / sqrtf(piv);
+        const float rs = rsqrtf(piv);
+        // column c of L for my rows; the trailing update uses only entries
+        // below column c, so the others are multiplied by 0
         float li[4], lj[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) li[i] = col[r0 + i] * rs;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) lj[j] = col[c0 + j] * rs;
+        for (int j = 0; j < 4; ++j) lj[j] = (c0 + j > c) ? col[c0 + j] * rs : 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int gi = r0 + i, gj = c0 + j;
-                if (gj == c && gi >= c) a[i][j] = li[i];
-                else if (gj > c && gi >= gj) a[i][j] = fmaf(-li[i], lj[j], a[i][j]);
+            for (int j = 0; j < 4; ++j) a[i][j] = fmaf(-li[i], lj[j], a[i][j]);
+        if (tx == (c >> 2)) {
+            const int jc = c & 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (r0 + i >= c) {
+                    if (jc == 0) a[i][0] = li[i];
+                    if (jc == 1) a[i][1] = li[i];
+                    if (jc == 2) a[i][2] = li[i];
+                    if (jc == 3) a[i][3] = li[i];
+                }
             }
+        }
         const int cn = c + 1;
         if (cn < kNB && tx == (cn >> 2)) {
 #pragma unroll
@@ -231,12 +241,11 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int j = 0; j < 4; ++j) rv[j] = vec[c & 1][c0 + j];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) lc[i] = Ls[r0 + i][c];
+        for (int i = 0; i < 4; ++i) lc[i] = (r0 + i > c) ? Ls[r0 + i][c] : 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            if (r0 + i > c)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) x[i][j] = fmaf(-lc[i], rv[j], x[i][j]);
+            for (int j = 0; j < 4; ++j) x[i][j] = fmaf(-lc[i], rv[j], x[i][j]);
         const int cn = c + 1;
         if (cn < kNB && ty == (cn >> 2)) {
             const float inv = 1.f / Ls[cn][cn];
@@ -273,10 +282,21 @@ __global__ void __launch_bounds__(256)
     // panel rows: P[i][j] = sum_{k <= j} T[i][k] X[j][k]
     const int pr0 = k0 + kb + (blockIdx.x - 1) * kNB;
     __syncthreads();
-    for (int idx = tid; idx < kNB * kNB; idx += 256) {
-        const int i = idx / kNB, j = idx % kNB;
-        const int r = pr0 + i;
-        Ls[i][j] = (r < d && j < kb) ? A[static_cast<int64_t>(r) * d + k0 + j] : 0.f;
+    {
+        // 64 x 64 tile: 16 loads per thread, all issued before any is used
+        float tv[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const int idx = tid + t * 256;
+            const int i = idx / kNB, j = idx % kNB;
+            const int r = pr0 + i;
+            tv[t] = (r < d && j < kb) ? A[static_cast<int64_t>(r) * d + k0 + j] : 0.f;
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const int idx = tid + t * 256;
+            Ls[idx / kNB][idx % kNB] = tv[t];
+        }
     }
     __syncthreads();
     float acc[4][4] = {};

@@ -25,13 +25,19 @@ namespace gptq {
 namespace {
 
 constexpr int QB = 128;           // largest block width
-constexpr int QTPR = 4;           // threads per row
-constexpr int QCPT = QB / QTPR;   // columns per thread (column 4m + p belongs to part p)
-constexpr int QROWS = 32;         // rows per CTA
+constexpr int QTPR = 8;           // threads per row
+constexpr int QCPT = QB / QTPR;   // registers per thread (column 8m + p belongs to part p)
+constexpr int QSUB = 16;          // columns per unrolled sub-block
+constexpr int QRPS = QSUB / QTPR; // registers a sub-block occupies per thread
+constexpr int QROWS = 16;         // rows per CTA
 constexpr int QTHREADS = QROWS * QTPR;
-constexpr int UT_PART = QCPT + 4; // padded part stride: the 4 parts of a U row hit distinct banks
+constexpr int UT_PART = QCPT + 4; // padded part stride (80 bytes): the 8 parts of a U row
+                                  // read by one 8-lane phase hit distinct banks
 constexpr int UT_LD = QTPR * UT_PART;
-constexpr size_t kBlockSmem = (static_cast<size_t>(QB) * UT_LD + QB) * sizeof(float);
+constexpr int ES_LD = QB + 4;
+constexpr size_t kBlockSmem =
+    (static_cast<size_t>(QB) * UT_LD + QB + static_cast<size_t>(QROWS) * ES_LD) * sizeof(float) +
+    static_cast<size_t>(QROWS) * ES_LD;
 
 struct QArgs {
     float* Wp;            // [d_out][d_in] working weights, processing order
@@ -54,21 +60,70 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, 
     z = rintf(__fdiv_rn(-mn, s));
 }
 
+// rint(w / s) with w / s correctly rounded, from the product w * rs (rs the
+// correctly rounded 1 / s).  The product is within 2^-23 relative of w / s,
+// so the two round to the same integer unless w / s lies that close to a
+// half-integer; only then is the division carried out.
+__device__ __forceinline__ float rint_div(float w, float s, float rs)
+{
+    const float t = w * rs;
+    const float fr = t - floorf(t);
+    if (fabsf(fr - 0.5f) <= 4.8e-7f * fmaxf(fabsf(t), 1.f)) return rintf(__fdiv_rn(w, s));
+    return rintf(t);
+}
+
+// Register slot of in-block column k (owned by part k % QTPR) while sub-block
+// S is processed: the QCPT-slot window rotates by QRPS slots per sub-block,
+// so the current sub-block always sits in slots 0..QRPS-1.
+__device__ __forceinline__ int slot_of(int k, int S) { return (k / QTPR - QRPS * S) & (QCPT - 1); }
+
+// Scale and zero of the group starting at in-block column c, from the row's
+// current values: each part reduces its registers whose column lies in
+// [c, c + gs) and below bw, then the QTPR parts combine.
+__device__ __forceinline__ void group_grid(const float (&w)[QCPT], int S, int part, int c, int gs,
+                                           int bw, float maxq, float& s, float& z)
+{
+    float mn = 0.f, mx = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < QCPT; ++mm) {
+        const int col = QTPR * ((mm + QRPS * S) & (QCPT - 1)) + part;
+        const bool in = col >= c && col < c + gs && col < bw;
+        const float v = in ? w[mm] : 0.f;
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+    }
+#pragma unroll
+    for (int o = 1; o < QTPR; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    grid_from_range(mn, mx, maxq, s, z);
+}
+
 // One lazy-batch block [j0, j0 + bw) of the column loop for QROWS rows.
-// Part p of a row holds columns 4m + p (m = 0..31) of the block in registers.
-// Per column c the row's value is known to all four parts through `nxt`
-// (a look-ahead copy of column c+1 fetched one step early), so the shuffle is
-// off the dependency chain  w_c -> q -> e -> w_{c+1}.  Only registers m >=
-// c/4 can still change, so step c updates 32 - c/4 of them.
+// Part p of a row holds columns 8m + p of the block in 16 registers.  Per
+// column c every part knows the row's current value through `nxt` (a copy of
+// column c+1 fetched one step early with a shuffle), computes the same q and
+// e, and corrects its own registers with U row c from shared memory.  The U
+// rows are stored in the register order of their sub-block, in which columns
+// already quantized have coefficient 0.  Only 16 steps are unrolled; the
+// window rotates after each sub-block, which keeps the code small enough for
+// the instruction cache.  Nothing is stored inside a step: the step's U row
+// is read first, errors and codes stay in registers until the sub-block ends.
+// kGroupsInStep: a group may start inside a 16-column sub-block (group sizes
+// that are not multiples of 16); otherwise groups start at sub-block starts.
+template <bool kGroupsInStep>
 __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
 {
     extern __shared__ __align__(16) float qsm[];
-    float* Ut = qsm;                  // Ut[c][p][m] = U[j0+c][j0+4m+p] for 4m+p > c
-    float* rdiag = qsm + QB * UT_LD;  // 1 / U[c][c]
+    float* Ut = qsm;                         // [c][p][slot]
+    float* rdiag = qsm + QB * UT_LD;         // 1 / U[c][c]
+    float* Es = rdiag + QB;                  // [row][c] errors e
+    uint8_t* Cs = reinterpret_cast<uint8_t*>(Es + QROWS * ES_LD);  // [row][c] codes
     const int tid = threadIdx.x;
     const int j0 = a.j0, bw = a.bw, d_in = a.d_in;
 
-    // U block: 128 rows x 32 float4 = 4096 float4 loads, 32 per thread, 8 in flight
+    // U block: 128 rows x 32 float4 loads, 8 in flight per thread
 #pragma unroll 1
     for (int base = 0; base < QB * (QB / 4); base += QTHREADS * 8) {
         float4 v[8];
@@ -84,11 +139,12 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
         for (int i = 0; i < 8; ++i) {
             const int idx = base + i * QTHREADS + tid;
             const int c = idx / (QB / 4), k = (idx % (QB / 4)) * 4;
+            const int S = c / QSUB;
             const float e4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                const int kk = k + t;  // column kk = 4m + p with m = kk/4, p = kk%4 = t
-                Ut[c * UT_LD + t * UT_PART + (kk >> 2)] = (kk > c && kk < bw) ? e4[t] : 0.f;
+                const int kk = k + t;
+                Ut[c * UT_LD + (kk % QTPR) * UT_PART + slot_of(kk, S)] = (kk > c && kk < bw) ? e4[t] : 0.f;
             }
             if (k <= c && c < k + 4 && c < bw) {
                 const int t = c - k;
@@ -106,11 +162,11 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
     const int lane_base = lane & ~(QTPR - 1);
     const float maxq = static_cast<float>((1 << a.bits) - 1);
     const int64_t rowoff = static_cast<int64_t>(r) * d_in;
-    const float* wsrc = a.Wp + rowoff + j0 + part;
 
     float w[QCPT];
 #pragma unroll
-    for (int m = 0; m < QCPT; ++m) w[m] = (valid && 4 * m + part < bw) ? wsrc[4 * m] : 0.f;
+    for (int m = 0; m < QCPT; ++m)
+        w[m] = (valid && QTPR * m + part < bw) ? a.Wp[rowoff + j0 + QTPR * m + part] : 0.f;
 
     // grid of the group in effect at the block start
     float s = 1.f, z = 0.f;
@@ -128,10 +184,11 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
                 mn = fminf(mn, v);
                 mx = fmaxf(mx, v);
             }
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+#pragma unroll
+            for (int o = 1; o < QTPR; o <<= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
             grid_from_range(mn, mx, maxq, s, z);
             if (valid && part == 0) {
                 a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
@@ -142,78 +199,110 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
             z = a.zeros[static_cast<int64_t>(r) * a.n_groups + g];
         }
     }
+    float rs = 1.f / s;
     const int gs_in = (a.gs > 0 && a.gs <= a.block) ? a.gs : 0;
     int next_group = gs_in ? 0 : 1 << 30;
 
-    float ereg[QCPT];
-    uint32_t qreg[QCPT / 4];
-#pragma unroll
-    for (int i = 0; i < QCPT; ++i) ereg[i] = 0.f;
-#pragma unroll
-    for (int i = 0; i < QCPT / 4; ++i) qreg[i] = 0u;
     float errsum = 0.f;
     float nxt = __shfl_sync(0xffffffffu, w[0], lane_base | 0);   // column 0
+    const int nsub = (bw + QSUB - 1) / QSUB;
 
-#pragma unroll
-    for (int c = 0; c < QB; ++c) {
-        if (c >= bw) continue;   // uniform: the ragged last block of a row
-        const int m = c >> 2, po = c & 3;
-        // value of column c+1 after the updates of steps < c (owner's register)
-        const float pre = (c + 1 < QB) ? __shfl_sync(0xffffffffu, w[(c + 1) >> 2], lane_base | ((c + 1) & 3)) : 0.f;
-        if (c == next_group) {
-            float mn = 0.f, mx = 0.f;
-#pragma unroll
-            for (int mm = m; mm < QCPT; ++mm) {
-                const int col = 4 * mm + part;
-                const bool in = col >= c && col < c + gs_in && col < bw;
-                const float v = in ? w[mm] : 0.f;
-                mn = fminf(mn, v);
-                mx = fmaxf(mx, v);
-            }
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            grid_from_range(mn, mx, maxq, s, z);
+#pragma unroll 1
+    for (int S = 0; S < nsub; ++S) {
+        const float* ub = Ut + S * QSUB * UT_LD;
+        const float* rd = rdiag + S * QSUB;
+        if (!kGroupsInStep && S * QSUB == next_group) {
+            group_grid(w, S, part, S * QSUB, gs_in, bw, maxq, s, z);
+            rs = 1.f / s;
             if (valid && part == 0) {
-                const int g = (j0 + c) / gs_in;
+                const int g = (j0 + S * QSUB) / gs_in;
                 a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
                 a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
             }
             next_group += gs_in;
         }
-        const float wc = nxt;
-        float q = rintf(__fdiv_rn(wc, s)) + z;
-        q = fminf(fmaxf(q, 0.f), maxq);
-        const float what = s * (q - z);
-        const float e = (wc - what) * rdiag[c];
-        if (part == po) {
-            w[m] = what;
-            ereg[m] = e;
-            qreg[m >> 2] |= static_cast<uint32_t>(q) << (8 * (m & 3));
-            errsum = fmaf(e, e, errsum);
-        }
-        const float* urow = Ut + c * UT_LD + part * UT_PART;
-        if (c + 1 < QB) nxt = fmaf(-e, Ut[c * UT_LD + ((c + 1) & 3) * UT_PART + ((c + 1) >> 2)], pre);
+        float e_own[QRPS], q_own[QRPS];
 #pragma unroll
-        for (int mm = m; mm < QCPT; ++mm) w[mm] = fmaf(-e, urow[mm], w[mm]);
+        for (int i = 0; i < QRPS; ++i) e_own[i] = q_own[i] = 0.f;
+#pragma unroll
+        for (int cl = 0; cl < QSUB; ++cl) {
+            const int c = S * QSUB + cl;
+            if (c < bw) {
+                const int m = cl / QTPR, po = cl % QTPR;
+                const int mn1 = (cl + 1) / QTPR, pn1 = (cl + 1) % QTPR;
+                const float* urow = ub + cl * UT_LD;
+                // operands of this step that do not depend on its error
+                float u[QCPT];
+#pragma unroll
+                for (int mm = (m & ~3); mm < QCPT; mm += 4) {
+                    const float4 u4 = *reinterpret_cast<const float4*>(urow + part * UT_PART + mm);
+                    u[mm] = u4.x;
+                    u[mm + 1] = u4.y;
+                    u[mm + 2] = u4.z;
+                    u[mm + 3] = u4.w;
+                }
+                const float unext = urow[pn1 * UT_PART + mn1];
+                const float rdc = rd[cl];
+                // column c+1 after the corrections of steps < c (its owner's register)
+                const float pre = __shfl_sync(0xffffffffu, w[mn1], lane_base | pn1);
+                if (kGroupsInStep && c == next_group) {
+                    group_grid(w, S, part, c, gs_in, bw, maxq, s, z);
+                    rs = 1.f / s;
+                    if (valid && part == 0) {
+                        const int g = (j0 + c) / gs_in;
+                        a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
+                        a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
+                    }
+                    next_group += gs_in;
+                }
+                const float wc = nxt;
+                float q = rint_div(wc, s, rs) + z;
+                q = fminf(fmaxf(q, 0.f), maxq);
+                const float what = s * (q - z);
+                const float e = (wc - what) * rdc;
+                nxt = fmaf(-e, unext, pre);
+                if (part == po) {
+                    w[m] = what;
+                    e_own[m] = e;
+                    q_own[m] = q;
+                    errsum = fmaf(e, e, errsum);
+                }
+#pragma unroll
+                for (int mm = m; mm < QCPT; ++mm) w[mm] = fmaf(-e, u[mm], w[mm]);
+            }
+        }
+        // sub-block S is final in slots 0..QRPS-1: store, then rotate the window
+#pragma unroll
+        for (int i = 0; i < QRPS; ++i) {
+            const int col = S * QSUB + QTPR * i + part;
+            if (col < bw) {
+                if (valid) a.Wp[rowoff + j0 + col] = w[i];
+                Es[lrow * ES_LD + col] = e_own[i];
+                Cs[lrow * ES_LD + col] = static_cast<uint8_t>(q_own[i]);
+            }
+        }
+        float t[QRPS];
+#pragma unroll
+        for (int i = 0; i < QRPS; ++i) t[i] = w[i];
+#pragma unroll
+        for (int i = 0; i < QCPT - QRPS; ++i) w[i] = w[i + QRPS];
+#pragma unroll
+        for (int i = 0; i < QRPS; ++i) w[QCPT - QRPS + i] = t[i];
     }
 
-    errsum += __shfl_xor_sync(0xffffffffu, errsum, 1);
-    errsum += __shfl_xor_sync(0xffffffffu, errsum, 2);
-    if (!valid) return;
-    float* wdst = a.Wp + rowoff + j0 + part;
-    float* edst = a.E + static_cast<int64_t>(r) * QB + part;
-    uint8_t* cdst = a.codes_p + rowoff + j0 + part;
 #pragma unroll
-    for (int m = 0; m < QCPT; ++m) {
-        if (4 * m + part < bw) {
-            wdst[4 * m] = w[m];
-            edst[4 * m] = ereg[m];
-            cdst[4 * m] = static_cast<uint8_t>(qreg[m >> 2] >> (8 * (m & 3)));
+    for (int o = 1; o < QTPR; o <<= 1) errsum += __shfl_xor_sync(0xffffffffu, errsum, o);
+    __syncthreads();
+    // errors and codes of the CTA's rows, row-contiguous
+    for (int idx = tid; idx < QROWS * QB; idx += QTHREADS) {
+        const int rl = idx / QB, c = idx % QB;
+        const int rr = blockIdx.x * QROWS + rl;
+        if (rr < a.d_out && c < bw) {
+            a.E[static_cast<int64_t>(rr) * QB + c] = Es[rl * ES_LD + c];
+            a.codes_p[static_cast<int64_t>(rr) * d_in + j0 + c] = Cs[rl * ES_LD + c];
         }
     }
-    if (a.err_sq && part == 0) a.err_sq[r] += errsum;
+    if (valid && a.err_sq && part == 0) a.err_sq[r] += errsum;
 }
 
 // One (scale, zero) per row from the whole original row (group_size = -1).
@@ -358,11 +447,17 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
     int dev = 0;
     GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
     if (dev < 64 && !attr_set[dev]) {
-        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel,
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kBlockSmem)));
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kBlockSmem)));
         attr_set[dev] = true;
     }
+    // groups start only at 16-column sub-block starts when group_size is a
+    // multiple of 16 that fits the block (or there are no in-block groups)
+    const bool groups_in_step = gs > 0 && gs <= block && (gs % QSUB) != 0;
 
     float* work = W;
     if (perm) {
@@ -386,7 +481,10 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
         const int bw = (d_in - j0 < block) ? d_in - j0 : block;
         QArgs a{work, U, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
                 codes_p, E, err_sq};
-        gptq_block_kernel<<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+        if (groups_in_step)
+            gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+        else
+            gptq_block_kernel<false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
         GPTQ_LAUNCH_CHECK();
         const int rest = d_in - j0 - bw;
         if (rest > 0) {

@@ -6,13 +6,14 @@
 The inputs follow the workload's recipe (see synth.py) with `--tokens`
 overriding the calibration size, so a profiler can capture a launch on a case
 that is larger than L2 but small in device memory.  Prints the mean CUDA-event
-time of the call.
+time of the call and the host time spent enqueueing it.
 """
 from __future__ import annotations
 
 import argparse
 import os
 import sys
+import time
 
 import numpy as np
 import torch
@@ -60,12 +61,14 @@ def main():
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
+    t0 = time.perf_counter()
     for _ in range(a.reps):
         once()
+    t_host = (time.perf_counter() - t0) / a.reps
     e1.record()
     torch.cuda.synchronize()
-    print(f"{a.call} {spec.name} tokens={spec.n_tokens}: {e0.elapsed_time(e1) / a.reps:.3f} ms/call, "
-          f"status {B.gptq_device_status()}")
+    print(f"{a.call} {spec.name} tokens={spec.n_tokens}: {e0.elapsed_time(e1) / a.reps:.3f} ms/call on "
+          f"the device, {t_host * 1e3:.3f} ms/call to enqueue on the host, status {B.gptq_device_status()}")
 
 
 if __name__ == "__main__":
