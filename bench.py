@@ -214,7 +214,7 @@ def main():
     import torch.distributed as dist
     from post_weight_quantization_accumulate_b200 import binding as B
     from post_weight_quantization_accumulate_b200 import build as build_mod
-    from post_weight_quantization_accumulate_b200 import synth
+    from post_weight_quantization_accumulate_b200 import ranks, synth
     from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
 
     if rank == 0:
@@ -230,7 +230,7 @@ def main():
     B.lib()
 
     base = synth.WORKLOADS[args.workload]
-    spec = synth.scaled(base, tensor_id=rank)       # an independent layer per rank
+    spec = ranks.rank_workload(base, rank)          # an independent layer per rank
     threads = len(os.sched_getaffinity(0))
 
     # inputs: generated on the host, pinned, copied to HBM once
@@ -283,10 +283,7 @@ def main():
     ms = t_start.elapsed_time(t_end) / args.steps
     h_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_h)
     status = B.gptq_device_status()
-    if world > 1:
-        t = torch.tensor([ms, h_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, h_ms = float(t[0]), float(t[1])
+    ms, h_ms = ranks.max_over_ranks([ms, h_ms], device=dev)
     clocks = clk.summary()
 
     # one step broken down by stage (after the timed region)
@@ -336,13 +333,10 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = ranks.max_over_ranks([e2e_ms], device=dev)[0]
         h2d = X_host.numel() * 2 + W_host.numel() * W_host.element_size()
         d2h = (packed_h.numel() + scales_h.numel() * 4 + zeros_h.numel() * 4 + gidx_h.numel() * 4)
-        e2e = {"value": world * spec.d_out * spec.d_in / (e2e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": ranks.job_rate(world, spec.d_out, spec.d_in, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     cpu = None
@@ -358,7 +352,7 @@ def main():
         traffic = profiled_traffic(os.path.join(ROOT, "post_weight_quantization_accumulate_b200",
                                                 "csrc", "hessian.cu"))
         line = {
-            "metric": METRIC, "value": world * spec.d_out * spec.d_in / (ms / 1e3), "unit": UNIT,
+            "metric": METRIC, "value": ranks.job_rate(world, spec.d_out, spec.d_in, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": config_of(spec, world),
