@@ -134,136 +134,158 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
     }
 }
 
-// Element r (0..3) of four register values, without dynamic indexing.
-__device__ __forceinline__ float pick4(float v0, float v1, float v2, float v3, int r)
-{
-    return r == 0 ? v0 : r == 1 ? v1 : r == 2 ? v2 : v3;
-}
-
 // One panel step of the blocked Cholesky, fused:
 //   every CTA factors the kb x kb diagonal block at (k0, k0) (redundantly, so
 //   no other launch has to wait for it) and inverts the factor; CTA 0 writes
-//   L_kk^{-1} into Dinv[k0 .. k0+kb); CTA b >= 1 solves the
-//   panel rows k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T}.
-// 256 threads as 16 x 16; thread (ty, tx) keeps the 4 x 4 sub-block rows
-// 4ty.., cols 4tx.. in registers.  Each column (row) step needs one barrier:
-// the column (row) for step c+1 is published to shared memory during step c.
+//   L_kk^{-1} into Dinv[k0 .. k0+kb); CTA b >= 1 solves the panel rows
+//   k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T}.
+// Factorisation of the 64 x 64 block in shared memory, in 16 strips of 4
+// columns: warp 0 factors the strip with shuffles (lane l holds rows 4P+l and
+// 4P+l+32), then all warps subtract its rank-4 product from the trailing
+// lower triangle (thread (ty, tx) owns the 4 x 4 tile rows 4ty.., cols 4tx..).
+// Inverse Z = L^{-1} by recursive doubling: the 16 diagonal 4 x 4 inverses,
+// then Z21 = -Z22 (L21 Z11) for block sizes 8, 16, 32, 64.
 __global__ void __launch_bounds__(256)
     chol_panel_kernel(float* __restrict__ A, int d, int k0, int kb, float* __restrict__ Dinv,
                       PrepHeader* hdr)
 {
-    __shared__ float Ls[kNB][kNB + 1];
-    __shared__ float Xs[kNB][kNB + 1];
-    __shared__ float vec[2][kNB];
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    __shared__ float As[kNB][kNB + 1];
+    __shared__ float Zs[kNB][kNB + 1];
+    __shared__ float Ys[32 * 33];
+    __shared__ int bad_any;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
 
     // diagonal block (lower part); padding beyond kb is the identity
-    float a[4][4];
+    {
+        float tv[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int gi = r0 + i, gj = c0 + j;
-            float v = (gi == gj) ? 1.f : 0.f;
-            if (gi < kb && gj < kb && gj <= gi) v = A[static_cast<int64_t>(k0 + gi) * d + k0 + gj];
-            a[i][j] = v;
+        for (int t = 0; t < 16; ++t) {
+            const int idx = tid + t * 256;
+            const int i = idx / kNB, j = idx % kNB;
+            float v = (i == j) ? 1.f : 0.f;
+            if (i < kb && j < kb && j <= i) v = A[static_cast<int64_t>(k0 + i) * d + k0 + j];
+            tv[t] = v;
         }
-    if (tx == 0)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) vec[0][r0 + i] = a[i][0];
+        for (int t = 0; t < 16; ++t) {
+            const int idx = tid + t * 256;
+            As[idx / kNB][idx % kNB] = tv[t];
+            Zs[idx / kNB][idx % kNB] = 0.f;
+        }
+    }
+    if (tid == 0) bad_any = 0;
     __syncthreads();
-
     bool bad = false;
-    for (int c = 0; c < kNB; ++c) {
-        const float* col = vec[c & 1];
-        float piv = col[c];
-        if (!(piv > 0.f) || !isfinite(piv)) {
-            bad = true;
-            piv = 1.f;
-        }
-        const float rs = rsqrtf(piv);
-        // column c of L for my rows; the trailing update uses only entries
-        // below column c, so the others are multiplied by 0
-        float li[4], lj[4];
+
+    for (int P = 0; P < kNB / 4; ++P) {
+        const int cb = 4 * P;
+        if (warp == 0) {
+            const int ra = cb + lane, rb = cb + lane + 32;
+            float x[4], y[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) li[i] = col[r0 + i] * rs;
+            for (int t = 0; t < 4; ++t) {
+                x[t] = ra < kNB ? As[ra][cb + t] : 0.f;
+                y[t] = rb < kNB ? As[rb][cb + t] : 0.f;
+            }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) lj[j] = (c0 + j > c) ? col[c0 + j] * rs : 0.f;
+            for (int c = 0; c < 4; ++c) {
+                float piv = __shfl_sync(0xffffffffu, x[c], c);
+                if (!(piv > 0.f) || !isfinite(piv)) {
+                    bad = true;
+                    piv = 1.f;
+                }
+                const float rs = rsqrtf(piv);
+                const float lx = x[c] * rs, ly = y[c] * rs;
+                x[c] = lx;
+                y[c] = ly;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) a[i][j] = fmaf(-li[i], lj[j], a[i][j]);
-        if (tx == (c >> 2)) {
-            const int jc = c & 3;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if (r0 + i >= c) {
-                    if (jc == 0) a[i][0] = li[i];
-                    if (jc == 1) a[i][1] = li[i];
-                    if (jc == 2) a[i][2] = li[i];
-                    if (jc == 3) a[i][3] = li[i];
+                for (int j = c + 1; j < 4; ++j) {
+                    const float lj = __shfl_sync(0xffffffffu, lx, j);   // row cb+j, column c
+                    x[j] = fmaf(-lx, lj, x[j]);
+                    y[j] = fmaf(-ly, lj, y[j]);
                 }
             }
-        }
-        const int cn = c + 1;
-        if (cn < kNB && tx == (cn >> 2)) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) vec[cn & 1][r0 + i] = pick4(a[i][0], a[i][1], a[i][2], a[i][3], cn & 3);
+            for (int t = 0; t < 4; ++t) {
+                if (ra < kNB) As[ra][cb + t] = x[t];
+                if (rb < kNB) As[rb][cb + t] = y[t];
+            }
+        }
+        __syncthreads();
+        if (tx > P && ty >= tx) {
+            float li[4][4], lj[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    li[i][t] = As[r0 + i][cb + t];
+                    lj[i][t] = As[c0 + i][cb + t];
+                }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float acc = As[r0 + i][c0 + j];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) acc = fmaf(-li[i][t], lj[j][t], acc);
+                    As[r0 + i][c0 + j] = acc;
+                }
         }
         __syncthreads();
     }
-    if (bad && tid == 0 && blockIdx.x == 0) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Ls[r0 + i][c0 + j] = (c0 + j <= r0 + i) ? a[i][j] : 0.f;
-    __syncthreads();
 
-    // X = L^{-1}: row c of X is final once divided by L[c][c]; then rows > c
-    // subtract L[i][c] X[c][:].
-    float x[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) x[i][j] = (r0 + i == c0 + j) ? 1.f : 0.f;
-    if (ty == 0) {
-        const float inv = 1.f / Ls[0][0];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            x[0][j] *= inv;
-            vec[0][c0 + j] = x[0][j];
-        }
-    }
-    __syncthreads();
-    for (int c = 0; c < kNB; ++c) {
-        float rv[4], lc[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) rv[j] = vec[c & 1][c0 + j];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) lc[i] = (r0 + i > c) ? Ls[r0 + i][c] : 0.f;
+    // Z = L^{-1}: diagonal 4 x 4 inverses
+    if (tid < kNB / 4) {
+        const int o = 4 * tid;
+        float l[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) x[i][j] = fmaf(-lc[i], rv[j], x[i][j]);
-        const int cn = c + 1;
-        if (cn < kNB && ty == (cn >> 2)) {
-            const float inv = 1.f / Ls[cn][cn];
+            for (int j = 0; j < 4; ++j) l[i][j] = (j <= i) ? As[o + i][o + j] : 0.f;
+        float z[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (i == (cn & 3))
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        x[i][j] *= inv;
-                        vec[cn & 1][c0 + j] = x[i][j];
-                    }
+            for (int i = 0; i < 4; ++i) {
+                float acc = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int k = 0; k < i; ++k) acc = fmaf(-l[i][k], (k >= j) ? z[k][j] : 0.f, acc);
+                z[i][j] = (i >= j) ? acc / l[i][i] : 0.f;
+            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) Zs[o + i][o + j] = z[i][j];
+    }
+    __syncthreads();
+    // doubling: pairs of h-blocks at offsets o = p * 2h
+    for (int h = 4; h < kNB; h *= 2) {
+        const int n_out = (kNB / (2 * h)) * h * h;
+        // Y = L21 Z11: Y[i][j] = sum_{k >= j} L[o+h+i][o+k] Z[o+k][o+j]
+        for (int idx = tid; idx < n_out; idx += 256) {
+            const int p = idx / (h * h), rem = idx % (h * h), i = rem / h, j = rem % h;
+            const int o = p * 2 * h;
+            float acc = 0.f;
+            for (int k = j; k < h; ++k) acc = fmaf(As[o + h + i][o + k], Zs[o + k][o + j], acc);
+            Ys[idx] = acc;
+        }
+        __syncthreads();
+        // Z21[i][j] = -sum_{k <= i} Z[o+h+i][o+h+k] Y[k][j]
+        for (int idx = tid; idx < n_out; idx += 256) {
+            const int p = idx / (h * h), rem = idx % (h * h), i = rem / h, j = rem % h;
+            const int o = p * 2 * h;
+            const float* yp = Ys + p * h * h;
+            float acc = 0.f;
+            for (int k = 0; k <= i; ++k) acc = fmaf(Zs[o + h + i][o + h + k], yp[k * h + j], acc);
+            Zs[o + h + i][o + j] = -acc;
         }
         __syncthreads();
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Xs[r0 + i][c0 + j] = x[i][j];
+    if (bad) bad_any = 1;
+    __syncthreads();
+    if (bad_any && tid == 0 && blockIdx.x == 0) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
 
     if (blockIdx.x == 0) {
         // L_kk itself is not needed later (the inverse uses L_kk^{-1} and the
@@ -274,16 +296,14 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int gi = r0 + i, gj = c0 + j;
-                if (gi < kb && gj < kb) Dinv[static_cast<int64_t>(k0 + gi) * kNB + gj] = x[i][j];
+                if (gi < kb && gj < kb) Dinv[static_cast<int64_t>(k0 + gi) * kNB + gj] = Zs[gi][gj];
             }
         return;
     }
 
-    // panel rows: P[i][j] = sum_{k <= j} T[i][k] X[j][k]
+    // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k]
     const int pr0 = k0 + kb + (blockIdx.x - 1) * kNB;
-    __syncthreads();
     {
-        // 64 x 64 tile: 16 loads per thread, all issued before any is used
         float tv[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
@@ -295,7 +315,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
             const int idx = tid + t * 256;
-            Ls[idx / kNB][idx % kNB] = tv[t];
+            As[idx / kNB][idx % kNB] = tv[t];
         }
     }
     __syncthreads();
@@ -303,9 +323,9 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < kNB; ++k) {
         float t[4], xv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = Ls[r0 + i][k];
+        for (int i = 0; i < 4; ++i) t[i] = As[r0 + i][k];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) xv[j] = Xs[c0 + j][k];
+        for (int j = 0; j < 4; ++j) xv[j] = Zs[c0 + j][k];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
