@@ -171,9 +171,9 @@ int gptq_quantize(float *W, const float *Hinv_chol, const int32_t *perm, int64_t
                   float *err_sq, void *workspace, size_t ws_bytes, void *stream);
 
 /* Size of the fixed device array that gptq_quantize_static_scratch works in:
- * 96 MiB.  Every GPU on which the library's device code is loaded holds it
+ * 128 MiB.  Every GPU on which the library's device code is loaded holds it
  * from then until the process exits. */
-#define GPTQ_STATIC_SCRATCH_BYTES ((size_t)96 << 20)
+#define GPTQ_STATIC_SCRATCH_BYTES ((size_t)128 << 20)
 
 /*
  * gptq_quantize with no workspace argument, for callers that cannot allocate
@@ -187,7 +187,7 @@ int gptq_quantize(float *W, const float *Hinv_chol, const int32_t *perm, int64_t
  * a fixed array inside the library (GPTQ_STATIC_SCRATCH_BYTES), so the call
  * allocates nothing.  Limits and rules:
  *   - A layer whose working set exceeds the array (about 5 bytes per weight
- *     plus 512 bytes per output row: 4096 x 4096 needs about 82 MiB and fits,
+ *     plus 4 KiB per output row: 4096 x 4096 needs about 96 MiB and fits,
  *     4096 x 11008 does not) is refused with GPTQ_ERR_WORKSPACE before the
  *     device is touched.
  *   - The first call on each device looks up the array's device address with

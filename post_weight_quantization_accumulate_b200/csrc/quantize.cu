@@ -25,6 +25,7 @@ namespace gptq {
 namespace {
 
 constexpr int QB = 128;           // largest block width
+constexpr int kOuterMax = 1024;   // widest outer window of the two-level lazy batch
 constexpr int QTPR = 8;           // threads per row
 constexpr int QCPT = QB / QTPR;   // registers per thread (column 8m + p belongs to part p)
 constexpr int QSUB = 16;          // columns per unrolled sub-block
@@ -46,7 +47,8 @@ struct QArgs {
     float* scales;        // [d_out][n_groups]
     float* zeros;
     uint8_t* codes_p;     // [d_out][d_in], processing order
-    float* E;             // [d_out][QB]
+    float* E;             // [d_out][kOuterMax] errors of the current outer window
+    int e_off;            // column of this block inside the outer window
     float* err_sq;        // [d_out] or null
 };
 
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
         const int rl = idx / QB, c = idx % QB;
         const int rr = blockIdx.x * QROWS + rl;
         if (rr < a.d_out && c < bw) {
-            a.E[static_cast<int64_t>(rr) * QB + c] = Es[rl * ES_LD + c];
+            a.E[static_cast<int64_t>(rr) * kOuterMax + a.e_off + c] = Es[rl * ES_LD + c];
             a.codes_p[static_cast<int64_t>(rr) * d_in + j0 + c] = Cs[rl * ES_LD + c];
         }
     }
@@ -422,7 +424,7 @@ size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
 {
     const size_t n = static_cast<size_t>(d_out) * static_cast<size_t>(d_in);
     return 256 + up256(n * sizeof(float)) + up256(n) +
-           up256(static_cast<size_t>(d_out) * QB * sizeof(float)) +
+           up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)) +
            up256(static_cast<size_t>(d_in) * sizeof(int32_t));
 }
 
@@ -438,7 +440,7 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
     uint8_t* codes_p = ws + 256 + up256(n * sizeof(float));
     float* E = reinterpret_cast<float*>(ws + 256 + up256(n * sizeof(float)) + up256(n));
     int32_t* inv = reinterpret_cast<int32_t*>(ws + 256 + up256(n * sizeof(float)) + up256(n) +
-                                              up256(static_cast<size_t>(d_out) * QB * sizeof(float)));
+                                              up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)));
     const int nsm = sm_count();
     int* status = device_status_ptr();
     const int n_groups = gs > 0 ? d_in / gs : 1;
@@ -476,21 +478,42 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
                                                                        scales, zeros);
         GPTQ_LAUNCH_CHECK();
     }
+    // Two-level lazy batch: a block's errors correct the rest of its outer
+    // window right away (K = block), and the columns beyond the window once
+    // per window (K = window width).  A group wider than a block must lie in
+    // one window; groups wider than kOuterMax use one level.
+    int outer;
+    if (gs > kOuterMax)
+        outer = block;
+    else if (gs > block)
+        outer = (kOuterMax / gs) * gs;
+    else
+        outer = (kOuterMax / block) * block;
     const int grid = (d_out + QROWS - 1) / QROWS;
-    for (int j0 = 0; j0 < d_in; j0 += block) {
-        const int bw = (d_in - j0 < block) ? d_in - j0 : block;
-        QArgs a{work, U, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
-                codes_p, E, err_sq};
-        if (groups_in_step)
-            gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
-        else
-            gptq_block_kernel<false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
-        GPTQ_LAUNCH_CHECK();
-        const int rest = d_in - j0 - bw;
+    for (int J0 = 0; J0 < d_in; J0 += outer) {
+        const int J1 = (d_in - J0 < outer) ? d_in : J0 + outer;
+        for (int j0 = J0; j0 < J1; j0 += block) {
+            const int bw = (J1 - j0 < block) ? J1 - j0 : block;
+            QArgs a{work, U, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
+                    codes_p, E, j0 - J0, err_sq};
+            if (groups_in_step)
+                gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+            else
+                gptq_block_kernel<false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+            GPTQ_LAUNCH_CHECK();
+            const int rest_in = J1 - j0 - bw;
+            if (rest_in > 0) {
+                int rc = launch_sgemm(false, d_out, rest_in, bw, -1.f, E + (j0 - J0), kOuterMax, 0,
+                                      U + static_cast<int64_t>(j0) * d_in + j0 + bw, d_in, 0, 1.f,
+                                      work + j0 + bw, d_in, 0, 1, 0, stream);
+                if (rc) return rc;
+            }
+        }
+        const int rest = d_in - J1;
         if (rest > 0) {
-            int rc = launch_sgemm(false, d_out, rest, bw, -1.f, E, QB, 0,
-                                  U + static_cast<int64_t>(j0) * d_in + j0 + bw, d_in, 0, 1.f,
-                                  work + j0 + bw, d_in, 0, 1, 0, stream);
+            int rc = launch_sgemm(false, d_out, rest, J1 - J0, -1.f, E, kOuterMax, 0,
+                                  U + static_cast<int64_t>(J0) * d_in + J1, d_in, 0, 1.f,
+                                  work + J1, d_in, 0, 1, 0, stream);
             if (rc) return rc;
         }
     }
