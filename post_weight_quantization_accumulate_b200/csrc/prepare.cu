@@ -16,6 +16,7 @@
 #include "gemm.cuh"
 
 #include <algorithm>
+#include <mutex>
 
 namespace gptq {
 
@@ -145,38 +146,89 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
 // lower triangle (thread (ty, tx) owns the 4 x 4 tile rows 4ty.., cols 4tx..).
 // Inverse Z = L^{-1} by recursive doubling: the 16 diagonal 4 x 4 inverses,
 // then Z21 = -Z22 (L21 Z11) for block sizes 8, 16, 32, 64.
-__global__ void __launch_bounds__(256)
-    chol_panel_kernel(float* __restrict__ A, int d, int k0, int kb, float* __restrict__ Dinv,
-                      PrepHeader* hdr)
+typedef float Tile64[kNB + 1];
+constexpr size_t kPanelSmem = (4 * kNB * (kNB + 1) + 32 * 33) * sizeof(float) + 16;
+
+// acc[i][j] (tile rows 4ty.., cols 4tx..) -= X[rows] . Y[cols] over 64 columns:
+// the rank-64 correction of the previous panel applied on the fly.
+__device__ __forceinline__ void tile_minus_xyT(float (&acc)[4][4], const Tile64* X, const Tile64* Y,
+                                               int r0, int c0)
 {
-    __shared__ float As[kNB][kNB + 1];
-    __shared__ float Zs[kNB][kNB + 1];
-    __shared__ float Ys[32 * 33];
-    __shared__ int bad_any;
+    for (int k = 0; k < kNB; ++k) {
+        float xv[4], yv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[i] = X[r0 + i][k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) yv[j] = Y[c0 + j][k];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(-xv[i], yv[j], acc[i][j]);
+    }
+}
+
+// 64 x 64 tile of A (rows r_begin.., columns c_begin..c_begin+ncols) into smem;
+// rows >= d or columns >= ncols read as `pad` on the diagonal, 0 elsewhere
+// (lower_only: entries above the diagonal read as 0 too).
+__device__ __forceinline__ void load_tile(Tile64* dst, const float* A, int d, int r_begin, int nrows,
+                                          int c_begin, int ncols, bool lower_only, bool pad_identity)
+{
+    const int tid = threadIdx.x;
+    float tv[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        float v = (pad_identity && i == j) ? 1.f : 0.f;
+        if (i < nrows && j < ncols && (!lower_only || j <= i))
+            v = A[static_cast<int64_t>(r_begin + i) * d + c_begin + j];
+        tv[t] = v;
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        dst[idx / kNB][idx % kNB] = tv[t];
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    chol_panel_kernel(float* __restrict__ A, int d, int k0, int kb, int pk0,
+                      float* __restrict__ Dinv, PrepHeader* hdr)
+{
+    extern __shared__ __align__(16) float psm[];
+    Tile64* As = reinterpret_cast<Tile64*>(psm);
+    Tile64* Zs = As + kNB;
+    Tile64* Pd = Zs + kNB;       // previous panel, rows of this diagonal block
+    Tile64* Pr = Pd + kNB;       // previous panel, rows of this CTA's panel block
+    float* Ys = reinterpret_cast<float*>(Pr + kNB);
+    int& bad_any = *reinterpret_cast<int*>(Ys + 32 * 33);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
 
     // diagonal block (lower part); padding beyond kb is the identity
-    {
-        float tv[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int idx = tid + t * 256;
-            const int i = idx / kNB, j = idx % kNB;
-            float v = (i == j) ? 1.f : 0.f;
-            if (i < kb && j < kb && j <= i) v = A[static_cast<int64_t>(k0 + i) * d + k0 + j];
-            tv[t] = v;
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int idx = tid + t * 256;
-            As[idx / kNB][idx % kNB] = tv[t];
-            Zs[idx / kNB][idx % kNB] = 0.f;
-        }
-    }
+    load_tile(As, A, d, k0, kb, k0, kb, true, true);
+    for (int idx = tid; idx < kNB * kNB; idx += 256) Zs[idx / kNB][idx % kNB] = 0.f;
+    if (pk0 >= 0) load_tile(Pd, A, d, k0, kb, pk0, kNB, false, false);
     if (tid == 0) bad_any = 0;
     __syncthreads();
+    if (pk0 >= 0) {
+        // A_kk -= P_prev,kk P_prev,kk^T (the previous panel's correction of
+        // this block column is applied here rather than in memory)
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = As[r0 + i][c0 + j];
+        if (ty >= tx) tile_minus_xyT(acc, Pd, Pd, r0, c0);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (c0 + j <= r0 + i) As[r0 + i][c0 + j] = acc[i][j];
+        __syncthreads();
+    }
     bool bad = false;
 
     for (int P = 0; P < kNB / 4; ++P) {
@@ -301,24 +353,27 @@ __global__ void __launch_bounds__(256)
         return;
     }
 
-    // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k]
+    // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k], with
+    // T = A[rows][block] - P_prev[rows] P_prev,kk^T
     const int pr0 = k0 + kb + (blockIdx.x - 1) * kNB;
-    {
-        float tv[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int idx = tid + t * 256;
-            const int i = idx / kNB, j = idx % kNB;
-            const int r = pr0 + i;
-            tv[t] = (r < d && j < kb) ? A[static_cast<int64_t>(r) * d + k0 + j] : 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int idx = tid + t * 256;
-            As[idx / kNB][idx % kNB] = tv[t];
-        }
-    }
+    const int prn = min(kNB, d - pr0);
+    load_tile(As, A, d, pr0, prn, k0, kb, false, false);
+    if (pk0 >= 0) load_tile(Pr, A, d, pr0, prn, pk0, kNB, false, false);
     __syncthreads();
+    if (pk0 >= 0) {
+        float t4[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) t4[i][j] = As[r0 + i][c0 + j];
+        tile_minus_xyT(t4, Pr, Pd, r0, c0);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = (c0 + j < kb) ? t4[i][j] : 0.f;
+        __syncthreads();
+    }
     float acc[4][4] = {};
     for (int k = 0; k < kNB; ++k) {
         float t[4], xv[4];
@@ -365,6 +420,36 @@ __global__ void reverse_upper_kernel(const float* __restrict__ Minv, int d, floa
 
 }  // namespace
 
+// Second stream of the factorisation (one per device, created on first use)
+// with its events; the caller's stream forks to it and joins it again.
+struct SideStream {
+    static constexpr int kRing = 4;
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, done_panel = nullptr;
+    cudaEvent_t ev[kRing] = {};
+};
+
+static int side_stream(SideStream** out)
+{
+    static SideStream streams[64];
+    static std::mutex mu;
+    int dev = 0;
+    GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return GPTQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(mu);
+    SideStream& st = streams[dev];
+    if (!st.s) {
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithFlags(&st.s, cudaStreamNonBlocking));
+        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming));
+        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming));
+        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.done_panel, cudaEventDisableTiming));
+        for (int i = 0; i < SideStream::kRing; ++i)
+            GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.ev[i], cudaEventDisableTiming));
+    }
+    *out = &st;
+    return GPTQ_OK;
+}
+
 int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t* perm, float* U,
                 void* workspace, cudaStream_t stream, int* host_status)
 {
@@ -399,19 +484,50 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     }
     GPTQ_LAUNCH_CHECK();
 
-    // blocked right-looking Cholesky, A = M M^T (lower)
-    for (int k0 = 0; k0 < d; k0 += kNB) {
+    // Blocked right-looking Cholesky, A = M M^T (lower), with look-ahead:
+    // panel k+1 applies panel k's correction to its own block column on the
+    // fly; the correction of everything right of block column k+1 (the large
+    // symmetric update) runs on a side stream and is waited for only by panel
+    // k+2.  The critical path is the chain of panel kernels.
+    SideStream* side = nullptr;
+    int rc = side_stream(&side);
+    if (rc) return rc;
+    const int n_panels = (d + kNB - 1) / kNB;
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->fork, stream));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->fork, 0));
+    {
+        static bool attr_panel[64] = {};
+        int dev = 0;
+        GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
+        if (dev < 64 && !attr_panel[dev]) {
+            GPTQ_CUDA_CHECK(cudaFuncSetAttribute(chol_panel_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kPanelSmem)));
+            attr_panel[dev] = true;
+        }
+    }
+    for (int p = 0; p < n_panels; ++p) {
+        const int k0 = p * kNB;
         const int kb = std::min(kNB, d - k0);
         const int rest = d - k0 - kb;
-        chol_panel_kernel<<<1 + (rest + kNB - 1) / kNB, 256, 0, stream>>>(A, d, k0, kb, Dinv, hdr);
+        if (p >= 2) GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev[(p - 2) % SideStream::kRing], 0));
+        chol_panel_kernel<<<1 + (rest + kNB - 1) / kNB, 256, kPanelSmem, stream>>>(
+            A, d, k0, kb, p > 0 ? k0 - kNB : -1, Dinv, hdr);
         GPTQ_LAUNCH_CHECK();
-        if (rest <= 0) break;
-        float* P = A + static_cast<int64_t>(k0 + kb) * d + k0;
-        float* C = A + static_cast<int64_t>(k0 + kb) * d + k0 + kb;
-        int rc = launch_sgemm(true, rest, rest, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,
-                              kGemmLowerC, stream);
-        if (rc) return rc;
+        const int rest2 = rest - kNB;   // rows/columns right of block column p+1
+        if (rest2 > 0) {
+            GPTQ_CUDA_CHECK(cudaEventRecord(side->done_panel, stream));
+            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->done_panel, 0));
+            float* P = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0;
+            float* C = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0 + kb + kNB;
+            rc = launch_sgemm(true, rest2, rest2, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,
+                              kGemmLowerC, side->s);
+            if (rc) return rc;
+        }
+        GPTQ_CUDA_CHECK(cudaEventRecord(side->ev[p % SideStream::kRing], side->s));
     }
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->join, side->s));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join, 0));
 
     // M^{-1}: leaves from Dinv, then recursive doubling
     //   [A 0; B C]^{-1} = [A^-1 0; -C^-1 B A^-1  C^-1]
