@@ -17,16 +17,20 @@ enum GemmFlags : int {
 // Runs on the tensor cores (3xTF32, gemm_tc.cu) whenever A and B are 16-byte
 // aligned with leading dimensions and batch strides that are multiples of 4
 // floats (the TMA rules), else on the SIMT kernel (gemm_simt.cu).
+// max_ctas > 0 caps the number of CTAs (and so of SMs) the product occupies,
+// which leaves SMs free for latency-critical work on another stream.
 int launch_sgemm(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                  int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
-                 int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream);
+                 int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream,
+                 int max_ctas = 0);
 
 int launch_sgemm_simt(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                       int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                       int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream);
 int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                    int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
-                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream);
+                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream,
+                   int max_ctas = 0);
 bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, int64_t ldb,
                        int64_t sB, int batch);
 

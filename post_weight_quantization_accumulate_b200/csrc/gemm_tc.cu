@@ -356,7 +356,7 @@ bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, 
 
 int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                    int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
-                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream)
+                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream, int max_ctas)
 {
     if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
     static bool attr_set[64] = {};
@@ -392,7 +392,9 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     g.n_nt = (N + TBN - 1) / TBN;
     g.status = device_status_ptr();
     const int64_t units = static_cast<int64_t>(g.n_mt) * g.n_nt * batch;
-    const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
+    int cap = sm_count();
+    if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;
+    const int grid = static_cast<int>(units < cap ? units : cap);
     gemm_tc_kernel<<<grid, TTHREADS, GEMM_SMEM, stream>>>(mA, mB, g);
     GPTQ_LAUNCH_CHECK();
     return GPTQ_OK;

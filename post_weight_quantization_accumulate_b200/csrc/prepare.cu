@@ -33,8 +33,7 @@ size_t prepare_workspace_bytes(int64_t d)
 {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t dd = static_cast<size_t>(d) * static_cast<size_t>(d) * sizeof(float);
-    return 256 + up(dd) /*A,M*/ + up(dd) /*Minv*/ + up(dd) /*T*/ +
-           up(static_cast<size_t>(d) * kNB * sizeof(float)) /*Dinv*/;
+    return 256 + up(dd) /*A,M*/ + up(dd) /*Minv*/ + up(dd) /*T*/;
 }
 
 namespace {
@@ -138,7 +137,7 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
 // One panel step of the blocked Cholesky, fused:
 //   every CTA factors the kb x kb diagonal block at (k0, k0) (redundantly, so
 //   no other launch has to wait for it) and inverts the factor; CTA 0 writes
-//   L_kk^{-1} into Dinv[k0 .. k0+kb); CTA b >= 1 solves the panel rows
+//   L_kk^{-1} into M^{-1}; CTA b >= 1 solves the panel rows
 //   k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T}.
 // Factorisation of the 64 x 64 block in shared memory, in 16 strips of 4
 // columns: warp 0 factors the strip with shuffles (lane l holds rows 4P+l and
@@ -193,7 +192,7 @@ __device__ __forceinline__ void load_tile(Tile64* dst, const float* A, int d, in
 
 __global__ void __launch_bounds__(256)
     chol_panel_kernel(float* __restrict__ A, int d, int k0, int kb, int pk0,
-                      float* __restrict__ Dinv, PrepHeader* hdr)
+                      float* __restrict__ Minv, PrepHeader* hdr)
 {
     extern __shared__ __align__(16) float psm[];
     Tile64* As = reinterpret_cast<Tile64*>(psm);
@@ -342,14 +341,55 @@ __global__ void __launch_bounds__(256)
     if (blockIdx.x == 0) {
         // L_kk itself is not needed later (the inverse uses L_kk^{-1} and the
         // off-diagonal panels), and the other CTAs of this launch may still be
-        // reading the diagonal block of A, so only Dinv is written.
+        // reading the diagonal block of A, so only M^{-1} is written: its
+        // diagonal block, and for an odd panel also the block left of it,
+        //   M^{-1}[k, k-1] = -Z_kk (M[k, k-1] Z_{k-1,k-1})
+        // (first level of the recursive inverse; M[k, k-1] is Pd).
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int gi = r0 + i, gj = c0 + j;
-                if (gi < kb && gj < kb) Dinv[static_cast<int64_t>(k0 + gi) * kNB + gj] = Zs[gi][gj];
+                if (gi < kb && gj < kb) Minv[static_cast<int64_t>(k0 + gi) * d + k0 + gj] = Zs[gi][gj];
             }
+        if (pk0 >= 0 && ((k0 / kNB) & 1)) {
+            load_tile(Pr, Minv, d, pk0, kNB, pk0, kNB, true, false);   // Z_{k-1,k-1}
+            __syncthreads();
+            float y[4][4] = {};
+            for (int k = 0; k < kNB; ++k) {
+                float a4[4], b4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a4[i] = Pd[r0 + i][k];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) b4[j] = Pr[k][c0 + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) y[i][j] = fmaf(a4[i], b4[j], y[i][j]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = y[i][j];
+            __syncthreads();
+            float x[4][4] = {};
+            for (int k = 0; k < kNB; ++k) {
+                float a4[4], b4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a4[i] = Zs[r0 + i][k];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) b4[j] = As[k][c0 + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) x[i][j] = fmaf(a4[i], b4[j], x[i][j]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (r0 + i < kb) Minv[static_cast<int64_t>(k0 + r0 + i) * d + pk0 + c0 + j] = -x[i][j];
+        }
         return;
     }
 
@@ -395,18 +435,6 @@ __global__ void __launch_bounds__(256)
         }
 }
 
-// Minv diagonal blocks from Dinv.
-__global__ void place_dinv_kernel(float* __restrict__ Minv, int d, const float* __restrict__ Dinv)
-{
-    const int64_t n = static_cast<int64_t>(d) * kNB;
-    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int r = static_cast<int>(idx / kNB), j = static_cast<int>(idx % kNB);
-        const int c = (r / kNB) * kNB + j;
-        if (c < d && j <= r % kNB) Minv[static_cast<int64_t>(r) * d + c] = Dinv[idx];
-    }
-}
-
 // U[i][j] = Minv[d-1-i][d-1-j] for i <= j, 0 below the diagonal.
 __global__ void reverse_upper_kernel(const float* __restrict__ Minv, int d, float* __restrict__ U)
 {
@@ -424,8 +452,9 @@ __global__ void reverse_upper_kernel(const float* __restrict__ Minv, int d, floa
 // with its events; the caller's stream forks to it and joins it again.
 struct SideStream {
     static constexpr int kRing = 4;
-    cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr, done_panel = nullptr;
+    cudaStream_t s = nullptr;          // trailing symmetric updates
+    cudaStream_t s2 = nullptr;         // levels >= 256 of the recursive inverse
+    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr, done_panel = nullptr;
     cudaEvent_t ev[kRing] = {};
 };
 
@@ -439,9 +468,14 @@ static int side_stream(SideStream** out)
     std::lock_guard<std::mutex> lk(mu);
     SideStream& st = streams[dev];
     if (!st.s) {
-        GPTQ_CUDA_CHECK(cudaStreamCreateWithFlags(&st.s, cudaStreamNonBlocking));
+        // lowest priority: CTAs of the panel chain are placed first on free SMs
+        int lo = 0, hi = 0;
+        GPTQ_CUDA_CHECK(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s, cudaStreamNonBlocking, lo));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s2, cudaStreamNonBlocking, lo));
         GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming));
         GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming));
+        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join2, cudaEventDisableTiming));
         GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.done_panel, cudaEventDisableTiming));
         for (int i = 0; i < SideStream::kRing; ++i)
             GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.ev[i], cudaEventDisableTiming));
@@ -461,7 +495,6 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     float* A = reinterpret_cast<float*>(ws + 256);
     float* Minv = reinterpret_cast<float*>(ws + 256 + up(dd));
     float* T = reinterpret_cast<float*>(ws + 256 + 2 * up(dd));
-    float* Dinv = reinterpret_cast<float*>(ws + 256 + 3 * up(dd));
     const int nsm = sm_count();
 
     GPTQ_CUDA_CHECK(cudaMemsetAsync(hdr, 0, sizeof(PrepHeader), stream));
@@ -493,8 +526,15 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     int rc = side_stream(&side);
     if (rc) return rc;
     const int n_panels = (d + kNB - 1) / kNB;
+    // M^{-1} by recursive doubling,
+    //   [A 0; B C]^{-1} = [A^-1 0; -C^-1 B A^-1  C^-1],
+    // grown as the factorisation advances: the 64-blocks and the first level
+    // come from the panel kernels, pairs of level s >= 256 run on the second
+    // side stream as soon as the panels they cover are done.
+    GPTQ_CUDA_CHECK(cudaMemsetAsync(Minv, 0, dd, stream));
     GPTQ_CUDA_CHECK(cudaEventRecord(side->fork, stream));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->fork, 0));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->fork, 0));
     {
         static bool attr_panel[64] = {};
         int dev = 0;
@@ -508,56 +548,63 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     }
     for (int p = 0; p < n_panels; ++p) {
         const int k0 = p * kNB;
+        // SMs the side products may hold: the rest after this panel's CTAs
+        const int side_ctas = std::max(16, nsm - (1 + (d - k0 + kNB - 1) / kNB));
         const int kb = std::min(kNB, d - k0);
         const int rest = d - k0 - kb;
         if (p >= 2) GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev[(p - 2) % SideStream::kRing], 0));
         chol_panel_kernel<<<1 + (rest + kNB - 1) / kNB, 256, kPanelSmem, stream>>>(
-            A, d, k0, kb, p > 0 ? k0 - kNB : -1, Dinv, hdr);
+            A, d, k0, kb, p > 0 ? k0 - kNB : -1, Minv, hdr);
         GPTQ_LAUNCH_CHECK();
+        GPTQ_CUDA_CHECK(cudaEventRecord(side->done_panel, stream));
+        // inverse pairs that end with this panel: level s covers [end - s, end)
+        const int end = k0 + kb;
+        if (kb == kNB) {
+            bool waited = false;
+            for (int sz = 4 * kNB; sz <= end; sz *= 2) {
+                if (end % sz) break;
+                if (!waited) {
+                    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->done_panel, 0));
+                    waited = true;
+                }
+                const int o = end - sz, h = sz / 2;
+                rc = launch_sgemm(false, h, h, h, 1.f, A + static_cast<int64_t>(o + h) * d + o, d, 0,
+                                  Minv + static_cast<int64_t>(o) * d + o, d, 0, 0.f, T, h, 0, 1,
+                                  kGemmLowerB, side->s2, side_ctas);
+                if (rc) return rc;
+                rc = launch_sgemm(false, h, h, h, -1.f, Minv + static_cast<int64_t>(o + h) * d + o + h, d,
+                                  0, T, h, 0, 0.f, Minv + static_cast<int64_t>(o + h) * d + o, d, 0, 1,
+                                  kGemmLowerA, side->s2, side_ctas);
+                if (rc) return rc;
+            }
+        }
         const int rest2 = rest - kNB;   // rows/columns right of block column p+1
         if (rest2 > 0) {
-            GPTQ_CUDA_CHECK(cudaEventRecord(side->done_panel, stream));
             GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->done_panel, 0));
             float* P = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0;
             float* C = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0 + kb + kNB;
             rc = launch_sgemm(true, rest2, rest2, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,
-                              kGemmLowerC, side->s);
+                              kGemmLowerC, side->s, side_ctas);
             if (rc) return rc;
         }
         GPTQ_CUDA_CHECK(cudaEventRecord(side->ev[p % SideStream::kRing], side->s));
     }
     GPTQ_CUDA_CHECK(cudaEventRecord(side->join, side->s));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join, 0));
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->join2, side->s2));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join2, 0));
 
-    // M^{-1}: leaves from Dinv, then recursive doubling
-    //   [A 0; B C]^{-1} = [A^-1 0; -C^-1 B A^-1  C^-1]
-    GPTQ_CUDA_CHECK(cudaMemsetAsync(Minv, 0, dd, stream));
-    place_dinv_kernel<<<nsm * 4, 256, 0, stream>>>(Minv, d, Dinv);
-    GPTQ_LAUNCH_CHECK();
-    for (int s = 2 * kNB; s / 2 < d; s *= 2) {
+    // Ragged pairs of the recursive inverse (sizes that are not a power of two
+    // times 64); level 128 was completed by the panel kernels.
+    for (int s = 4 * kNB; s / 2 < d; s *= 2) {
         const int h = s / 2;
-        const int nfull = d / s;               // subproblems of full size s
-        // full-size subproblems, batched
-        if (nfull > 0) {
-            const int64_t stride = static_cast<int64_t>(s) * d + s;  // diagonal step
-            int rc = launch_sgemm(false, h, h, h, 1.f, A + static_cast<int64_t>(h) * d, d, stride,
-                                  Minv, d, stride, 0.f, T, h, static_cast<int64_t>(h) * h, nfull,
-                                  kGemmLowerB, stream);
-            if (rc) return rc;
-            rc = launch_sgemm(false, h, h, h, -1.f, Minv + static_cast<int64_t>(h) * d + h, d,
-                              stride, T, h, static_cast<int64_t>(h) * h, 0.f,
-                              Minv + static_cast<int64_t>(h) * d, d, stride, nfull, kGemmLowerA,
-                              stream);
-            if (rc) return rc;
-        }
-        // ragged tail subproblem: offset o = nfull * s, size d - o > h
-        const int o = nfull * s;
+        const int o = (d / s) * s;
         const int m2 = d - o - h;
         if (m2 > 0) {
             const float* Bo = A + static_cast<int64_t>(o + h) * d + o;
             const float* Ai = Minv + static_cast<int64_t>(o) * d + o;
-            int rc = launch_sgemm(false, m2, h, h, 1.f, Bo, d, 0, Ai, d, 0, 0.f, T, h, 0, 1,
-                                  kGemmLowerB, stream);
+            rc = launch_sgemm(false, m2, h, h, 1.f, Bo, d, 0, Ai, d, 0, 0.f, T, h, 0, 1,
+                              kGemmLowerB, stream);
             if (rc) return rc;
             const float* Ci = Minv + static_cast<int64_t>(o + h) * d + o + h;
             rc = launch_sgemm(false, m2, h, m2, -1.f, Ci, d, 0, T, h, 0, 0.f,
