@@ -230,42 +230,79 @@ __global__ void __launch_bounds__(256)
     }
     bool bad = false;
 
+    // Strips of 4 columns with look-ahead: while warps 1-7 subtract strip P's
+    // rank-4 product from the columns right of strip P+1, warp 0 applies it to
+    // strip P+1 itself and factors that strip, so each strip costs one barrier
+    // and the long update is off the chain.  Warp 0 keeps rows 4P+l and
+    // 4P+l+32 of a strip in registers (lane l).
+    auto factor_strip = [&](int cb, float (&x)[4], float (&y)[4]) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float piv = __shfl_sync(0xffffffffu, x[c], c);
+            if (!(piv > 0.f) || !isfinite(piv)) {
+                bad = true;
+                piv = 1.f;
+            }
+            const float rs = rsqrtf(piv);
+            const float lx = x[c] * rs, ly = y[c] * rs;
+            x[c] = lx;
+            y[c] = ly;
+#pragma unroll
+            for (int j = c + 1; j < 4; ++j) {
+                const float lj = __shfl_sync(0xffffffffu, lx, j);   // row cb+j, column c
+                x[j] = fmaf(-lx, lj, x[j]);
+                y[j] = fmaf(-ly, lj, y[j]);
+            }
+        }
+        const int ra = cb + lane, rb = cb + lane + 32;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if (ra < kNB) As[ra][cb + t] = x[t];
+            if (rb < kNB) As[rb][cb + t] = y[t];
+        }
+    };
+    if (warp == 0) {
+        float x[4], y[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            x[t] = As[lane][t];
+            y[t] = As[lane + 32][t];
+        }
+        factor_strip(0, x, y);
+    }
+    __syncthreads();
     for (int P = 0; P < kNB / 4; ++P) {
         const int cb = 4 * P;
         if (warp == 0) {
-            const int ra = cb + lane, rb = cb + lane + 32;
-            float x[4], y[4];
+            if (P + 1 < kNB / 4) {
+                const int nb = cb + 4;
+                const int ra = nb + lane, rb = nb + lane + 32;
+                float lstrip[4][4];   // L[nb + t][cb + u]
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                x[t] = ra < kNB ? As[ra][cb + t] : 0.f;
-                y[t] = rb < kNB ? As[rb][cb + t] : 0.f;
-            }
+                for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float piv = __shfl_sync(0xffffffffu, x[c], c);
-                if (!(piv > 0.f) || !isfinite(piv)) {
-                    bad = true;
-                    piv = 1.f;
+                    for (int u = 0; u < 4; ++u) lstrip[t][u] = As[nb + t][cb + u];
+                float x[4], y[4], la[4], lb[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    la[u] = ra < kNB ? As[ra][cb + u] : 0.f;
+                    lb[u] = rb < kNB ? As[rb][cb + u] : 0.f;
                 }
-                const float rs = rsqrtf(piv);
-                const float lx = x[c] * rs, ly = y[c] * rs;
-                x[c] = lx;
-                y[c] = ly;
 #pragma unroll
-                for (int j = c + 1; j < 4; ++j) {
-                    const float lj = __shfl_sync(0xffffffffu, lx, j);   // row cb+j, column c
-                    x[j] = fmaf(-lx, lj, x[j]);
-                    y[j] = fmaf(-ly, lj, y[j]);
+                for (int t = 0; t < 4; ++t) {
+                    float xa = ra < kNB ? As[ra][nb + t] : 0.f;
+                    float ya = rb < kNB ? As[rb][nb + t] : 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        xa = fmaf(-la[u], lstrip[t][u], xa);
+                        ya = fmaf(-lb[u], lstrip[t][u], ya);
+                    }
+                    x[t] = xa;
+                    y[t] = ya;
                 }
+                factor_strip(nb, x, y);
             }
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                if (ra < kNB) As[ra][cb + t] = x[t];
-                if (rb < kNB) As[rb][cb + t] = y[t];
-            }
-        }
-        __syncthreads();
-        if (tx > P && ty >= tx) {
+        } else if (tx > P + 1 && ty >= tx) {
             float li[4][4], lj[4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -311,26 +348,51 @@ __global__ void __launch_bounds__(256)
             for (int j = 0; j < 4; ++j) Zs[o + i][o + j] = z[i][j];
     }
     __syncthreads();
-    // doubling: pairs of h-blocks at offsets o = p * 2h
+    // doubling: pairs of h-blocks at offsets o = p * 2h; every thread owns
+    // 2 x 2 output tiles (four independent accumulators)
     for (int h = 4; h < kNB; h *= 2) {
-        const int n_out = (kNB / (2 * h)) * h * h;
+        const int hh = h / 2;
+        const int n_tiles = (kNB / (2 * h)) * hh * hh;
         // Y = L21 Z11: Y[i][j] = sum_{k >= j} L[o+h+i][o+k] Z[o+k][o+j]
-        for (int idx = tid; idx < n_out; idx += 256) {
-            const int p = idx / (h * h), rem = idx % (h * h), i = rem / h, j = rem % h;
+        for (int t = tid; t < n_tiles; t += 256) {
+            const int p = t / (hh * hh), rem = t % (hh * hh);
+            const int i = 2 * (rem / hh), j = 2 * (rem % hh);
             const int o = p * 2 * h;
-            float acc = 0.f;
-            for (int k = j; k < h; ++k) acc = fmaf(As[o + h + i][o + k], Zs[o + k][o + j], acc);
-            Ys[idx] = acc;
+            float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+            for (int k = j; k < h; ++k) {
+                const float a0 = As[o + h + i][o + k], a1 = As[o + h + i + 1][o + k];
+                const float b0 = Zs[o + k][o + j], b1 = Zs[o + k][o + j + 1];
+                y00 = fmaf(a0, b0, y00);
+                y01 = fmaf(a0, b1, y01);
+                y10 = fmaf(a1, b0, y10);
+                y11 = fmaf(a1, b1, y11);
+            }
+            float* yp = Ys + p * h * h;
+            yp[i * h + j] = y00;
+            yp[i * h + j + 1] = y01;
+            yp[(i + 1) * h + j] = y10;
+            yp[(i + 1) * h + j + 1] = y11;
         }
         __syncthreads();
         // Z21[i][j] = -sum_{k <= i} Z[o+h+i][o+h+k] Y[k][j]
-        for (int idx = tid; idx < n_out; idx += 256) {
-            const int p = idx / (h * h), rem = idx % (h * h), i = rem / h, j = rem % h;
+        for (int t = tid; t < n_tiles; t += 256) {
+            const int p = t / (hh * hh), rem = t % (hh * hh);
+            const int i = 2 * (rem / hh), j = 2 * (rem % hh);
             const int o = p * 2 * h;
             const float* yp = Ys + p * h * h;
-            float acc = 0.f;
-            for (int k = 0; k <= i; ++k) acc = fmaf(Zs[o + h + i][o + h + k], yp[k * h + j], acc);
-            Zs[o + h + i][o + j] = -acc;
+            float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
+            for (int k = 0; k <= i + 1; ++k) {
+                const float a0 = Zs[o + h + i][o + h + k], a1 = Zs[o + h + i + 1][o + h + k];
+                const float b0 = yp[k * h + j], b1 = yp[k * h + j + 1];
+                z00 = fmaf(a0, b0, z00);
+                z01 = fmaf(a0, b1, z01);
+                z10 = fmaf(a1, b0, z10);
+                z11 = fmaf(a1, b1, z11);
+            }
+            Zs[o + h + i][o + j] = -z00;
+            Zs[o + h + i][o + j + 1] = -z01;
+            Zs[o + h + i + 1][o + j] = -z10;
+            Zs[o + h + i + 1][o + j + 1] = -z11;
         }
         __syncthreads();
     }
