@@ -205,6 +205,13 @@ int gptq_quantize_static_scratch(float *W, const float *Hinv_chol, const int32_t
                                  uint8_t *packed_int4, int32_t *g_idx, float *err_sq,
                                  void *stream);
 
+/* Diagnostic of the bounded waits the tensor-core kernels use: launches one
+ * warp that waits on an mbarrier nothing completes, with a limit of
+ * `limit_cycles` SM clocks (0 < limit <= about 2e9), and returns what the
+ * device status word then holds: GPTQ_ERR_TIMEOUT when the wait gave up as
+ * designed.  The device stays usable afterwards.  Synchronises the device. */
+int gptq_selftest_bounded_wait(int64_t limit_cycles);
+
 /* dst[i] = (float) bf16 src[i] (exact widening), n >= 0 elements. */
 int gptq_bf16_to_f32(float *dst, const uint16_t *src, int64_t n, void *stream);
 

@@ -36,6 +36,7 @@ SIGNATURES = [
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize_static_scratch", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    ("gptq_selftest_bounded_wait", _I, [_I64]),
     ("gptq_bf16_to_f32", _I, [_P, _P, _I64, _P]),
 ]
 
@@ -192,6 +193,11 @@ def gptq_quantize_static_scratch(W: torch.Tensor, Hinv_chol: torch.Tensor, perm:
                                               bits, group_size, block_size, _ptr(codes),
                                               _ptr(scales), _ptr(zeros), _ptr(packed_int4),
                                               _ptr(g_idx), _ptr(err_sq), _stream(W, stream)))
+
+
+def gptq_selftest_bounded_wait(limit_cycles: int) -> int:
+    """Status of a deliberately unsatisfied, bounded device wait (expect 5)."""
+    return lib().gptq_selftest_bounded_wait(int(limit_cycles))
 
 
 def gptq_bf16_to_f32(dst: torch.Tensor, src: torch.Tensor, stream=None):

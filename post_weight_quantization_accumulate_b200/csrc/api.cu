@@ -103,6 +103,23 @@ static int hessian_device(float* H, const uint16_t* X, int64_t n, int64_t d, cud
     return GPTQ_OK;
 }
 
+// One thread waits, through the same bounded-wait helper the tensor-core
+// kernels use, on an mbarrier that nothing completes, with a limit of
+// `limit_cycles`; the wait gives up, records GPTQ_ERR_TIMEOUT and returns.
+__global__ void bounded_wait_selftest_kernel(long long limit_cycles, int* status)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, status, limit_cycles);
+    __syncthreads();
+}
+
 }  // namespace gptq
 
 using namespace gptq;
@@ -255,6 +272,18 @@ int gptq_quantize(float* W, const float* Hinv_chol, const int32_t* perm, int64_t
     return run_quantize(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
                         scales, zeros, packed_int4, g_idx, err_sq, workspace,
                         static_cast<cudaStream_t>(stream));
+}
+
+int gptq_selftest_bounded_wait(int64_t limit_cycles)
+{
+    if (limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return GPTQ_ERR_INVALID_ARG;
+    int rc = check_device();
+    if (rc) return rc;
+    int* status = device_status_ptr();
+    if (!status) return GPTQ_ERR_CUDA;
+    bounded_wait_selftest_kernel<<<1, 32>>>(limit_cycles, status);
+    GPTQ_LAUNCH_CHECK();
+    return gptq_device_status();
 }
 
 int gptq_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, void* stream)

@@ -80,17 +80,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 }
 
 // Waits for the phase of `bar` with the given parity.  Gives up when *abort
-// becomes non-zero or after kWaitLimitCycles; on a time-out it raises *abort
+// becomes non-zero or after `limit` cycles; on a time-out it raises *abort
 // and records GPTQ_ERR_TIMEOUT.  Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, int* status)
+                                                  volatile int* abort, int* status,
+                                                  long long limit = kWaitLimitCycles)
 {
     if (mbar_try_wait(bar, parity)) return true;
     long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             *abort = 1;
             record_status(status, GPTQ_ERR_TIMEOUT);
             return false;

@@ -90,3 +90,5 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.gptq_bf16_to_f32(None, fake, 10, None) == 1
     assert lib.gptq_hessian_accumulate_host(fake, fake, 16, 64, None, 8, None) == 1
     assert lib.gptq_hessian_accumulate_host(fake, fake, 16, 64, fake, 0, None) == 1
+    assert lib.gptq_selftest_bounded_wait(0) == 1
+    assert lib.gptq_selftest_bounded_wait(1 << 40) == 1

@@ -258,3 +258,12 @@ def test_launch_count_increases():
     _gpu_hessian(_rand_x(1, 128, 64))
     assert B.gptq_launch_count() >= before + 2
     assert B.gptq_device_status() == 0
+
+
+def test_bounded_wait_times_out_and_device_stays_usable():
+    """A wait nothing satisfies gives up after its limit (~1 ms here), records
+    GPTQ_ERR_TIMEOUT, and later work on the device still runs correctly."""
+    assert B.gptq_selftest_bounded_wait(2_000_000) == 5
+    assert B.gptq_device_status() == 0          # the word was read and cleared
+    xb = _rand_x(9, 256, 64)
+    np.testing.assert_allclose(_gpu_hessian(xb), oracle.hessian(xb), rtol=1e-5, atol=1e-3)
