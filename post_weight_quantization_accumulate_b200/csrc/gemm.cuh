@@ -8,7 +8,9 @@ namespace gptq {
 enum GemmFlags : int {
     kGemmLowerA = 1,  // A is lower triangular: only k <= m contributes
     kGemmLowerB = 2,  // B is lower triangular: only k >= n contributes
-    kGemmLowerC = 4,  // only the lower triangle (col <= row) of C is written
+    kGemmLowerC = 4,  // only the lower triangle (col <= row) of C is needed: tiles above
+                      // the diagonal are skipped, entries above it inside diagonal
+                      // tiles may be updated too
 };
 
 // C = alpha * A * B + beta * C (row-major; beta == 0 ignores C's contents).

@@ -16,11 +16,17 @@
 //   warp 0       TMA producer: fp32 tiles of A (K-major) and B (MN- or K-major)
 //   warp 1       MMA issuer + TMEM owner (two 128-column fp32 accumulators)
 //   warps 4-7    converters: the low tf32 parts of each stage in shared memory
-//   warps 8-11   epilogue: TMEM -> registers -> alpha acc + beta C -> global
-// Three 64 KB stages (A_hi, A_lo, B_hi, B_lo of 16 KB each).  All waits are
-// bounded (see mbar_wait_bounded).
+//   warps 8-11   epilogue: TMEM -> registers -> global.  With beta = 1 each
+//                warp stages alpha * acc for its 32 rows x 32 columns in
+//                shared memory and a TMA reduce-add applies it to C in L2
+//                (one rounding of C + alpha * acc, the same as the fma
+//                below); with beta = 0 a TMA store writes it; other betas
+//                (or a C that breaks the TMA rules) read C with plain loads.
+// Three 64 KB stages (A_hi, A_lo, B_hi, B_lo of 16 KB each) plus 32 KB of
+// epilogue staging.  All waits are bounded (see mbar_wait_bounded).
 #include "gemm.cuh"
 
+#include <cstring>
 #include <mutex>
 
 namespace gptq {
@@ -33,8 +39,11 @@ constexpr int STAGE_BYTES = 4 * TILE_BYTES;      // A_hi, A_lo, B_hi, B_lo
 constexpr int TTHREADS = 384;
 constexpr int TMEM_COLS = 2 * TBN;
 
+constexpr int CBUF_BYTES = 32 * 32 * 4;          // one warp's 32 x 32 chunk of C
+
 struct alignas(1024) GemmSmem {
     uint8_t stage[TSTAGES][STAGE_BYTES];
+    uint8_t cbuf[4][2][CBUF_BYTES];                  // per epilogue warp, double-buffered
     uint64_t full[TSTAGES];    // TMA landed
     uint64_t conv[TSTAGES];    // hi/lo split done
     uint64_t empty[TSTAGES];   // MMAs done reading
@@ -44,9 +53,12 @@ struct alignas(1024) GemmSmem {
     int abort;
 };
 constexpr size_t GEMM_SMEM = sizeof(GemmSmem) + 1024;
+static_assert(GEMM_SMEM <= 227 * 1024, "one CTA per SM: at most 227 KB of shared memory");
+
+enum CMode : int { kCPlain = 0, kCStore = 1, kCReduce = 2 };
 
 struct GemmArgs {
-    int M, N, K, batch, flags, trans_b;
+    int M, N, K, batch, flags, trans_b, c_mode;
     float alpha, beta;
     float* C;
     int64_t ldc, sC;
@@ -75,6 +87,37 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// C chunk from shared memory (128B-swizzled 32 x 32 fp32 box) to global:
+// added to C (reduce) or written (store), by the TMA unit.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x, int y,
+                                                  int z)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// at most one committed group may still be reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1()
+{
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Unit u -> (batch, m-tile, n-tile) and its K range [k0, k1) (multiples of TBK);
 // returns false for a tile the lower-triangular output flag skips.
 __device__ __forceinline__ bool unit_info(const GemmArgs& g, int u, int& b, int& mt, int& nt, int& k0,
@@ -96,7 +139,7 @@ __device__ __forceinline__ bool unit_info(const GemmArgs& g, int u, int& b, int&
 
 __global__ void __launch_bounds__(TTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                   const GemmArgs g)
+                   const __grid_constant__ CUtensorMap mapC, const GemmArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
     GemmSmem& S = *reinterpret_cast<GemmSmem*>(
@@ -118,6 +161,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
         fence_mbar_init();
         prefetch_tmap(&mapA);
         prefetch_tmap(&mapB);
+        if (g.c_mode != kCPlain) prefetch_tmap(&mapC);
     }
     if (warp == 1) {
         tmem_alloc(&S.tmem_base, TMEM_COLS);
@@ -237,11 +281,14 @@ __global__ void __launch_bounds__(TTHREADS, 1)
                 if (lane == 0) mbar_arrive(&S.conv[s]);
             }
         }
-    } else if (warp >= 8) {
-        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (= tile rows)
+    } else if (warp >= 8 && g.c_mode != kCPlain) {
+        // epilogue through the TMA unit: warp w stages rows 32*(w % 4) .. +31
+        // of a 32-column chunk (128B swizzle: 16-byte piece j of row r sits at
+        // piece j ^ (r % 8)) and one lane issues the reduce-add or store
         const int q = warp & 3;
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        uint32_t uc = 0;
+        const bool lower = (g.flags & kGemmLowerC) != 0;
+        uint32_t uc = 0, nbuf = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
             int b, mt, nt, k0, k1;
             if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
@@ -252,24 +299,104 @@ __global__ void __launch_bounds__(TTHREADS, 1)
             __syncwarp();
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
-            const bool have = k1 > k0;   // an empty K range leaves the accumulator unwritten
-            const int row = mt * TBM + q * 32 + lane;
-            float* crow = g.C + b * g.sC + static_cast<int64_t>(row) * g.ldc;
+            const bool have = k1 > k0;
+            const int row0 = mt * TBM + q * 32;
 #pragma unroll 1
             for (int c = 0; c < TBN / 32; ++c) {
+                const int col0 = nt * TBN + c * 32;
                 float v[32];
+                tmem_ld_32x32b_x32(tbase + lane_addr + acc * TBN + c * 32, v);
+                tmem_ld_wait();
+                // nothing of this chunk inside C (or, lower C, all above the diagonal)
+                if (row0 >= g.M || col0 >= g.N || (lower && col0 > row0 + 31)) continue;
+                uint8_t* buf = S.cbuf[q][nbuf & 1];
+                ++nbuf;
+                if (lane == 0) bulk_wait_read_1();
+                __syncwarp();
+                float4* rowp = reinterpret_cast<float4*>(buf + lane * 128);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 o;
+                    o.x = have ? g.alpha * v[4 * j] : 0.f;
+                    o.y = have ? g.alpha * v[4 * j + 1] : 0.f;
+                    o.z = have ? g.alpha * v[4 * j + 2] : 0.f;
+                    o.w = have ? g.alpha * v[4 * j + 3] : 0.f;
+                    rowp[j ^ (lane & 7)] = o;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (g.c_mode == kCReduce)
+                        tma_reduce_add_3d(&mapC, buf, col0, row0, b);
+                    else
+                        tma_store_3d(&mapC, buf, col0, row0, b);
+                    bulk_commit();
+                }
+                __syncwarp();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tempty[acc]);
+        }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    } else if (warp >= 8) {
+        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (= tile rows).  The
+        // C values of a 32-column chunk are loaded one chunk ahead, the first
+        // before the accumulator is ready, so the loads overlap the MMAs and
+        // the previous chunk's arithmetic.
+        const int q = warp & 3;
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        const bool lower = (g.flags & kGemmLowerC) != 0;
+        const bool read_c = g.beta != 0.f;
+        uint32_t uc = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            int b, mt, nt, k0, k1;
+            if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
+            const int acc = uc & 1;
+            const uint32_t aph = (uc >> 1) & 1;
+            ++uc;
+            const int row = mt * TBM + q * 32 + lane;
+            float* crow = g.C + b * g.sC + static_cast<int64_t>(row) * g.ldc;
+            // chunk c takes the vector path when it lies inside C, above no
+            // skipped (upper) element and 16-byte aligned
+            auto vec_ok = [&](int c) {
+                const int col0 = nt * TBN + c * 32;
+                return row < g.M && col0 + 32 <= g.N && !(lower && col0 + 31 > row) &&
+                       (reinterpret_cast<uintptr_t>(crow + col0) & 15) == 0;
+            };
+            float4 cn[8];
+            if (read_c && vec_ok(0)) {
+                const float4* p = reinterpret_cast<const float4*>(crow + nt * TBN);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) cn[m] = p[m];
+            }
+            const bool got = mbar_wait_bounded(&S.tfull[acc], aph, abort, status);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const bool have = k1 > k0;   // an empty K range leaves the accumulator unwritten
+#pragma unroll 1
+            for (int c = 0; c < TBN / 32; ++c) {
+                float4 cc[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) cc[m] = cn[m];
+                if (read_c && c + 1 < TBN / 32 && vec_ok(c + 1)) {
+                    const float4* p = reinterpret_cast<const float4*>(crow + nt * TBN + (c + 1) * 32);
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) cn[m] = p[m];
+                }
+                float v[32];
+                __syncwarp();   // the loads above may diverge; tcgen05.ld is warp-aligned
                 tmem_ld_32x32b_x32(tbase + lane_addr + acc * TBN + c * 32, v);
                 tmem_ld_wait();
                 const int col0 = nt * TBN + c * 32;
                 if (row >= g.M || col0 >= g.N) continue;
-                const bool lower = (g.flags & kGemmLowerC) != 0;
-                if (col0 + 32 <= g.N && !(lower && col0 + 31 > row) &&
-                    (reinterpret_cast<uintptr_t>(crow + col0) & 15) == 0) {
+                if (vec_ok(c)) {
                     float4* p = reinterpret_cast<float4*>(crow + col0);
 #pragma unroll
                     for (int m = 0; m < 8; ++m) {
-                        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (g.beta != 0.f) o = p[m];
+                        float4 o = read_c ? cc[m] : make_float4(0.f, 0.f, 0.f, 0.f);
                         const float a0 = have ? v[4 * m] : 0.f, a1 = have ? v[4 * m + 1] : 0.f;
                         const float a2 = have ? v[4 * m + 2] : 0.f, a3 = have ? v[4 * m + 3] : 0.f;
                         o.x = fmaf(g.alpha, a0, g.beta * o.x);
@@ -284,7 +411,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
                         const int col = col0 + m;
                         if (col >= g.N || (lower && col > row)) continue;
                         const float a = have ? v[m] : 0.f;
-                        const float old = (g.beta != 0.f) ? crow[col] : 0.f;
+                        const float old = read_c ? crow[col] : 0.f;
                         crow[col] = fmaf(g.alpha, a, g.beta * old);
                     }
                 }
@@ -368,7 +495,17 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
         attr_set[dev] = true;
     }
     const int Kp = K > 0 ? K : 1;
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mC;
+    int c_mode = kCPlain;
+    const bool c_tma = (reinterpret_cast<uintptr_t>(C) & 15) == 0 && (ldc & 3) == 0 &&
+                       (batch == 1 || (sC & 3) == 0);
+    if (c_tma && (beta == 1.f || beta == 0.f)) {
+        int rc = make_map_f32(&mC, C, N, M, ldc, batch, sC, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+        c_mode = beta == 1.f ? kCReduce : kCStore;
+    } else {
+        memset(&mC, 0, sizeof mC);
+    }
     int rc = make_map_f32(&mA, A, Kp, M, lda, batch, sA, TBK, TBM, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     if (trans_b)
@@ -383,6 +520,7 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     g.batch = batch;
     g.flags = flags;
     g.trans_b = trans_b ? 1 : 0;
+    g.c_mode = c_mode;
     g.alpha = alpha;
     g.beta = beta;
     g.C = C;
@@ -395,7 +533,7 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     int cap = sm_count();
     if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;
     const int grid = static_cast<int>(units < cap ? units : cap);
-    gemm_tc_kernel<<<grid, TTHREADS, GEMM_SMEM, stream>>>(mA, mB, g);
+    gemm_tc_kernel<<<grid, TTHREADS, GEMM_SMEM, stream>>>(mA, mB, mC, g);
     GPTQ_LAUNCH_CHECK();
     return GPTQ_OK;
 }

@@ -11,7 +11,10 @@
 //   M   = chol_lower(A)                    (blocked, right-looking, fp32)
 //   U   = J M^{-1} J                       (upper; U^T U = (P^T H_d P)^{-1})
 // which needs one Cholesky and one triangular inverse (2/3 d^3 flops) instead
-// of inverse + Cholesky of the inverse.
+// of inverse + Cholesky of the inverse.  M^{-1} is accumulated alongside the
+// factorisation, as forward elimination of [A | I]: once panel k is factored,
+// row block k of M^{-1} is M_kk^{-1} (E_k - sum_{j<k} M_kj (M^{-1})_j), and the
+// rows below receive -M_ik (M^{-1})_k right-looking, like the trailing update.
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -33,7 +36,7 @@ size_t prepare_workspace_bytes(int64_t d)
 {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t dd = static_cast<size_t>(d) * static_cast<size_t>(d) * sizeof(float);
-    return 256 + up(dd) /*A,M*/ + up(dd) /*Minv*/ + up(dd) /*T*/;
+    return 256 + up(dd) /*A,M*/ + up(dd) /*Minv*/;
 }
 
 namespace {
@@ -137,8 +140,11 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
 // One panel step of the blocked Cholesky, fused:
 //   every CTA factors the kb x kb diagonal block at (k0, k0) (redundantly, so
 //   no other launch has to wait for it) and inverts the factor; CTA 0 writes
-//   L_kk^{-1} into M^{-1}; CTA b >= 1 solves the panel rows
-//   k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T}.
+//   L_kk^{-1} into M^{-1}; CTA b in 1..n_trsm solves the panel rows
+//   k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T};
+//   CTA n_trsm+1+c finishes column block c < k0/64 of row block k of M^{-1}:
+//   Y_k = L_kk^{-1} (Y~_k - L_k,k-1 Y_{k-1}), Y~_k holding the updates of the
+//   panels before k-1 (applied in memory by the side stream).
 // Factorisation of the 64 x 64 block in shared memory, in 16 strips of 4
 // columns: warp 0 factors the strip with shuffles (lane l holds rows 4P+l and
 // 4P+l+32), then all warps subtract its rank-4 product from the trailing
@@ -401,12 +407,10 @@ __global__ void __launch_bounds__(256)
     if (bad_any && tid == 0 && blockIdx.x == 0) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
 
     if (blockIdx.x == 0) {
-        // L_kk itself is not needed later (the inverse uses L_kk^{-1} and the
-        // off-diagonal panels), and the other CTAs of this launch may still be
-        // reading the diagonal block of A, so only M^{-1} is written: its
-        // diagonal block, and for an odd panel also the block left of it,
-        //   M^{-1}[k, k-1] = -Z_kk (M[k, k-1] Z_{k-1,k-1})
-        // (first level of the recursive inverse; M[k, k-1] is Pd).
+        // L_kk itself is not needed later (the trailing updates use the
+        // off-diagonal panels, the inverse L_kk^{-1}), and the other CTAs of
+        // this launch may still be reading the diagonal block of A, so only
+        // the diagonal block of M^{-1} is written.
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -414,44 +418,54 @@ __global__ void __launch_bounds__(256)
                 const int gi = r0 + i, gj = c0 + j;
                 if (gi < kb && gj < kb) Minv[static_cast<int64_t>(k0 + gi) * d + k0 + gj] = Zs[gi][gj];
             }
-        if (pk0 >= 0 && ((k0 / kNB) & 1)) {
-            load_tile(Pr, Minv, d, pk0, kNB, pk0, kNB, true, false);   // Z_{k-1,k-1}
-            __syncthreads();
-            float y[4][4] = {};
-            for (int k = 0; k < kNB; ++k) {
-                float a4[4], b4[4];
+        return;
+    }
+    const int n_trsm = (d - k0 - kb + kNB - 1) / kNB;
+    if (static_cast<int>(blockIdx.x) > n_trsm) {
+        // column block cb of row block k of M^{-1} (pk0 >= 0 here)
+        const int cb = (blockIdx.x - 1 - n_trsm) * kNB;
+        load_tile(As, Minv, d, k0, kb, cb, kNB, false, false);   // Y~_k
+        load_tile(Pr, Minv, d, pk0, kNB, cb, kNB, false, false); // Y_{k-1}
+        __syncthreads();
+        float t4[4][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) a4[i] = Pd[r0 + i][k];
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) b4[j] = Pr[k][c0 + j];
+            for (int j = 0; j < 4; ++j) t4[i][j] = As[r0 + i][c0 + j];
+        for (int k = 0; k < kNB; ++k) {
+            float a4[4], b4[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i) a4[i] = Pd[r0 + i][k];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) y[i][j] = fmaf(a4[i], b4[j], y[i][j]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = y[i][j];
-            __syncthreads();
-            float x[4][4] = {};
-            for (int k = 0; k < kNB; ++k) {
-                float a4[4], b4[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) a4[i] = Zs[r0 + i][k];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) b4[j] = As[k][c0 + j];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) x[i][j] = fmaf(a4[i], b4[j], x[i][j]);
-            }
+            for (int j = 0; j < 4; ++j) b4[j] = Pr[k][c0 + j];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (r0 + i < kb) Minv[static_cast<int64_t>(k0 + r0 + i) * d + pk0 + c0 + j] = -x[i][j];
+                for (int j = 0; j < 4; ++j) t4[i][j] = fmaf(-a4[i], b4[j], t4[i][j]);
         }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = t4[i][j];
+        __syncthreads();
+        float y4[4][4] = {};
+        for (int k = 0; k < kNB; ++k) {
+            float a4[4], b4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a4[i] = Zs[r0 + i][k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b4[j] = As[k][c0 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) y4[i][j] = fmaf(a4[i], b4[j], y4[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (r0 + i < kb) Minv[static_cast<int64_t>(k0 + r0 + i) * d + cb + c0 + j] = y4[i][j];
         return;
     }
 
@@ -514,10 +528,11 @@ __global__ void reverse_upper_kernel(const float* __restrict__ Minv, int d, floa
 // with its events; the caller's stream forks to it and joins it again.
 struct SideStream {
     static constexpr int kRing = 4;
-    cudaStream_t s = nullptr;          // trailing symmetric updates
-    cudaStream_t s2 = nullptr;         // levels >= 256 of the recursive inverse
+    cudaStream_t s = nullptr;          // trailing symmetric updates of A
+    cudaStream_t s2 = nullptr;         // updates of the lower rows of M^{-1}
     cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr, done_panel = nullptr;
-    cudaEvent_t ev[kRing] = {};
+    cudaEvent_t cleared = nullptr;
+    cudaEvent_t ev[kRing] = {}, ev2[kRing] = {};
 };
 
 static int side_stream(SideStream** out)
@@ -539,8 +554,11 @@ static int side_stream(SideStream** out)
         GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming));
         GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join2, cudaEventDisableTiming));
         GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.done_panel, cudaEventDisableTiming));
-        for (int i = 0; i < SideStream::kRing; ++i)
+        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.cleared, cudaEventDisableTiming));
+        for (int i = 0; i < SideStream::kRing; ++i) {
             GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.ev[i], cudaEventDisableTiming));
+            GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.ev2[i], cudaEventDisableTiming));
+        }
     }
     *out = &st;
     return GPTQ_OK;
@@ -556,8 +574,18 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     PrepHeader* hdr = reinterpret_cast<PrepHeader*>(ws);
     float* A = reinterpret_cast<float*>(ws + 256);
     float* Minv = reinterpret_cast<float*>(ws + 256 + up(dd));
-    float* T = reinterpret_cast<float*>(ws + 256 + 2 * up(dd));
     const int nsm = sm_count();
+
+    SideStream* side = nullptr;
+    int rc = side_stream(&side);
+    if (rc) return rc;
+    // M^{-1} starts as zeros (its row blocks are accumulated in place); the
+    // clear runs on the second side stream next to the gather
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->fork, stream));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->fork, 0));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->fork, 0));
+    GPTQ_CUDA_CHECK(cudaMemsetAsync(Minv, 0, dd, side->s2));
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->cleared, side->s2));
 
     GPTQ_CUDA_CHECK(cudaMemsetAsync(hdr, 0, sizeof(PrepHeader), stream));
     diag_mean_kernel<<<1, 1024, 0, stream>>>(H, d, damp, hdr);
@@ -578,25 +606,15 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
         gather_rev_direct_kernel<<<nsm * 8, 256, 0, stream>>>(H, d, perm, hdr, A);
     }
     GPTQ_LAUNCH_CHECK();
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->cleared, 0));
 
     // Blocked right-looking Cholesky, A = M M^T (lower), with look-ahead:
-    // panel k+1 applies panel k's correction to its own block column on the
-    // fly; the correction of everything right of block column k+1 (the large
-    // symmetric update) runs on a side stream and is waited for only by panel
-    // k+2.  The critical path is the chain of panel kernels.
-    SideStream* side = nullptr;
-    int rc = side_stream(&side);
-    if (rc) return rc;
+    // panel k+1 applies panel k's correction to its own block column (and to
+    // its row block of M^{-1}) on the fly; the corrections of everything
+    // below block k+1 -- the symmetric trailing update of A on one side
+    // stream, the update of M^{-1}'s lower rows on the other -- are waited for
+    // only by panel k+2.  The critical path is the chain of panel kernels.
     const int n_panels = (d + kNB - 1) / kNB;
-    // M^{-1} by recursive doubling,
-    //   [A 0; B C]^{-1} = [A^-1 0; -C^-1 B A^-1  C^-1],
-    // grown as the factorisation advances: the 64-blocks and the first level
-    // come from the panel kernels, pairs of level s >= 256 run on the second
-    // side stream as soon as the panels they cover are done.
-    GPTQ_CUDA_CHECK(cudaMemsetAsync(Minv, 0, dd, stream));
-    GPTQ_CUDA_CHECK(cudaEventRecord(side->fork, stream));
-    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->fork, 0));
-    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->fork, 0));
     {
         static bool attr_panel[64] = {};
         int dev = 0;
@@ -610,71 +628,50 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     }
     for (int p = 0; p < n_panels; ++p) {
         const int k0 = p * kNB;
-        // SMs the side products may hold: the rest after this panel's CTAs
-        const int side_ctas = std::max(16, nsm - (1 + (d - k0 + kNB - 1) / kNB));
         const int kb = std::min(kNB, d - k0);
         const int rest = d - k0 - kb;
-        if (p >= 2) GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev[(p - 2) % SideStream::kRing], 0));
-        chol_panel_kernel<<<1 + (rest + kNB - 1) / kNB, 256, kPanelSmem, stream>>>(
-            A, d, k0, kb, p > 0 ? k0 - kNB : -1, Minv, hdr);
+        const int n_trsm = (rest + kNB - 1) / kNB;
+        const int n_cta = 1 + n_trsm + p;
+        // SMs the side products may hold: the rest after this panel's CTAs,
+        // split between the two side streams in proportion to their flops
+        // (rest2^2 / 2 for the symmetric update, rest2 (k0 + kb) for M^{-1})
+        const int free_sm = std::max(16, nsm - n_cta);
+        const double f_sym = 0.5 * std::max(rest - kNB, 0);
+        const double f_inv = static_cast<double>(k0 + kb);
+        const int ctas_sym = std::max(8, static_cast<int>(free_sm * f_sym / (f_sym + f_inv) + 0.5));
+        const int ctas_inv = std::max(8, free_sm - ctas_sym);
+        if (p >= 2) {
+            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev[(p - 2) % SideStream::kRing], 0));
+            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev2[(p - 2) % SideStream::kRing], 0));
+        }
+        chol_panel_kernel<<<n_cta, 256, kPanelSmem, stream>>>(A, d, k0, kb, p > 0 ? k0 - kNB : -1,
+                                                              Minv, hdr);
         GPTQ_LAUNCH_CHECK();
         GPTQ_CUDA_CHECK(cudaEventRecord(side->done_panel, stream));
-        // inverse pairs that end with this panel: level s covers [end - s, end)
-        const int end = k0 + kb;
-        if (kb == kNB) {
-            bool waited = false;
-            for (int sz = 4 * kNB; sz <= end; sz *= 2) {
-                if (end % sz) break;
-                if (!waited) {
-                    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->done_panel, 0));
-                    waited = true;
-                }
-                const int o = end - sz, h = sz / 2;
-                rc = launch_sgemm(false, h, h, h, 1.f, A + static_cast<int64_t>(o + h) * d + o, d, 0,
-                                  Minv + static_cast<int64_t>(o) * d + o, d, 0, 0.f, T, h, 0, 1,
-                                  kGemmLowerB, side->s2, side_ctas);
-                if (rc) return rc;
-                rc = launch_sgemm(false, h, h, h, -1.f, Minv + static_cast<int64_t>(o + h) * d + o + h, d,
-                                  0, T, h, 0, 0.f, Minv + static_cast<int64_t>(o + h) * d + o, d, 0, 1,
-                                  kGemmLowerA, side->s2, side_ctas);
-                if (rc) return rc;
-            }
-        }
-        const int rest2 = rest - kNB;   // rows/columns right of block column p+1
+        const int rest2 = rest - kNB;   // rows/columns below block k+1
         if (rest2 > 0) {
             GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->done_panel, 0));
+            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->done_panel, 0));
             float* P = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0;
             float* C = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0 + kb + kNB;
             rc = launch_sgemm(true, rest2, rest2, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,
-                              kGemmLowerC, side->s, side_ctas);
+                              kGemmLowerC, side->s, ctas_sym);
+            if (rc) return rc;
+            // (M^{-1})[below k+1][0 : k0+kb] -= M[below k+1][k] (M^{-1})_k
+            rc = launch_sgemm(false, rest2, k0 + kb, kb, -1.f, P, d, 0,
+                              Minv + static_cast<int64_t>(k0) * d, d, 0, 1.f,
+                              Minv + static_cast<int64_t>(k0 + kb + kNB) * d, d, 0, 1, 0, side->s2,
+                              ctas_inv);
             if (rc) return rc;
         }
         GPTQ_CUDA_CHECK(cudaEventRecord(side->ev[p % SideStream::kRing], side->s));
+        GPTQ_CUDA_CHECK(cudaEventRecord(side->ev2[p % SideStream::kRing], side->s2));
     }
     GPTQ_CUDA_CHECK(cudaEventRecord(side->join, side->s));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join, 0));
     GPTQ_CUDA_CHECK(cudaEventRecord(side->join2, side->s2));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join2, 0));
 
-    // Ragged pairs of the recursive inverse (sizes that are not a power of two
-    // times 64); level 128 was completed by the panel kernels.
-    for (int s = 4 * kNB; s / 2 < d; s *= 2) {
-        const int h = s / 2;
-        const int o = (d / s) * s;
-        const int m2 = d - o - h;
-        if (m2 > 0) {
-            const float* Bo = A + static_cast<int64_t>(o + h) * d + o;
-            const float* Ai = Minv + static_cast<int64_t>(o) * d + o;
-            rc = launch_sgemm(false, m2, h, h, 1.f, Bo, d, 0, Ai, d, 0, 0.f, T, h, 0, 1,
-                              kGemmLowerB, stream);
-            if (rc) return rc;
-            const float* Ci = Minv + static_cast<int64_t>(o + h) * d + o + h;
-            rc = launch_sgemm(false, m2, h, m2, -1.f, Ci, d, 0, T, h, 0, 0.f,
-                              Minv + static_cast<int64_t>(o + h) * d + o, d, 0, 1, kGemmLowerA,
-                              stream);
-            if (rc) return rc;
-        }
-    }
     reverse_upper_kernel<<<nsm * 8, 256, 0, stream>>>(Minv, d, U);
     GPTQ_LAUNCH_CHECK();
 

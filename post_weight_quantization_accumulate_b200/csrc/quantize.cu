@@ -13,10 +13,12 @@
 //   q = clamp(rint(w_c / s) + z, 0, maxq);  w^ = s (q - z);  e = (w_c - w^) / U[c][c]
 //   w[c+1 : block end] -= e U[c][c+1 : block end]         (fused kernel, registers)
 //   W[:, block end:]    -= E_blk U[blk, block end:]        (once per block, GEMM)
-// Rows are independent once U is known, so a CTA owns 32 rows; each row is
-// split over 4 threads of one warp that hold 32 columns each in registers.
-// The column value is broadcast with one shuffle, every thread computes the
-// same (q, e), and updates its own 32 columns from the U row in shared memory.
+// Rows are independent once U is known.  Each row is split over 4 adjacent
+// lanes of a warp; lane part p holds the row's in-block columns 32p..32p+31 in
+// registers.  Every lane of the row computes the same (q, e) for the current
+// column and corrects its own 32 registers with U row c from shared memory.
+// The block's U rows are laid out once per call by u_layout_kernel and arrive
+// in shared memory by bulk copies, one per 16-column sub-block.
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -26,23 +28,25 @@ namespace {
 
 constexpr int QB = 128;           // largest block width
 constexpr int kOuterMax = 1024;   // widest outer window of the two-level lazy batch
-constexpr int QTPR = 8;           // threads per row
-constexpr int QCPT = QB / QTPR;   // registers per thread (column 8m + p belongs to part p)
-constexpr int QSUB = 16;          // columns per unrolled sub-block
-constexpr int QRPS = QSUB / QTPR; // registers a sub-block occupies per thread
-constexpr int QROWS = 16;         // rows per CTA
+constexpr int QTPR = 4;           // lanes per row
+constexpr int QCPT = QB / QTPR;   // registers per lane: part p holds columns 32p .. 32p+31
+constexpr int QSUB = 16;          // columns per unrolled sub-block (one bulk copy each)
+constexpr int QNSUB = QB / QSUB;
+constexpr int QROWS = 32;         // rows per CTA
 constexpr int QTHREADS = QROWS * QTPR;
-constexpr int UT_PART = QCPT + 4; // padded part stride (80 bytes): the 8 parts of a U row
-                                  // read by one 8-lane phase hit distinct banks
+// U rows of a sub-block: [16 rows][4 parts][40] (32 coefficients + 8 pad, so the
+// four parts of a row fall in distinct bank groups), then 16 pairs
+// (1 / U[c][c], U[c][c+1]).
+constexpr int UT_PART = QCPT + 8;
 constexpr int UT_LD = QTPR * UT_PART;
-constexpr int ES_LD = QB + 4;
-constexpr size_t kBlockSmem =
-    (static_cast<size_t>(QB) * UT_LD + QB + static_cast<size_t>(QROWS) * ES_LD) * sizeof(float) +
-    static_cast<size_t>(QROWS) * ES_LD;
+constexpr int UCH_FLOATS = QSUB * UT_LD + 2 * QSUB;
+constexpr int UCH_BYTES = UCH_FLOATS * 4;          // 10368, a multiple of 16
+constexpr size_t kBlockSmem = static_cast<size_t>(QNSUB) * UCH_BYTES + 128;
+static_assert(UCH_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 struct QArgs {
     float* Wp;            // [d_out][d_in] working weights, processing order
-    const float* U;       // [d_in][d_in]
+    const float* Ul;      // U blocks in sub-block layout (u_layout_kernel)
     int d_out, d_in, j0, bw, block, bits, gs, n_groups;
     float* scales;        // [d_out][n_groups]
     float* zeros;
@@ -50,7 +54,50 @@ struct QArgs {
     float* E;             // [d_out][kOuterMax] errors of the current outer window
     int e_off;            // column of this block inside the outer window
     float* err_sq;        // [d_out] or null
+    int* status;
 };
+
+// Sub-block layout of U's diagonal blocks: chunk (b, S) covers rows
+// j0 + 16S .. j0 + 16S + 15 of block b (j0 = b * block, width bw).  Entry
+// [cl][p][k] is U[j0+c][j0+32p+k] for in-block column 32p+k > c (zero on and
+// below the diagonal and beyond bw); pair cl is (1 / U[c][c], U[c][c+1]),
+// zero past bw.  One CTA per chunk.
+__global__ void u_layout_kernel(const float* __restrict__ U, int d_in, int block, int nch_blk,
+                                float* __restrict__ Ul)
+{
+    const int b = blockIdx.x / nch_blk, S = blockIdx.x % nch_blk;
+    const int j0 = b * block;
+    const int bw = min(block, d_in - j0);
+    float* out = Ul + static_cast<int64_t>(blockIdx.x) * UCH_FLOATS;
+    for (int idx = threadIdx.x; idx < UCH_FLOATS; idx += blockDim.x) {
+        float v = 0.f;
+        if (idx < QSUB * UT_LD) {
+            const int cl = idx / UT_LD, rem = idx % UT_LD;
+            const int p = rem / UT_PART, k = rem % UT_PART;
+            const int c = S * QSUB + cl, col = QCPT * p + k;
+            if (k < QCPT && c < bw && col > c && col < bw)
+                v = U[static_cast<int64_t>(j0 + c) * d_in + j0 + col];
+        } else {
+            const int i = idx - QSUB * UT_LD;
+            const int c = S * QSUB + i / 2;
+            if (i % 2 == 0) {
+                if (c < bw) v = 1.f / U[static_cast<int64_t>(j0 + c) * d_in + j0 + c];
+            } else if (c + 1 < bw) {
+                v = U[static_cast<int64_t>(j0 + c) * d_in + j0 + c + 1];
+            }
+        }
+        out[idx] = v;
+    }
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 
 __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, float& s, float& z)
 {
@@ -62,35 +109,31 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, 
     z = rintf(__fdiv_rn(-mn, s));
 }
 
-// rint(w / s) with w / s correctly rounded, from the product w * rs (rs the
-// correctly rounded 1 / s).  The product is within 2^-23 relative of w / s,
-// so the two round to the same integer unless w / s lies that close to a
-// half-integer; only then is the division carried out.
+// rint(w / s) with w / s correctly rounded, from the product t = w * rs (rs the
+// correctly rounded 1 / s).  t is within 2^-23 relative of w / s, so the two
+// round to the same integer unless t lies that close to a half-integer; only
+// then is the division carried out.
 __device__ __forceinline__ float rint_div(float w, float s, float rs)
 {
     const float t = w * rs;
-    const float fr = t - floorf(t);
-    if (fabsf(fr - 0.5f) <= 4.8e-7f * fmaxf(fabsf(t), 1.f)) return rintf(__fdiv_rn(w, s));
-    return rintf(t);
+    const float r = rintf(t);
+    const float thr = fmaf(-4.8e-7f, fmaxf(fabsf(t), 1.f), 0.5f);
+    if (fabsf(t - r) >= thr) return rintf(__fdiv_rn(w, s));
+    return r;
 }
-
-// Register slot of in-block column k (owned by part k % QTPR) while sub-block
-// S is processed: the QCPT-slot window rotates by QRPS slots per sub-block,
-// so the current sub-block always sits in slots 0..QRPS-1.
-__device__ __forceinline__ int slot_of(int k, int S) { return (k / QTPR - QRPS * S) & (QCPT - 1); }
 
 // Scale and zero of the group starting at in-block column c, from the row's
 // current values: each part reduces its registers whose column lies in
-// [c, c + gs) and below bw, then the QTPR parts combine.
-__device__ __forceinline__ void group_grid(const float (&w)[QCPT], int S, int part, int c, int gs,
-                                           int bw, float maxq, float& s, float& z)
+// [c, c + gs) and below bw, then the row's QTPR parts combine.
+__device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int c, int gs, int bw,
+                                           float maxq, float& s, float& z)
 {
     float mn = 0.f, mx = 0.f;
 #pragma unroll
-    for (int mm = 0; mm < QCPT; ++mm) {
-        const int col = QTPR * ((mm + QRPS * S) & (QCPT - 1)) + part;
+    for (int k = 0; k < QCPT; ++k) {
+        const int col = QCPT * part + k;
         const bool in = col >= c && col < c + gs && col < bw;
-        const float v = in ? w[mm] : 0.f;
+        const float v = in ? w[k] : 0.f;
         mn = fminf(mn, v);
         mx = fmaxf(mx, v);
     }
@@ -103,59 +146,41 @@ __device__ __forceinline__ void group_grid(const float (&w)[QCPT], int S, int pa
 }
 
 // One lazy-batch block [j0, j0 + bw) of the column loop for QROWS rows.
-// Part p of a row holds columns 8m + p of the block in 16 registers.  Per
-// column c every part knows the row's current value through `nxt` (a copy of
-// column c+1 fetched one step early with a shuffle), computes the same q and
-// e, and corrects its own registers with U row c from shared memory.  The U
-// rows are stored in the register order of their sub-block, in which columns
-// already quantized have coefficient 0.  Only 16 steps are unrolled; the
-// window rotates after each sub-block, which keeps the code small enough for
-// the instruction cache.  Nothing is stored inside a step: the step's U row
-// is read first, errors and codes stay in registers until the sub-block ends.
+// Per column c every lane of the row knows the row's current value through
+// `nxt` (column c+1 fetched one step early with a shuffle from its owner and
+// corrected by this step's error), computes the same q and e, writes e, the
+// code and w^ to global memory, and corrects its own registers with U row c.
+// Columns at and before c have coefficient 0 in the laid-out U rows, so the
+// register file is updated whole and stays compile-time indexed; a 16-step
+// sub-block is unrolled (the half of the 32-register window it sits in is
+// chosen by a select).
 // kGroupsInStep: a group may start inside a 16-column sub-block (group sizes
 // that are not multiples of 16); otherwise groups start at sub-block starts.
 template <bool kGroupsInStep>
-__global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
+__global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
 {
-    extern __shared__ __align__(16) float qsm[];
-    float* Ut = qsm;                         // [c][p][slot]
-    float* rdiag = qsm + QB * UT_LD;         // 1 / U[c][c]
-    float* Es = rdiag + QB;                  // [row][c] errors e
-    uint8_t* Cs = reinterpret_cast<uint8_t*>(Es + QROWS * ES_LD);  // [row][c] codes
+    extern __shared__ __align__(128) uint8_t qsm_raw[];
+    float* Ut = reinterpret_cast<float*>(qsm_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qsm_raw + QNSUB * UCH_BYTES);
+    int* abort_flag = reinterpret_cast<int*>(bars + QNSUB);
     const int tid = threadIdx.x;
     const int j0 = a.j0, bw = a.bw, d_in = a.d_in;
+    const int nsub = (bw + QSUB - 1) / QSUB;
+    const int nch_blk = (a.block + QSUB - 1) / QSUB;
 
-    // U block: 128 rows x 32 float4 loads, 8 in flight per thread
-#pragma unroll 1
-    for (int base = 0; base < QB * (QB / 4); base += QTHREADS * 8) {
-        float4 v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int idx = base + i * QTHREADS + tid;
-            const int c = idx / (QB / 4), k = (idx % (QB / 4)) * 4;
-            v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (c < bw && k < bw)
-                v[i] = *reinterpret_cast<const float4*>(a.U + static_cast<int64_t>(j0 + c) * d_in + j0 + k);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int idx = base + i * QTHREADS + tid;
-            const int c = idx / (QB / 4), k = (idx % (QB / 4)) * 4;
-            const int S = c / QSUB;
-            const float e4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int kk = k + t;
-                Ut[c * UT_LD + (kk % QTPR) * UT_PART + slot_of(kk, S)] = (kk > c && kk < bw) ? e4[t] : 0.f;
-            }
-            if (k <= c && c < k + 4 && c < bw) {
-                const int t = c - k;
-                const float dv = t == 0 ? v[i].x : t == 1 ? v[i].y : t == 2 ? v[i].z : v[i].w;
-                rdiag[c] = 1.f / dv;
-            }
-        }
+    if (tid == 0) {
+        for (int S = 0; S < QNSUB; ++S) mbar_init(&bars[S], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
     }
     __syncthreads();
+    if (tid == 0) {
+        const float* src = a.Ul + static_cast<int64_t>(j0 / a.block) * nch_blk * UCH_FLOATS;
+        for (int S = 0; S < nsub; ++S) {
+            mbar_arrive_expect_tx(&bars[S], UCH_BYTES);
+            bulk_load(qsm_raw + S * UCH_BYTES, src + S * UCH_FLOATS, UCH_BYTES, &bars[S]);
+        }
+    }
 
     const int lrow = tid / QTPR, part = tid % QTPR;
     const int r = blockIdx.x * QROWS + lrow;
@@ -163,12 +188,19 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
     const int lane = tid & 31;
     const int lane_base = lane & ~(QTPR - 1);
     const float maxq = static_cast<float>((1 << a.bits) - 1);
-    const int64_t rowoff = static_cast<int64_t>(r) * d_in;
+    const int64_t rowoff = static_cast<int64_t>(valid ? r : 0) * d_in;
 
     float w[QCPT];
 #pragma unroll
-    for (int m = 0; m < QCPT; ++m)
-        w[m] = (valid && QTPR * m + part < bw) ? a.Wp[rowoff + j0 + QTPR * m + part] : 0.f;
+    for (int m = 0; m < QCPT / 4; ++m) {
+        const int col = QCPT * part + 4 * m;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid && col < bw) v = *reinterpret_cast<const float4*>(a.Wp + rowoff + j0 + col);
+        w[4 * m] = v.x;
+        w[4 * m + 1] = v.y;
+        w[4 * m + 2] = v.z;
+        w[4 * m + 3] = v.w;
+    }
 
     // grid of the group in effect at the block start
     float s = 1.f, z = 0.f;
@@ -205,103 +237,74 @@ __global__ void __launch_bounds__(QTHREADS) gptq_block_kernel(QArgs a)
     const int gs_in = (a.gs > 0 && a.gs <= a.block) ? a.gs : 0;
     int next_group = gs_in ? 0 : 1 << 30;
 
+    float* e_out = a.E + static_cast<int64_t>(valid ? r : 0) * kOuterMax + a.e_off;
+    uint8_t* q_out = a.codes_p + rowoff + j0;
+    float* w_out = a.Wp + rowoff + j0;
+
     float errsum = 0.f;
-    float nxt = __shfl_sync(0xffffffffu, w[0], lane_base | 0);   // column 0
-    const int nsub = (bw + QSUB - 1) / QSUB;
+    float nxt = __shfl_sync(0xffffffffu, w[0], lane_base);   // column 0 (part 0)
 
 #pragma unroll 1
     for (int S = 0; S < nsub; ++S) {
-        const float* ub = Ut + S * QSUB * UT_LD;
-        const float* rd = rdiag + S * QSUB;
-        if (!kGroupsInStep && S * QSUB == next_group) {
-            group_grid(w, S, part, S * QSUB, gs_in, bw, maxq, s, z);
+        const bool got = mbar_wait_bounded(&bars[S], 0, abort_flag, a.status);
+        if (!__syncthreads_and(got)) break;
+        const float* ub = Ut + S * UCH_FLOATS;
+        const float2* pairs = reinterpret_cast<const float2*>(ub + QSUB * UT_LD);
+        const bool hi = (S & 1) != 0;                 // sub-block sits in registers 16..31
+        const int src_in = lane_base | (S >> 1);      // owner of columns 16S .. 16S+15
+        const int src_next = lane_base | min((S + 1) >> 1, QTPR - 1);
+        const int cbase = S * QSUB;
+        if (!kGroupsInStep && cbase == next_group) {
+            group_grid(w, part, cbase, gs_in, bw, maxq, s, z);
             rs = 1.f / s;
             if (valid && part == 0) {
-                const int g = (j0 + S * QSUB) / gs_in;
+                const int g = (j0 + cbase) / gs_in;
                 a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
                 a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
             }
             next_group += gs_in;
         }
-        float e_own[QRPS], q_own[QRPS];
-#pragma unroll
-        for (int i = 0; i < QRPS; ++i) e_own[i] = q_own[i] = 0.f;
 #pragma unroll
         for (int cl = 0; cl < QSUB; ++cl) {
-            const int c = S * QSUB + cl;
-            if (c < bw) {
-                const int m = cl / QTPR, po = cl % QTPR;
-                const int mn1 = (cl + 1) / QTPR, pn1 = (cl + 1) % QTPR;
-                const float* urow = ub + cl * UT_LD;
-                // operands of this step that do not depend on its error
-                float u[QCPT];
+            const int c = cbase + cl;
+            const float* urow = ub + cl * UT_LD + part * UT_PART;
+            float u[QCPT];
 #pragma unroll
-                for (int mm = (m & ~3); mm < QCPT; mm += 4) {
-                    const float4 u4 = *reinterpret_cast<const float4*>(urow + part * UT_PART + mm);
-                    u[mm] = u4.x;
-                    u[mm + 1] = u4.y;
-                    u[mm + 2] = u4.z;
-                    u[mm + 3] = u4.w;
-                }
-                const float unext = urow[pn1 * UT_PART + mn1];
-                const float rdc = rd[cl];
-                // column c+1 after the corrections of steps < c (its owner's register)
-                const float pre = __shfl_sync(0xffffffffu, w[mn1], lane_base | pn1);
-                if (kGroupsInStep && c == next_group) {
-                    group_grid(w, S, part, c, gs_in, bw, maxq, s, z);
-                    rs = 1.f / s;
-                    if (valid && part == 0) {
-                        const int g = (j0 + c) / gs_in;
-                        a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
-                        a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
-                    }
-                    next_group += gs_in;
-                }
-                const float wc = nxt;
-                float q = rint_div(wc, s, rs) + z;
-                q = fminf(fmaxf(q, 0.f), maxq);
-                const float what = s * (q - z);
-                const float e = (wc - what) * rdc;
-                nxt = fmaf(-e, unext, pre);
-                if (part == po) {
-                    w[m] = what;
-                    e_own[m] = e;
-                    q_own[m] = q;
-                    errsum = fmaf(e, e, errsum);
-                }
-#pragma unroll
-                for (int mm = m; mm < QCPT; ++mm) w[mm] = fmaf(-e, u[mm], w[mm]);
+            for (int k = 0; k < QCPT; k += 4) {
+                const float4 u4 = *reinterpret_cast<const float4*>(urow + k);
+                u[k] = u4.x;
+                u[k + 1] = u4.y;
+                u[k + 2] = u4.z;
+                u[k + 3] = u4.w;
             }
-        }
-        // sub-block S is final in slots 0..QRPS-1: store, then rotate the window
-#pragma unroll
-        for (int i = 0; i < QRPS; ++i) {
-            const int col = S * QSUB + QTPR * i + part;
-            if (col < bw) {
-                if (valid) a.Wp[rowoff + j0 + col] = w[i];
-                Es[lrow * ES_LD + col] = e_own[i];
-                Cs[lrow * ES_LD + col] = static_cast<uint8_t>(q_own[i]);
+            const float2 rn = pairs[cl];   // (1 / U[c][c], U[c][c+1])
+            // column c+1 after the corrections of steps < c, from its owner
+            const float cand = hi ? w[(QSUB + 1 + cl) & (QCPT - 1)] : w[cl + 1];
+            const float pre = __shfl_sync(0xffffffffu, cand, cl + 1 < QSUB ? src_in : src_next);
+            if (kGroupsInStep && c == next_group && c < bw) {
+                group_grid(w, part, c, gs_in, bw, maxq, s, z);
+                rs = 1.f / s;
+                if (valid && part == 0) {
+                    const int g = (j0 + c) / gs_in;
+                    a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
+                    a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
+                }
+                next_group += gs_in;
             }
-        }
-        float t[QRPS];
+            const float wc = nxt;
+            float q = rint_div(wc, s, rs) + z;
+            q = fminf(fmaxf(q, 0.f), maxq);
+            const float what = s * (q - z);
+            const float e = (wc - what) * rn.x;
+            nxt = fmaf(-e, rn.y, pre);
+            errsum = fmaf(e, e, errsum);
+            if (valid && c < bw) {
+                e_out[c] = e;
+                q_out[c] = static_cast<uint8_t>(q);
+                w_out[c] = what;
+            }
 #pragma unroll
-        for (int i = 0; i < QRPS; ++i) t[i] = w[i];
-#pragma unroll
-        for (int i = 0; i < QCPT - QRPS; ++i) w[i] = w[i + QRPS];
-#pragma unroll
-        for (int i = 0; i < QRPS; ++i) w[QCPT - QRPS + i] = t[i];
-    }
-
-#pragma unroll
-    for (int o = 1; o < QTPR; o <<= 1) errsum += __shfl_xor_sync(0xffffffffu, errsum, o);
-    __syncthreads();
-    // errors and codes of the CTA's rows, row-contiguous
-    for (int idx = tid; idx < QROWS * QB; idx += QTHREADS) {
-        const int rl = idx / QB, c = idx % QB;
-        const int rr = blockIdx.x * QROWS + rl;
-        if (rr < a.d_out && c < bw) {
-            a.E[static_cast<int64_t>(rr) * kOuterMax + a.e_off + c] = Es[rl * ES_LD + c];
-            a.codes_p[static_cast<int64_t>(rr) * d_in + j0 + c] = Cs[rl * ES_LD + c];
+            for (int k = 0; k < QCPT; ++k) w[k] = fmaf(-e, u[k], w[k]);
         }
     }
     if (valid && a.err_sq && part == 0) a.err_sq[r] += errsum;
@@ -420,12 +423,19 @@ inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+// Sub-block chunks of the U layout for any block width 8..128: each block of
+// width bw has ceil(bw / 16) <= bw / 8 chunks, plus one for a ragged last block.
+inline size_t u_layout_bytes(int64_t d_in)
+{
+    return static_cast<size_t>(d_in / 8 + 16) * UCH_BYTES;
+}
+
 size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
 {
     const size_t n = static_cast<size_t>(d_out) * static_cast<size_t>(d_in);
     return 256 + up256(n * sizeof(float)) + up256(n) +
            up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)) +
-           up256(static_cast<size_t>(d_in) * sizeof(int32_t));
+           up256(static_cast<size_t>(d_in) * sizeof(int32_t)) + up256(u_layout_bytes(d_in));
 }
 
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64, int64_t d_in64,
@@ -441,6 +451,8 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
     float* E = reinterpret_cast<float*>(ws + 256 + up256(n * sizeof(float)) + up256(n));
     int32_t* inv = reinterpret_cast<int32_t*>(ws + 256 + up256(n * sizeof(float)) + up256(n) +
                                               up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)));
+    float* Ul = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(inv) +
+                                         up256(static_cast<size_t>(d_in) * sizeof(int32_t)));
     const int nsm = sm_count();
     int* status = device_status_ptr();
     const int n_groups = gs > 0 ? d_in / gs : 1;
@@ -460,6 +472,11 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
     // groups start only at 16-column sub-block starts when group_size is a
     // multiple of 16 that fits the block (or there are no in-block groups)
     const bool groups_in_step = gs > 0 && gs <= block && (gs % QSUB) != 0;
+
+    const int nch_blk = (block + QSUB - 1) / QSUB;
+    const int n_blocks = (d_in + block - 1) / block;
+    u_layout_kernel<<<n_blocks * nch_blk, 256, 0, stream>>>(U, d_in, block, nch_blk, Ul);
+    GPTQ_LAUNCH_CHECK();
 
     float* work = W;
     if (perm) {
@@ -494,8 +511,8 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
         const int J1 = (d_in - J0 < outer) ? d_in : J0 + outer;
         for (int j0 = J0; j0 < J1; j0 += block) {
             const int bw = (J1 - j0 < block) ? J1 - j0 : block;
-            QArgs a{work, U, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
-                    codes_p, E, j0 - J0, err_sq};
+            QArgs a{work, Ul, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
+                    codes_p, E, j0 - J0, err_sq, status};
             if (groups_in_step)
                 gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
             else
