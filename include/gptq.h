@@ -212,6 +212,14 @@ int gptq_quantize_static_scratch(float *W, const float *Hinv_chol, const int32_t
  * designed.  The device stays usable afterwards.  Synchronises the device. */
 int gptq_selftest_bounded_wait(int64_t limit_cycles);
 
+/* Diagnostic of the column loop's division-free quotient (the rounding of
+ * w / s that decides each code): evaluates it on n_pairs > 0 operand pairs
+ * drawn from `seed` (log-uniform scales over 2^-40 .. 2^20, scales with
+ * all-ones significands, and quotients within 4 ulps of a half-integer) and
+ * stores in *mismatches how many differ from IEEE round-to-nearest division.
+ * Expected 0.  Uses the default stream and synchronises the device. */
+int gptq_selftest_quotient(int64_t n_pairs, uint64_t seed, int64_t* mismatches);
+
 /* dst[i] = (float) bf16 src[i] (exact widening), n >= 0 elements. */
 int gptq_bf16_to_f32(float *dst, const uint16_t *src, int64_t n, void *stream);
 

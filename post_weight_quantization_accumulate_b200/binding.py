@@ -37,6 +37,7 @@ SIGNATURES = [
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize_static_scratch", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     ("gptq_selftest_bounded_wait", _I, [_I64]),
+    ("gptq_selftest_quotient", _I, [_I64, ctypes.c_uint64, _P]),
     ("gptq_bf16_to_f32", _I, [_P, _P, _I64, _P]),
 ]
 
@@ -198,6 +199,15 @@ def gptq_quantize_static_scratch(W: torch.Tensor, Hinv_chol: torch.Tensor, perm:
 def gptq_selftest_bounded_wait(limit_cycles: int) -> int:
     """Status of a deliberately unsatisfied, bounded device wait (expect 5)."""
     return lib().gptq_selftest_bounded_wait(int(limit_cycles))
+
+
+def gptq_selftest_quotient(n_pairs: int, seed: int = 0) -> int:
+    """Mismatches of the column loop's division-free quotient against IEEE
+    division over n_pairs device-generated operand pairs (expect 0)."""
+    out = ctypes.c_int64(-1)
+    _check("gptq_selftest_quotient",
+           lib().gptq_selftest_quotient(int(n_pairs), ctypes.c_uint64(seed), ctypes.byref(out)))
+    return out.value
 
 
 def gptq_bf16_to_f32(dst: torch.Tensor, src: torch.Tensor, stream=None):

@@ -20,6 +20,7 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                  int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
                  uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, cudaStream_t s);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
+int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
@@ -284,6 +285,14 @@ int gptq_selftest_bounded_wait(int64_t limit_cycles)
     bounded_wait_selftest_kernel<<<1, 32>>>(limit_cycles, status);
     GPTQ_LAUNCH_CHECK();
     return gptq_device_status();
+}
+
+int gptq_selftest_quotient(int64_t n_pairs, uint64_t seed, int64_t* mismatches)
+{
+    if (n_pairs <= 0 || !mismatches) return GPTQ_ERR_INVALID_ARG;
+    int rc = check_device();
+    if (rc) return rc;
+    return run_quotient_selftest(n_pairs, seed, mismatches);
 }
 
 int gptq_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, void* stream)

@@ -13,12 +13,13 @@
 //   q = clamp(rint(w_c / s) + z, 0, maxq);  w^ = s (q - z);  e = (w_c - w^) / U[c][c]
 //   w[c+1 : block end] -= e U[c][c+1 : block end]         (fused kernel, registers)
 //   W[:, block end:]    -= E_blk U[blk, block end:]        (once per block, GEMM)
-// Rows are independent once U is known.  Each row is split over 4 adjacent
-// lanes of a warp; lane part p holds the row's in-block columns 32p..32p+31 in
-// registers.  Every lane of the row computes the same (q, e) for the current
-// column and corrects its own 32 registers with U row c from shared memory.
-// The block's U rows are laid out once per call by u_layout_kernel and arrive
-// in shared memory by bulk copies, one per 16-column sub-block.
+// Rows are independent once U is known.  A lane holds two rows and 16 of
+// their in-block columns in registers (part p of 8 lanes: columns 16p ..
+// 16p+15), so each U value read from shared memory serves two rows.  Every
+// lane of a row pair computes the same (q, e) for the current column of both
+// rows and corrects its own registers with U row c.  The block's U rows are
+// laid out once per call by u_layout_kernel and arrive in shared memory by
+// bulk copies, one per 16-column sub-block.
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -28,16 +29,18 @@ namespace {
 
 constexpr int QB = 128;           // largest block width
 constexpr int kOuterMax = 1024;   // widest outer window of the two-level lazy batch
-constexpr int QTPR = 4;           // lanes per row
-constexpr int QCPT = QB / QTPR;   // registers per lane: part p holds columns 32p .. 32p+31
-constexpr int QSUB = 16;          // columns per unrolled sub-block (one bulk copy each)
+constexpr int QTPR = 8;           // lanes per row pair
+constexpr int QCPT = QB / QTPR;   // 16 registers per row: part p holds columns 16p .. 16p+15
+constexpr int QSUB = 16;          // columns per sub-block = one part's columns
 constexpr int QNSUB = QB / QSUB;
-constexpr int QROWS = 32;         // rows per CTA
-constexpr int QTHREADS = QROWS * QTPR;
-// U rows of a sub-block: [16 rows][4 parts][40] (32 coefficients + 8 pad, so the
-// four parts of a row fall in distinct bank groups), then 16 pairs
+constexpr int QPAIRS = 16;        // row pairs per CTA
+constexpr int QROWS = 2 * QPAIRS;
+constexpr int QTHREADS = QPAIRS * QTPR;
+static_assert(QSUB == QCPT, "sub-block S is the register range of part S");
+// U rows of a sub-block: [16 rows][8 parts][20] (16 coefficients + 4 pad, so
+// the 8 parts of a row fall in distinct 16-byte bank groups), then 16 pairs
 // (1 / U[c][c], U[c][c+1]).
-constexpr int UT_PART = QCPT + 8;
+constexpr int UT_PART = QCPT + 4;
 constexpr int UT_LD = QTPR * UT_PART;
 constexpr int UCH_FLOATS = QSUB * UT_LD + 2 * QSUB;
 constexpr int UCH_BYTES = UCH_FLOATS * 4;          // 10368, a multiple of 16
@@ -59,7 +62,7 @@ struct QArgs {
 
 // Sub-block layout of U's diagonal blocks: chunk (b, S) covers rows
 // j0 + 16S .. j0 + 16S + 15 of block b (j0 = b * block, width bw).  Entry
-// [cl][p][k] is U[j0+c][j0+32p+k] for in-block column 32p+k > c (zero on and
+// [cl][p][k] is U[j0+c][j0+16p+k] for in-block column 16p+k > c (zero on and
 // below the diagonal and beyond bw); pair cl is (1 / U[c][c], U[c][c+1]),
 // zero past bw.  One CTA per chunk.
 __global__ void u_layout_kernel(const float* __restrict__ U, int d_in, int block, int nch_blk,
@@ -109,22 +112,20 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, 
     z = rintf(__fdiv_rn(-mn, s));
 }
 
-// rint(w / s) with w / s correctly rounded, from the product t = w * rs (rs the
-// correctly rounded 1 / s).  t is within 2^-23 relative of w / s, so the two
-// round to the same integer unless t lies that close to a half-integer; only
-// then is the division carried out.
-__device__ __forceinline__ float rint_div(float w, float s, float rs)
+// w / s correctly rounded, without a division: t = w * rs with rs = RN(1 / s),
+// then one correction with the exact residual fma(-t, s, w) (Markstein's
+// correction step, P. Markstein, "IA-64 and Elementary Functions", 2000).
+// Being free of branches it keeps the unrolled column steps one basic block.
+// gptq_selftest_quotient compares it with IEEE division on the device.
+__device__ __forceinline__ float div_rn(float w, float s, float rs)
 {
     const float t = w * rs;
-    const float r = rintf(t);
-    const float thr = fmaf(-4.8e-7f, fmaxf(fabsf(t), 1.f), 0.5f);
-    if (fabsf(t - r) >= thr) return rintf(__fdiv_rn(w, s));
-    return r;
+    return fmaf(fmaf(-t, s, w), rs, t);
 }
 
-// Scale and zero of the group starting at in-block column c, from the row's
+// Scale and zero of the group starting at in-block column c, from one row's
 // current values: each part reduces its registers whose column lies in
-// [c, c + gs) and below bw, then the row's QTPR parts combine.
+// [c, c + gs) and below bw, then the QTPR parts of the row pair combine.
 __device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int c, int gs, int bw,
                                            float maxq, float& s, float& z)
 {
@@ -146,16 +147,17 @@ __device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int
 }
 
 // One lazy-batch block [j0, j0 + bw) of the column loop for QROWS rows.
-// Per column c every lane of the row knows the row's current value through
-// `nxt` (column c+1 fetched one step early with a shuffle from its owner and
-// corrected by this step's error), computes the same q and e, writes e, the
-// code and w^ to global memory, and corrects its own registers with U row c.
-// Columns at and before c have coefficient 0 in the laid-out U rows, so the
-// register file is updated whole and stays compile-time indexed; a 16-step
-// sub-block is unrolled (the half of the 32-register window it sits in is
-// chosen by a select).
+// Per column c every lane of a row pair knows both rows' current values
+// through `nxt` (column c+1 fetched one step early with a shuffle from its
+// owner and corrected by this step's error), computes the same q and e, and
+// corrects its own registers with U row c.  Columns at and before c have
+// coefficient 0 in the laid-out U rows, so the registers are updated whole
+// and stay compile-time indexed.  Lane part p keeps the results of steps 2p
+// and 2p+1 of a sub-block and writes them (e, w^, codes) with one vector
+// store each when the sub-block ends.
 // kGroupsInStep: a group may start inside a 16-column sub-block (group sizes
-// that are not multiples of 16); otherwise groups start at sub-block starts.
+// that are not multiples of 16); otherwise groups start at sub-block starts
+// and w^ is formed from the code at the store.
 template <bool kGroupsInStep>
 __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
 {
@@ -182,67 +184,76 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
         }
     }
 
-    const int lrow = tid / QTPR, part = tid % QTPR;
-    const int r = blockIdx.x * QROWS + lrow;
-    const bool valid = r < a.d_out;
+    const int pair = tid / QTPR, part = tid % QTPR;
     const int lane = tid & 31;
     const int lane_base = lane & ~(QTPR - 1);
     const float maxq = static_cast<float>((1 << a.bits) - 1);
-    const int64_t rowoff = static_cast<int64_t>(valid ? r : 0) * d_in;
-
-    float w[QCPT];
+    int r[2];
+    bool valid[2];
+    int64_t rowoff[2];
 #pragma unroll
-    for (int m = 0; m < QCPT / 4; ++m) {
-        const int col = QCPT * part + 4 * m;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid && col < bw) v = *reinterpret_cast<const float4*>(a.Wp + rowoff + j0 + col);
-        w[4 * m] = v.x;
-        w[4 * m + 1] = v.y;
-        w[4 * m + 2] = v.z;
-        w[4 * m + 3] = v.w;
+    for (int h = 0; h < 2; ++h) {
+        r[h] = blockIdx.x * QROWS + 2 * pair + h;
+        valid[h] = r[h] < a.d_out;
+        rowoff[h] = static_cast<int64_t>(valid[h] ? r[h] : 0) * d_in;
     }
+
+    float w[2][QCPT];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int m = 0; m < QCPT / 4; ++m) {
+            const int col = QCPT * part + 4 * m;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (valid[h] && col < bw) v = *reinterpret_cast<const float4*>(a.Wp + rowoff[h] + j0 + col);
+            w[h][4 * m] = v.x;
+            w[h][4 * m + 1] = v.y;
+            w[h][4 * m + 2] = v.z;
+            w[h][4 * m + 3] = v.w;
+        }
 
     // grid of the group in effect at the block start
-    float s = 1.f, z = 0.f;
-    if (a.gs < 0) {
-        if (valid) {
-            s = a.scales[r];
-            z = a.zeros[r];
-        }
-    } else if (a.gs > a.block) {
-        const int g = j0 / a.gs;
-        if (j0 % a.gs == 0) {
-            float mn = 0.f, mx = 0.f;
-            for (int k = part; k < a.gs; k += QTPR) {
-                const float v = valid ? a.Wp[rowoff + j0 + k] : 0.f;
-                mn = fminf(mn, v);
-                mx = fmaxf(mx, v);
-            }
+    float s[2] = {1.f, 1.f}, z[2] = {0.f, 0.f};
 #pragma unroll
-            for (int o = 1; o < QTPR; o <<= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int h = 0; h < 2; ++h) {
+        if (a.gs < 0) {
+            if (valid[h]) {
+                s[h] = a.scales[r[h]];
+                z[h] = a.zeros[r[h]];
             }
-            grid_from_range(mn, mx, maxq, s, z);
-            if (valid && part == 0) {
-                a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
-                a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
+        } else if (a.gs > a.block) {
+            const int g = j0 / a.gs;
+            if (j0 % a.gs == 0) {
+                float mn = 0.f, mx = 0.f;
+                for (int k = part; k < a.gs; k += QTPR) {
+                    const float v = valid[h] ? a.Wp[rowoff[h] + j0 + k] : 0.f;
+                    mn = fminf(mn, v);
+                    mx = fmaxf(mx, v);
+                }
+#pragma unroll
+                for (int o = 1; o < QTPR; o <<= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
+                grid_from_range(mn, mx, maxq, s[h], z[h]);
+                if (valid[h] && part == 0) {
+                    a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g] = s[h];
+                    a.zeros[static_cast<int64_t>(r[h]) * a.n_groups + g] = z[h];
+                }
+            } else if (valid[h]) {
+                s[h] = a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g];
+                z[h] = a.zeros[static_cast<int64_t>(r[h]) * a.n_groups + g];
             }
-        } else if (valid) {
-            s = a.scales[static_cast<int64_t>(r) * a.n_groups + g];
-            z = a.zeros[static_cast<int64_t>(r) * a.n_groups + g];
         }
     }
-    float rs = 1.f / s;
+    float rs[2] = {1.f / s[0], 1.f / s[1]};
     const int gs_in = (a.gs > 0 && a.gs <= a.block) ? a.gs : 0;
     int next_group = gs_in ? 0 : 1 << 30;
 
-    float* e_out = a.E + static_cast<int64_t>(valid ? r : 0) * kOuterMax + a.e_off;
-    uint8_t* q_out = a.codes_p + rowoff + j0;
-    float* w_out = a.Wp + rowoff + j0;
-
-    float errsum = 0.f;
-    float nxt = __shfl_sync(0xffffffffu, w[0], lane_base);   // column 0 (part 0)
+    float errsum[2] = {0.f, 0.f};
+    float nxt[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) nxt[h] = __shfl_sync(0xffffffffu, w[h][0], lane_base);   // column 0
 
 #pragma unroll 1
     for (int S = 0; S < nsub; ++S) {
@@ -250,20 +261,23 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
         if (!__syncthreads_and(got)) break;
         const float* ub = Ut + S * UCH_FLOATS;
         const float2* pairs = reinterpret_cast<const float2*>(ub + QSUB * UT_LD);
-        const bool hi = (S & 1) != 0;                 // sub-block sits in registers 16..31
-        const int src_in = lane_base | (S >> 1);      // owner of columns 16S .. 16S+15
-        const int src_next = lane_base | min((S + 1) >> 1, QTPR - 1);
+        const int src_in = lane_base | S;                          // owner of this sub-block
+        const int src_next = lane_base | min(S + 1, QTPR - 1);     // owner of the next one
         const int cbase = S * QSUB;
         if (!kGroupsInStep && cbase == next_group) {
-            group_grid(w, part, cbase, gs_in, bw, maxq, s, z);
-            rs = 1.f / s;
-            if (valid && part == 0) {
-                const int g = (j0 + cbase) / gs_in;
-                a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
-                a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                group_grid(w[h], part, cbase, gs_in, bw, maxq, s[h], z[h]);
+                rs[h] = 1.f / s[h];
+                if (valid[h] && part == 0) {
+                    const int g = (j0 + cbase) / gs_in;
+                    a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g] = s[h];
+                    a.zeros[static_cast<int64_t>(r[h]) * a.n_groups + g] = z[h];
+                }
             }
             next_group += gs_in;
         }
+        float ke[2][2], kq[2][2], kw[2][2];   // results of steps 2*part, 2*part + 1
 #pragma unroll
         for (int cl = 0; cl < QSUB; ++cl) {
             const int c = cbase + cl;
@@ -278,36 +292,66 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                 u[k + 3] = u4.w;
             }
             const float2 rn = pairs[cl];   // (1 / U[c][c], U[c][c+1])
-            // column c+1 after the corrections of steps < c, from its owner
-            const float cand = hi ? w[(QSUB + 1 + cl) & (QCPT - 1)] : w[cl + 1];
-            const float pre = __shfl_sync(0xffffffffu, cand, cl + 1 < QSUB ? src_in : src_next);
+            // column c+1 of both rows after the corrections of steps < c
+            float pre[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                pre[h] = __shfl_sync(0xffffffffu, w[h][(cl + 1) % QCPT], cl + 1 < QSUB ? src_in : src_next);
             if (kGroupsInStep && c == next_group && c < bw) {
-                group_grid(w, part, c, gs_in, bw, maxq, s, z);
-                rs = 1.f / s;
-                if (valid && part == 0) {
-                    const int g = (j0 + c) / gs_in;
-                    a.scales[static_cast<int64_t>(r) * a.n_groups + g] = s;
-                    a.zeros[static_cast<int64_t>(r) * a.n_groups + g] = z;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    group_grid(w[h], part, c, gs_in, bw, maxq, s[h], z[h]);
+                    rs[h] = 1.f / s[h];
+                    if (valid[h] && part == 0) {
+                        const int g = (j0 + c) / gs_in;
+                        a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g] = s[h];
+                        a.zeros[static_cast<int64_t>(r[h]) * a.n_groups + g] = z[h];
+                    }
                 }
                 next_group += gs_in;
             }
-            const float wc = nxt;
-            float q = rint_div(wc, s, rs) + z;
-            q = fminf(fmaxf(q, 0.f), maxq);
-            const float what = s * (q - z);
-            const float e = (wc - what) * rn.x;
-            nxt = fmaf(-e, rn.y, pre);
-            errsum = fmaf(e, e, errsum);
-            if (valid && c < bw) {
-                e_out[c] = e;
-                q_out[c] = static_cast<uint8_t>(q);
-                w_out[c] = what;
-            }
+            const bool keep = part == cl / 2;
 #pragma unroll
-            for (int k = 0; k < QCPT; ++k) w[k] = fmaf(-e, u[k], w[k]);
+            for (int h = 0; h < 2; ++h) {
+                const float wc = nxt[h];
+                // q = clamp(rint(w / s) + z, 0, maxq) and w^ = s (q - z); with
+                // integer-valued floats, q - z = clamp(rint(w / s), -z, maxq - z)
+                const float qz = fminf(fmaxf(rintf(div_rn(wc, s[h], rs[h])), -z[h]), maxq - z[h]);
+                const float q = qz + z[h];
+                const float what = s[h] * qz;
+                const float e = (wc - what) * rn.x;
+                nxt[h] = fmaf(-e, rn.y, pre[h]);
+                errsum[h] = fmaf(e, e, errsum[h]);
+                if (keep) {
+                    ke[h][cl % 2] = e;
+                    kq[h][cl % 2] = q;
+                    if (kGroupsInStep) kw[h][cl % 2] = what;
+                }
+#pragma unroll
+                for (int k = 0; k < QCPT; ++k) w[h][k] = fmaf(-e, u[k], w[h][k]);
+            }
+        }
+        // this lane's two columns of the sub-block: e, w^ and the codes
+        const int col = cbase + 2 * part;
+        if (col < bw) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (!valid[h]) continue;
+                if (!kGroupsInStep) {
+                    kw[h][0] = s[h] * (kq[h][0] - z[h]);
+                    kw[h][1] = s[h] * (kq[h][1] - z[h]);
+                }
+                *reinterpret_cast<float2*>(a.E + static_cast<int64_t>(r[h]) * kOuterMax + a.e_off + col) =
+                    make_float2(ke[h][0], ke[h][1]);
+                *reinterpret_cast<float2*>(a.Wp + rowoff[h] + j0 + col) = make_float2(kw[h][0], kw[h][1]);
+                const uint32_t q2 = static_cast<uint32_t>(kq[h][0]) | (static_cast<uint32_t>(kq[h][1]) << 8);
+                *reinterpret_cast<uint16_t*>(a.codes_p + rowoff[h] + j0 + col) = static_cast<uint16_t>(q2);
+            }
         }
     }
-    if (valid && a.err_sq && part == 0) a.err_sq[r] += errsum;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        if (valid[h] && a.err_sq && part == 0) a.err_sq[r[h]] += errsum[h];
 }
 
 // One (scale, zero) per row from the whole original row (group_size = -1).
@@ -417,6 +461,52 @@ __global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ src, float* __re
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         dst[i] = __uint_as_float(static_cast<uint32_t>(src[i]) << 16);
+}
+
+// Counter-based test operands (splitmix64 finaliser) for the quotient check.
+__device__ __forceinline__ uint32_t st_mix(uint64_t x)
+{
+    x ^= x >> 33;
+    x *= 0xff51afd7ed558ccdULL;
+    x ^= x >> 33;
+    x *= 0xc4ceb9fe1a85ec53ULL;
+    x ^= x >> 33;
+    return static_cast<uint32_t>(x);
+}
+
+__device__ __forceinline__ float st_unif(uint64_t k) { return (st_mix(k) >> 8) * (1.0f / 16777216.0f); }
+
+__device__ unsigned long long g_quotient_bad;   // mismatch count of the self-test
+
+// div_rn against IEEE division on three operand families: s log-uniform in
+// [2^-40, 2^20] with |w / s| < 2^12, s with an all-ones significand, and w
+// within 4 ulps of (n + 1/2) s (quotients next to a rounding tie of rint).
+__global__ void quotient_selftest_kernel(uint64_t seed, int64_t n, unsigned long long* bad)
+{
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    unsigned long long local = 0;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
+        const uint64_t k = (seed << 40) ^ (4 * static_cast<uint64_t>(i));
+        const int mode = static_cast<int>(i % 3);
+        float s, w;
+        if (mode == 0) {
+            s = exp2f(-40.f + 60.f * st_unif(k));
+            w = s * (st_unif(k + 1) * 8192.f - 4096.f);
+        } else if (mode == 1) {
+            const int e = static_cast<int>(st_mix(k) % 60) - 40;
+            const uint32_t m = 0x7FFFFFu - (st_mix(k + 2) & 7u);
+            s = __uint_as_float((static_cast<uint32_t>(e + 127) << 23) | m);
+            w = s * (st_unif(k + 1) * 600.f - 300.f);
+        } else {
+            s = exp2f(-20.f + 24.f * st_unif(k));
+            const float m = floorf(st_unif(k + 1) * 600.f - 300.f);
+            const float w0 = (m + 0.5f) * s;
+            w = __uint_as_float(__float_as_uint(w0) + static_cast<int>(st_mix(k + 3) % 9) - 4);
+        }
+        const float rs = 1.f / s;
+        if (div_rn(w, s, rs) != __fdiv_rn(w, s)) ++local;
+    }
+    if (local) atomicAdd(bad, local);
 }
 
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -543,6 +633,20 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
         g_idx_kernel<<<(d_in + 255) / 256, 256, 0, stream>>>(perm, d_in, gs, g_idx);
         GPTQ_LAUNCH_CHECK();
     }
+    return GPTQ_OK;
+}
+
+int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches)
+{
+    void* p = nullptr;
+    GPTQ_CUDA_CHECK(cudaGetSymbolAddress(&p, g_quotient_bad));
+    unsigned long long* d = static_cast<unsigned long long*>(p);
+    GPTQ_CUDA_CHECK(cudaMemset(d, 0, sizeof(unsigned long long)));
+    quotient_selftest_kernel<<<sm_count() * 8, 256>>>(seed, n, d);
+    GPTQ_LAUNCH_CHECK();
+    unsigned long long h = 0;
+    GPTQ_CUDA_CHECK(cudaMemcpy(&h, d, sizeof h, cudaMemcpyDeviceToHost));
+    *mismatches = static_cast<int64_t>(h);
     return GPTQ_OK;
 }
 

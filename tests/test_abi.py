@@ -92,3 +92,5 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.gptq_hessian_accumulate_host(fake, fake, 16, 64, fake, 0, None) == 1
     assert lib.gptq_selftest_bounded_wait(0) == 1
     assert lib.gptq_selftest_bounded_wait(1 << 40) == 1
+    assert lib.gptq_selftest_quotient(0, 0, fake) == 1
+    assert lib.gptq_selftest_quotient(16, 0, None) == 1

@@ -267,3 +267,10 @@ def test_bounded_wait_times_out_and_device_stays_usable():
     assert B.gptq_device_status() == 0          # the word was read and cleared
     xb = _rand_x(9, 256, 64)
     np.testing.assert_allclose(_gpu_hessian(xb), oracle.hessian(xb), rtol=1e-5, atol=1e-3)
+
+
+def test_division_free_quotient_matches_ieee_division():
+    """The column loop decides each code from w / s rounded without a
+    division instruction; on the device it must agree with IEEE division on
+    random, all-ones-significand and near-tie operands."""
+    assert B.gptq_selftest_quotient(3 << 26, seed=7) == 0
