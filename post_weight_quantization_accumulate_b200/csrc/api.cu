@@ -15,10 +15,11 @@ int launch_mirror(float* H, int64_t d, cudaStream_t s);
 size_t prepare_workspace_bytes(int64_t d);
 size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in);
 int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* perm, float* U,
-                void* ws, cudaStream_t s, int* host_status);
+                void* ws, cudaStream_t s, int* host_status, bool graphed);
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
                  int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
-                 uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, cudaStream_t s);
+                 uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, cudaStream_t s,
+                 bool graphed);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
 
@@ -46,7 +47,18 @@ struct StreamPair {
 StreamPair g_streams[kMaxDevices];
 }  // namespace
 
-void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+namespace {
+thread_local uint64_t t_launches = 0;   // this thread's launches (graph capture accounting)
+}
+
+void note_launch()
+{
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    ++t_launches;
+}
+void note_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+void unnote_launches(uint64_t n) { g_launches.fetch_sub(n, std::memory_order_relaxed); }
+uint64_t launch_count() { return t_launches; }
 
 int cuda_fail(cudaError_t e)
 {
@@ -119,6 +131,33 @@ __global__ void bounded_wait_selftest_kernel(long long limit_cycles, int* status
     __syncthreads();
     if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, status, limit_cycles);
     __syncthreads();
+}
+
+// Argument checks and the column loop; `graphed` replays a cached CUDA graph
+// of the launch sequence (the allocation-free entry point enqueues directly).
+int quantize_entry(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
+                   int64_t d_in, int bits, int group_size, int block_size, uint8_t* codes,
+                   float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,
+                   float* err_sq, void* workspace, size_t ws_bytes, void* stream, bool graphed)
+{
+    if (!W || !Hinv_chol || !scales || !zeros || d_out <= 0 || d_in <= 0 || d_in > kMaxDim ||
+        d_out > (int64_t(1) << 31) / 2 || d_in % 8 != 0 || bits < 1 || bits > 8 ||
+        block_size < 8 || block_size > 128 || block_size % 8 != 0 || !aligned(W, 16))
+        return GPTQ_ERR_INVALID_ARG;
+    if (group_size != -1) {
+        if (group_size <= 0 || d_in % group_size != 0) return GPTQ_ERR_INVALID_ARG;
+        if (group_size % block_size != 0 && block_size % group_size != 0)
+            return GPTQ_ERR_INVALID_ARG;
+    }
+    if (packed_int4 && bits > 4) return GPTQ_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(d_out) * d_in >= (int64_t(1) << 40)) return GPTQ_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < quantize_workspace_bytes(d_out, d_in))
+        return GPTQ_ERR_WORKSPACE;
+    int rc = check_device();
+    if (rc) return rc;
+    return run_quantize(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
+                        scales, zeros, packed_int4, g_idx, err_sq, workspace,
+                        static_cast<cudaStream_t>(stream), graphed);
 }
 
 }  // namespace gptq
@@ -245,7 +284,7 @@ int gptq_prepare(const float* H, int64_t d_in, float damp, int act_order, int32_
     if (rc) return rc;
     int st = 0;
     rc = run_prepare(H, d_in, damp, act_order ? 1 : 0, perm, Hinv_chol, workspace,
-                     static_cast<cudaStream_t>(stream), &st);
+                     static_cast<cudaStream_t>(stream), &st, true);
     if (rc) return rc;
     return st;
 }
@@ -255,24 +294,9 @@ int gptq_quantize(float* W, const float* Hinv_chol, const int32_t* perm, int64_t
                   float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,
                   float* err_sq, void* workspace, size_t ws_bytes, void* stream)
 {
-    if (!W || !Hinv_chol || !scales || !zeros || d_out <= 0 || d_in <= 0 || d_in > kMaxDim ||
-        d_out > (int64_t(1) << 31) / 2 || d_in % 8 != 0 || bits < 1 || bits > 8 ||
-        block_size < 8 || block_size > 128 || block_size % 8 != 0 || !aligned(W, 16))
-        return GPTQ_ERR_INVALID_ARG;
-    if (group_size != -1) {
-        if (group_size <= 0 || d_in % group_size != 0) return GPTQ_ERR_INVALID_ARG;
-        if (group_size % block_size != 0 && block_size % group_size != 0)
-            return GPTQ_ERR_INVALID_ARG;
-    }
-    if (packed_int4 && bits > 4) return GPTQ_ERR_INVALID_ARG;
-    if (static_cast<int64_t>(d_out) * d_in >= (int64_t(1) << 40)) return GPTQ_ERR_INVALID_ARG;
-    if (!workspace || !aligned(workspace, 256) || ws_bytes < quantize_workspace_bytes(d_out, d_in))
-        return GPTQ_ERR_WORKSPACE;
-    int rc = check_device();
-    if (rc) return rc;
-    return run_quantize(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
-                        scales, zeros, packed_int4, g_idx, err_sq, workspace,
-                        static_cast<cudaStream_t>(stream));
+    return quantize_entry(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
+                          scales, zeros, packed_int4, g_idx, err_sq, workspace, ws_bytes, stream,
+                          true);
 }
 
 int gptq_selftest_bounded_wait(int64_t limit_cycles)

@@ -8,11 +8,25 @@
 
 #include "../../include/gptq.h"
 
+#include <functional>
+#include <vector>
+
 namespace gptq {
 
 // ---------------------------------------------------------------- host side
 // Records a launch (for gptq_launch_count) and checks the launch error.
 void note_launch();
+void note_launches(uint64_t n);     // a graph replay of n launches
+void unnote_launches(uint64_t n);   // launches recorded into a graph, not run
+uint64_t launch_count();            // launches recorded by the calling thread
+
+// Runs enqueue(stream, status_host) directly on `stream`, or replays a CUDA
+// graph captured from it for the same `key` (every argument that shapes the
+// launch sequence).  With want_status, *status_out is a pinned word that holds
+// the run's status after `stream` is synchronised.
+int run_graphed(const std::vector<uint64_t>& key, bool want_status,
+                const std::function<int(cudaStream_t, int*)>& enqueue, cudaStream_t stream,
+                int** status_out);
 int cuda_fail(cudaError_t e);          // stores the message, returns GPTQ_ERR_CUDA
 int* device_status_ptr();              // status word of the current device (device memory)
 int sm_count();                        // SMs of the current device

@@ -19,6 +19,7 @@
 #include "gemm.cuh"
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 namespace gptq {
@@ -564,8 +565,10 @@ static int side_stream(SideStream** out)
     return GPTQ_OK;
 }
 
-int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t* perm, float* U,
-                void* workspace, cudaStream_t stream, int* host_status)
+// Enqueues the whole factorisation on `stream`; the status word of the run
+// is copied into the pinned word status_host.
+static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t* perm,
+                           float* U, void* workspace, cudaStream_t stream, int* status_host)
 {
     const int d = static_cast<int>(d64);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -675,10 +678,39 @@ int run_prepare(const float* H, int64_t d64, float damp, int act_order, int32_t*
     reverse_upper_kernel<<<nsm * 8, 256, 0, stream>>>(Minv, d, U);
     GPTQ_LAUNCH_CHECK();
 
-    int st = 0;
-    GPTQ_CUDA_CHECK(cudaMemcpyAsync(&st, &hdr->status, sizeof(int), cudaMemcpyDeviceToHost, stream));
+    GPTQ_CUDA_CHECK(cudaMemcpyAsync(status_host, &hdr->status, sizeof(int), cudaMemcpyDeviceToHost,
+                                    stream));
+    return GPTQ_OK;
+}
+
+int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* perm, float* U,
+                void* workspace, cudaStream_t stream, int* host_status, bool graphed)
+{
+    uint32_t damp_bits = 0;
+    static_assert(sizeof damp_bits == sizeof damp, "float is 32-bit");
+    memcpy(&damp_bits, &damp, sizeof damp);
+    const std::vector<uint64_t> key = {1,
+                                       reinterpret_cast<uintptr_t>(H),
+                                       static_cast<uint64_t>(d),
+                                       damp_bits,
+                                       static_cast<uint64_t>(act_order),
+                                       reinterpret_cast<uintptr_t>(perm),
+                                       reinterpret_cast<uintptr_t>(U),
+                                       reinterpret_cast<uintptr_t>(workspace)};
+    auto enq = [&](cudaStream_t s, int* st) {
+        return enqueue_prepare(H, d, damp, act_order, perm, U, workspace, s, st);
+    };
+    int* st = nullptr;
+    int rc = graphed ? run_graphed(key, true, enq, stream, &st) : GPTQ_OK;
+    if (!graphed) {
+        static thread_local int* direct = nullptr;
+        if (!direct) GPTQ_CUDA_CHECK(cudaMallocHost(&direct, sizeof(int)));
+        st = direct;
+        rc = enq(stream, st);
+    }
+    if (rc) return rc;
     GPTQ_CUDA_CHECK(cudaStreamSynchronize(stream));
-    *host_status = st;
+    *host_status = *st;
     return GPTQ_OK;
 }
 

@@ -528,10 +528,10 @@ size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
            up256(static_cast<size_t>(d_in) * sizeof(int32_t)) + up256(u_layout_bytes(d_in));
 }
 
-int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64, int64_t d_in64,
-                 int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
-                 uint8_t* packed, int32_t* g_idx, float* err_sq, void* workspace,
-                 cudaStream_t stream)
+static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
+                            int64_t d_in64, int bits, int gs, int block, uint8_t* codes,
+                            float* scales, float* zeros, uint8_t* packed, int32_t* g_idx,
+                            float* err_sq, void* workspace, cudaStream_t stream)
 {
     const int d_out = static_cast<int>(d_out64), d_in = static_cast<int>(d_in64);
     const size_t n = static_cast<size_t>(d_out) * d_in;
@@ -634,6 +634,24 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
         GPTQ_LAUNCH_CHECK();
     }
     return GPTQ_OK;
+}
+
+int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in, int bits,
+                 int gs, int block, uint8_t* codes, float* scales, float* zeros, uint8_t* packed,
+                 int32_t* g_idx, float* err_sq, void* workspace, cudaStream_t stream, bool graphed)
+{
+    auto enq = [&](cudaStream_t s, int*) {
+        return enqueue_quantize(W, U, perm, d_out, d_in, bits, gs, block, codes, scales, zeros,
+                                packed, g_idx, err_sq, workspace, s);
+    };
+    if (!graphed) return enq(stream, nullptr);
+    auto P = [](const void* p) { return static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p)); };
+    const std::vector<uint64_t> key = {2, P(W), P(U), P(perm), static_cast<uint64_t>(d_out),
+                                       static_cast<uint64_t>(d_in), static_cast<uint64_t>(bits),
+                                       static_cast<uint64_t>(static_cast<int64_t>(gs)),
+                                       static_cast<uint64_t>(block), P(codes), P(scales), P(zeros),
+                                       P(packed), P(g_idx), P(err_sq), P(workspace)};
+    return run_graphed(key, false, enq, stream, nullptr);
 }
 
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches)
