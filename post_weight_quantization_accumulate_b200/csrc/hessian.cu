@@ -6,18 +6,26 @@
 // for calibration sets much larger than d.
 //
 // Design (B200):
-//  * H is symmetric, so only tiles meeting the upper triangle are computed:
-//    128 x 256 output tiles, (ti, tj) with tj >= ti / 2.  The strict lower
-//    triangle is written afterwards by a transpose copy (mirror_upper_kernel),
-//    so H is bitwise symmetric.
-//  * Both operands are slices of the same X rows: A = X[t, 128 i-cols],
-//    B = X[t, 256 j-cols].  Their contraction index (tokens) is the outer
-//    dimension of X, so both are MN-major; TMA brings 64-token x 64-column
-//    boxes with 128-byte swizzle, which is the canonical MN-major SW128
-//    layout tcgen05.mma reads directly.
+//  * H is symmetric, so only 256 x 256 output tiles (ti, tj) with tj >= ti
+//    are computed; the strict lower triangle is written afterwards by a
+//    transpose copy (mirror_upper_kernel), so H is bitwise symmetric.
+//  * A tile is computed by a pair of CTAs (a cluster of two on neighbouring
+//    SMs) with the pair form of the tensor-core MMA (M = 256, N = 256): CTA r
+//    of the pair holds the 128 rows 256 ti + 128 r (its A operand) and the
+//    128 columns 256 tj + 128 r (its half of B), and each SM keeps its 128 x
+//    256 accumulator in its own tensor memory.  Per SM and token this moves
+//    half of the B operand a single-CTA 128 x 256 tile would, which keeps the
+//    shared-memory traffic (TMA writes + MMA reads) under the shared-memory
+//    bandwidth at the full MMA rate.
+//  * Both operands are slices of the same X rows: A = X[t, rows], B = X[t,
+//    cols].  Their contraction index (tokens) is the outer dimension of X, so
+//    both are MN-major; TMA brings 64-token x 64-column boxes with 128-byte
+//    swizzle, the canonical MN-major SW128 layout tcgen05.mma reads.  Each CTA
+//    loads its own boxes (no multicast); the loads of both CTAs complete on
+//    the first CTA's barrier, whose thread issues the MMAs.
 //  * Work units = (tile, token span of kSpanTokens).  A persistent grid of
-//    one CTA per SM walks the units span-major, so concurrently running
-//    units read the same token rows of X (L2 reuse).
+//    one pair per two SMs walks the units span-major, so concurrently
+//    running units read the same token rows of X (L2 reuse).
 //  * Accumulation precision: the tensor core adds each MMA's result into the
 //    fp32 TMEM accumulator with a rounding that is biased for long chains
 //    (measured: sums of squares come out ~0.25 ulp low per MMA).  So a TMEM
@@ -25,77 +33,163 @@
 //    each chain into fp32 registers with round-to-nearest adds, and flushes
 //    the span's sum into H with one fp32 red.add per element.
 //  * Warp roles per CTA (384 threads, three warpgroups): warp 0 = TMA
-//    producer, warp 1 = MMA issuer + TMEM owner (warpgroup 0 gives its
-//    registers up to 56); warps 4-11 = epilogue (raised to 224 registers);
-//    warps w and w+4 share TMEM lanes 32*(w%4)..+31 and split the 256 columns
-//    in halves, 128 fp32 registers of running sum each.  The launch budget
-//    384 x 168 equals 128 x 56 + 256 x 224.  A 4-stage shared-memory ring (48 KB per
-//    stage) and two TMEM chain buffers (2 x 256 columns) let the promotion of
-//    one chain overlap the MMAs of the next.
-//  * Every mbarrier wait is bounded; a time-out records GPTQ_ERR_TIMEOUT,
-//    releases the other roles, and the CTA still frees its TMEM.
+//    producer, warp 1 = MMA issuer (first CTA of the pair) and TMEM owner
+//    (warpgroup 0 gives its registers up to 64); warps 4-11 = epilogue (raised
+//    to 216 registers); warps w and w+4 share TMEM lanes 32*(w%4)..+31 and
+//    split the 256 columns in halves, 128 fp32 registers of running sum each.
+//    128 x 64 + 256 x 216 = 63488 fits the launch budget 384 x 168.  A 6-stage
+//    shared-memory ring (32 KB per stage) and two TMEM chain buffers (2 x 256
+//    columns) let the promotion of one chain overlap the MMAs of the next.
+//  * Every mbarrier wait is bounded; a time-out records GPTQ_ERR_TIMEOUT and
+//    ends the role; both CTAs meet at a cluster barrier before the pair frees
+//    its tensor memory.
 #include "common.cuh"
 
+#include <algorithm>
 #include <mutex>
 
 namespace gptq {
 
 namespace {
 
-constexpr int kBM = 128;          // H rows per tile (UMMA M)
-constexpr int kBN = 256;          // H cols per tile (UMMA N)
+constexpr int kBM = 128;          // H rows per CTA (half of the pair's M = 256)
+constexpr int kBN = 256;          // H cols per tile (MMA N)
+constexpr int kTile = 256;        // tile edge
 constexpr int kBK = 64;           // tokens per pipeline stage
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kBoxCols = 64;      // 64 bf16 = 128 bytes = one swizzle row
 constexpr int kBoxBytes = kBK * kBoxCols * 2;           // 8 KB
-constexpr int kABytes = kBoxBytes * (kBM / kBoxCols);   // 16 KB
-constexpr int kBBytes = kBoxBytes * (kBN / kBoxCols);   // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;          // 48 KB
+constexpr int kABytes = kBoxBytes * (kBM / kBoxCols);   // 16 KB: 128 rows of A
+constexpr int kBBytes = kBoxBytes * (kBN / 2 / kBoxCols);  // 16 KB: this CTA's 128 columns of B
+constexpr int kStageBytes = kABytes + kBBytes;          // 32 KB
 constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr int kTmemCols = 512;    // two 256-column fp32 chain buffers
 constexpr int kChainTokens = 512; // tokens per TMEM accumulation chain
 constexpr int kSpanTokens = 16384;  // tokens per work unit (one flush into H)
-constexpr uint32_t kIdesc = idesc_f32acc(1 /*bf16*/, 1, 1, kBM, kBN);
+constexpr uint32_t kIdesc = idesc_f32acc(1 /*bf16*/, 1, 1, 2 * kBM, kBN);
 
 struct alignas(1024) HessSmem {
     uint8_t stage[kStages][kStageBytes];
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t full[kStages];     // first CTA: TMA bytes of both CTAs landed
+    uint64_t empty[kStages];    // MMAs done reading the stage (both CTAs)
+    uint64_t tfull[2];          // chain complete (both CTAs)
+    uint64_t tempty[2];         // first CTA: both epilogues drained the buffer
     uint32_t tmem_base;
     int abort;
 };
 constexpr size_t kSmemBytes = sizeof(HessSmem) + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "one CTA per SM");
 
-// Upper-triangle tile number -> (ti, tj); row block ti has tiles tj in
-// [ti/2, n_tj).
-__device__ __forceinline__ void tile_coords(int tile, int n_ti, int n_tj, int& ti, int& tj)
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank)
+{
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+    return out;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// barrier at cluster address `bar` (the first CTA's), pair form, no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x,
+                                                 int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on the barrier at this offset in both CTAs of the pair when
+// the MMAs issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar)
+{
+    const uint16_t mask = 3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(mask)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Upper-triangle tile number -> (ti, tj), tj >= ti.
+__device__ __forceinline__ void tile_coords(int tile, int n_t, int& ti, int& tj)
 {
     int idx = tile;
-    for (int i = 0; i < n_ti; ++i) {
-        int cnt = n_tj - (i >> 1);
+    for (int i = 0; i < n_t; ++i) {
+        const int cnt = n_t - i;
         if (idx < cnt) {
             ti = i;
-            tj = (i >> 1) + idx;
+            tj = i + idx;
             return;
         }
         idx -= cnt;
     }
-    ti = n_ti - 1;
-    tj = n_tj - 1;
+    ti = n_t - 1;
+    tj = n_t - 1;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int d,
-                      int n_tokens, int n_ti, int n_tj, int n_tiles, int n_split, int* status)
+                      int n_tokens, int n_t, int n_tiles, int n_split, int* status)
 {
     extern __shared__ uint8_t smem_raw[];
     HessSmem& S = *reinterpret_cast<HessSmem*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -104,53 +198,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&S.tfull[b], 1);
-            mbar_init(&S.tempty[b], kEpiWarps);
+            mbar_init(&S.tempty[b], 2 * kEpiWarps);
         }
         S.abort = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap);
     }
     if (warp == 1) {
-        tmem_alloc(&S.tmem_base, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(&S.tmem_base, kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();   // both CTAs' barriers and tensor memory exist before any use
     tc_fence_after();
     const uint32_t tbase = S.tmem_base;
     volatile int* abort = &S.abort;
     const int n_units = n_tiles * n_split;
 
     if (warp < 4) {
-        regs_dealloc<56>();
+        regs_dealloc<64>();
         if (warp == 0 && lane == 0) {
             uint32_t it = 0;
-            for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+            for (int u = pair; u < n_units && !*abort; u += n_pairs) {
                 int ti, tj;
-                tile_coords(u % n_tiles, n_ti, n_tj, ti, tj);
+                tile_coords(u % n_tiles, n_t, ti, tj);
                 const int t0 = (u / n_tiles) * kSpanTokens;
                 const int t1 = min(n_tokens, t0 + kSpanTokens);
+                const int col_a = ti * kTile + static_cast<int>(rank) * kBM;
+                const int col_b = tj * kTile + static_cast<int>(rank) * (kBN / 2);
                 bool ok = true;
                 for (int t = t0; t < t1 && ok; t += kBK, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S.full[s], kStageBytes);
+                    if (leader) mbar_arrive_expect_tx(&S.full[s], 2 * kStageBytes);
+                    const uint32_t fb = cluster_addr(&S.full[s], 0);
                     uint8_t* a = S.stage[s];
                     uint8_t* b = a + kABytes;
 #pragma unroll
                     for (int m = 0; m < kBM / kBoxCols; ++m)
-                        tma_load_2d(a + m * kBoxBytes, &tmap, &S.full[s], ti * kBM + m * kBoxCols, t);
+                        tma_load_2d_pair(a + m * kBoxBytes, &tmap, fb, col_a + m * kBoxCols, t);
 #pragma unroll
-                    for (int m = 0; m < kBN / kBoxCols; ++m)
-                        tma_load_2d(b + m * kBoxBytes, &tmap, &S.full[s], tj * kBN + m * kBoxCols, t);
+                    for (int m = 0; m < kBN / 2 / kBoxCols; ++m)
+                        tma_load_2d_pair(b + m * kBoxBytes, &tmap, fb, col_b + m * kBoxCols, t);
                 }
                 if (!ok) break;
             }
-        } else if (warp == 1 && lane == 0) {
+        } else if (warp == 1 && lane == 0 && leader) {
             uint32_t it = 0, ch = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < n_units && ok && !*abort; u += gridDim.x) {
+            for (int u = pair; u < n_units && ok && !*abort; u += n_pairs) {
                 const int t0 = (u / n_tiles) * kSpanTokens;
                 const int t1 = min(n_tokens, t0 + kSpanTokens);
                 for (int c0 = t0; c0 < t1 && ok; c0 += kChainTokens, ++ch) {
@@ -172,25 +270,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // 16 tokens = two 8-row swizzle groups = 2048 bytes
                             const uint64_t ad = sdesc_sw128(a0 + k * 2048, kBoxBytes, 1024);
                             const uint64_t bd = sdesc_sw128(b0 + k * 2048, kBoxBytes, 1024);
-                            umma_f16(dt, ad, bd, kIdesc, (kk | k) != 0);
+                            umma_f16_pair(dt, ad, bd, kIdesc, (kk | k) != 0);
                         }
-                        umma_commit(&S.empty[s]);
+                        umma_commit_pair(&S.empty[s]);
                     }
-                    if (ok) umma_commit(&S.tfull[b]);
+                    if (ok) umma_commit_pair(&S.tfull[b]);
                 }
             }
         }
         __syncwarp();
     } else {
-        regs_alloc<224>();
+        regs_alloc<216>();
         // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31, column half h
         const int q = warp & 3;
         const int h = (warp - 4) / 4;
-        const int row_in_tile = q * 32 + lane;
+        const int row_in_tile = static_cast<int>(rank) * kBM + q * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
         uint32_t ch = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        for (int u = pair; u < n_units && ok; u += n_pairs) {
             const int t0 = (u / n_tiles) * kSpanTokens;
             const int t1 = min(n_tokens, t0 + kSpanTokens);
             float acc[kBN / 2];
@@ -215,15 +313,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.tempty[b]);
+                if (lane == 0) mbar_arrive_cluster(cluster_addr(&S.tempty[b], 0));
             }
             if (!ok) break;
             int ti, tj;
-            tile_coords(u % n_tiles, n_ti, n_tj, ti, tj);
-            const int row = ti * kBM + row_in_tile;
+            tile_coords(u % n_tiles, n_t, ti, tj);
+            const int row = ti * kTile + row_in_tile;
 #pragma unroll
             for (int c = 0; c < kBN / 64; ++c) {
-                const int col0 = tj * kBN + h * (kBN / 2) + c * 32;
+                const int col0 = tj * kTile + h * (kBN / 2) + c * 32;
                 if (row < d && col0 < d && col0 + 31 >= row) {
                     float* dst = H + static_cast<int64_t>(row) * d + col0;
                     if (col0 + 32 <= d) {
@@ -244,9 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();   // no MMA, commit or remote arrive of the pair is still in flight
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, kTmemCols);
+        tmem_dealloc_pair(tbase, kTmemCols);
     }
 }
 
@@ -325,15 +424,32 @@ int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
     CUtensorMap map;
     int rc = make_x_tmap(&map, X, n_rows, d);
     if (rc) return rc;
-    const int n_ti = static_cast<int>((d + kBM - 1) / kBM);
-    const int n_tj = static_cast<int>((d + kBN - 1) / kBN);
-    int n_tiles = 0;
-    for (int i = 0; i < n_ti; ++i) n_tiles += n_tj - (i >> 1);
+    const int n_t = static_cast<int>((d + kTile - 1) / kTile);
+    const int n_tiles = n_t * (n_t + 1) / 2;
     const int n_split = static_cast<int>((n_rows + kSpanTokens - 1) / kSpanTokens);
     const int64_t units = static_cast<int64_t>(n_tiles) * n_split;
-    const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
-    hessian_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
-        map, H, static_cast<int>(d), static_cast<int>(n_rows), n_ti, n_tj, n_tiles, n_split,
+    // pairs that can be resident at once (a GPC with an odd number of free
+    // SMs holds one pair less than half its SMs)
+    static int resident_pairs[64] = {};
+    int max_pairs = sm_count() / 2;
+    if (dev < 64) {
+        if (!resident_pairs[dev]) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * max_pairs);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = kSmemBytes;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, hessian_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+                (void)cudaGetLastError();
+                n = max_pairs;
+            }
+            resident_pairs[dev] = n;
+        }
+        max_pairs = std::min(max_pairs, resident_pairs[dev]);
+    }
+    const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
+    hessian_tc_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(
+        map, H, static_cast<int>(d), static_cast<int>(n_rows), n_t, n_tiles, n_split,
         device_status_ptr());
     GPTQ_LAUNCH_CHECK();
     return GPTQ_OK;
