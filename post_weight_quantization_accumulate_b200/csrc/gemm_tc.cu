@@ -3,27 +3,32 @@
 // C = alpha * A * B + beta * C with float32 operands, computed as three
 // tcgen05 kind::tf32 products (3xTF32): the tensor core reads a float32
 // operand as tf32 by dropping its 13 low mantissa bits, so with hi = x as
-// loaded and lo = x - trunc_tf32(x) (exact, formed in shared memory)
+// stored and lo = x - trunc_tf32(x) (exact)
 //     A B ~= A_hi B_hi + A_hi B_lo + A_lo B_hi
 // keeps about 2^-21 relative error per product, close to float32 (measured
 // 1e-6 relative on K = 128 against float64).
 //
 // Used for the lazy-batch update of the column loop (W[:, j+B:] -= E U_blk),
 // the trailing update of the blocked Cholesky (A22 -= L21 L21^T) and the
-// recursive triangular inverse.
+// accumulation of the factor's inverse.
 //
-// Per CTA (384 threads, persistent over 128 x 128 output tiles x batch):
+// Two variants, persistent over output tiles x batch, 384 threads per CTA:
+//  * 128 x 128 tiles, low parts formed in shared memory (three 64 KB stages:
+//    A_hi, A_lo, B_hi, B_lo of 16 KB) -- for operands produced on the fly;
+//  * 128 x 256 tiles with the low parts supplied by the caller as two more
+//    matrices (two 96 KB stages) -- no conversion pass, and N = 256 MMAs read
+//    A once per 256 columns: a third less shared-memory traffic per flop.
+// Roles:
 //   warp 0       TMA producer: fp32 tiles of A (K-major) and B (MN- or K-major)
-//   warp 1       MMA issuer + TMEM owner (two 128-column fp32 accumulators)
-//   warps 4-7    converters: the low tf32 parts of each stage in shared memory
+//   warp 1       MMA issuer + TMEM owner (two fp32 accumulators of TN columns)
+//   warps 4-7    converters (first variant): the low tf32 parts of a stage
 //   warps 8-11   epilogue: TMEM -> registers -> global.  With beta = 1 each
 //                warp stages alpha * acc for its 32 rows x 32 columns in
 //                shared memory and a TMA reduce-add applies it to C in L2
 //                (one rounding of C + alpha * acc, the same as the fma
 //                below); with beta = 0 a TMA store writes it; other betas
 //                (or a C that breaks the TMA rules) read C with plain loads.
-// Three 64 KB stages (A_hi, A_lo, B_hi, B_lo of 16 KB each) plus 32 KB of
-// epilogue staging.  All waits are bounded (see mbar_wait_bounded).
+// Plus 32 KB of epilogue staging.  All waits are bounded (mbar_wait_bounded).
 #include "gemm.cuh"
 
 #include <cstring>
@@ -32,33 +37,45 @@
 namespace gptq {
 namespace {
 
-constexpr int TBM = 128, TBN = 128, TBK = 32;   // 32 fp32 = 128 bytes = one swizzle row
-constexpr int TSTAGES = 3;
-constexpr int TILE_BYTES = TBM * TBK * 4;        // 16 KB (A tile; also B tile: 128 x 32)
-constexpr int STAGE_BYTES = 4 * TILE_BYTES;      // A_hi, A_lo, B_hi, B_lo
+constexpr int TBM = 128, TBK = 32;              // 32 fp32 = 128 bytes = one swizzle row
 constexpr int TTHREADS = 384;
-constexpr int TMEM_COLS = 2 * TBN;
-
+constexpr int A_BYTES = TBM * TBK * 4;           // 16 KB
 constexpr int CBUF_BYTES = 32 * 32 * 4;          // one warp's 32 x 32 chunk of C
 
+template <int TN, bool PRELO>
+struct GemmCfg {
+    static constexpr int B_BYTES = TN * TBK * 4;
+    static constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // hi and lo of A and B
+    static constexpr int STAGES = TN == 256 ? 2 : 3;
+    static constexpr int TMEM_COLS = 2 * TN;
+    static constexpr uint32_t TX_BYTES = PRELO ? 2 * (A_BYTES + B_BYTES) : A_BYTES + B_BYTES;
+};
+
+template <int TN, bool PRELO>
 struct alignas(1024) GemmSmem {
-    uint8_t stage[TSTAGES][STAGE_BYTES];
-    uint8_t cbuf[4][2][CBUF_BYTES];                  // per epilogue warp, double-buffered
-    uint64_t full[TSTAGES];    // TMA landed
-    uint64_t conv[TSTAGES];    // hi/lo split done
-    uint64_t empty[TSTAGES];   // MMAs done reading
+    using C = GemmCfg<TN, PRELO>;
+    uint8_t stage[C::STAGES][C::STAGE_BYTES];      // A_hi | A_lo | B_hi | B_lo
+    uint8_t cbuf[4][2][CBUF_BYTES];                // per epilogue warp, double-buffered
+    uint64_t full[C::STAGES];    // TMA landed
+    uint64_t conv[C::STAGES];    // hi/lo split done (converter variant)
+    uint64_t empty[C::STAGES];   // MMAs done reading
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint32_t tmem_base;
     int abort;
 };
-constexpr size_t GEMM_SMEM = sizeof(GemmSmem) + 1024;
-static_assert(GEMM_SMEM <= 227 * 1024, "one CTA per SM: at most 227 KB of shared memory");
+template <int TN, bool PRELO>
+constexpr size_t gemm_smem_bytes()
+{
+    return sizeof(GemmSmem<TN, PRELO>) + 1024;
+}
+static_assert(gemm_smem_bytes<128, false>() <= 227 * 1024, "one CTA per SM");
+static_assert(gemm_smem_bytes<256, true>() <= 227 * 1024, "one CTA per SM");
 
 enum CMode : int { kCPlain = 0, kCStore = 1, kCReduce = 2 };
 
 struct GemmArgs {
-    int M, N, K, batch, flags, trans_b, c_mode;
+    int M, N, K, batch, flags, trans_b, c_mode, tn;
     float alpha, beta;
     float* C;
     int64_t ldc, sC;
@@ -128,7 +145,7 @@ __device__ __forceinline__ bool unit_info(const GemmArgs& g, int u, int& b, int&
     const int t = u % per;
     mt = t / g.n_nt;
     nt = t % g.n_nt;
-    const int m0 = mt * TBM, n0 = nt * TBN;
+    const int m0 = mt * TBM, n0 = nt * g.tn;
     if ((g.flags & kGemmLowerC) && n0 > m0 + TBM - 1) return false;
     k0 = 0;
     k1 = g.K;
@@ -137,18 +154,23 @@ __device__ __forceinline__ bool unit_info(const GemmArgs& g, int u, int& b, int&
     return true;
 }
 
+template <int TN, bool PRELO>
 __global__ void __launch_bounds__(TTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   const __grid_constant__ CUtensorMap mapAlo, const __grid_constant__ CUtensorMap mapBlo,
                    const __grid_constant__ CUtensorMap mapC, const GemmArgs g)
 {
+    using Cfg = GemmCfg<TN, PRELO>;
+    constexpr int STAGES = Cfg::STAGES;
+    constexpr int B_BYTES = Cfg::B_BYTES;
     extern __shared__ uint8_t smem_raw[];
-    GemmSmem& S = *reinterpret_cast<GemmSmem*>(
+    GemmSmem<TN, PRELO>& S = *reinterpret_cast<GemmSmem<TN, PRELO>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < TSTAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&S.full[s], 1);
             mbar_init(&S.conv[s], 4);
             mbar_init(&S.empty[s], 1);
@@ -161,10 +183,14 @@ __global__ void __launch_bounds__(TTHREADS, 1)
         fence_mbar_init();
         prefetch_tmap(&mapA);
         prefetch_tmap(&mapB);
+        if (PRELO) {
+            prefetch_tmap(&mapAlo);
+            prefetch_tmap(&mapBlo);
+        }
         if (g.c_mode != kCPlain) prefetch_tmap(&mapC);
     }
     if (warp == 1) {
-        tmem_alloc(&S.tmem_base, TMEM_COLS);
+        tmem_alloc(&S.tmem_base, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -183,19 +209,25 @@ __global__ void __launch_bounds__(TTHREADS, 1)
                 int b, mt, nt, k0, k1;
                 if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
                 for (int k = k0; k < k1; k += TBK, ++it) {
-                    const int s = it % TSTAGES;
-                    const uint32_t ph = (it / TSTAGES) & 1;
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S.full[s], 2 * TILE_BYTES);
+                    mbar_arrive_expect_tx(&S.full[s], Cfg::TX_BYTES);
                     uint8_t* st = S.stage[s];
+                    uint8_t* bh = st + 2 * A_BYTES;
                     tma_load_3d(st, &mapA, &S.full[s], k, mt * TBM, b);
-                    uint8_t* bh = st + 2 * TILE_BYTES;
+                    if (PRELO) tma_load_3d(st + A_BYTES, &mapAlo, &S.full[s], k, mt * TBM, b);
                     if (g.trans_b) {
-                        tma_load_3d(bh, &mapB, &S.full[s], k, nt * TBN, b);
+                        tma_load_3d(bh, &mapB, &S.full[s], k, nt * TN, b);
+                        if (PRELO) tma_load_3d(bh + B_BYTES, &mapBlo, &S.full[s], k, nt * TN, b);
                     } else {
 #pragma unroll
-                        for (int q = 0; q < TBN / 32; ++q)   // 32-column x 32-row boxes
-                            tma_load_3d(bh + q * (TBK * 32 * 4), &mapB, &S.full[s], nt * TBN + q * 32, k, b);
+                        for (int q = 0; q < TN / 32; ++q) {   // 32-column x 32-row boxes
+                            tma_load_3d(bh + q * (TBK * 32 * 4), &mapB, &S.full[s], nt * TN + q * 32, k, b);
+                            if (PRELO)
+                                tma_load_3d(bh + B_BYTES + q * (TBK * 32 * 4), &mapBlo, &S.full[s],
+                                            nt * TN + q * 32, k, b);
+                        }
                     }
                 }
             }
@@ -203,7 +235,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, g.trans_b ? 0u : 1u, TBM, TBN);
+            const uint32_t idesc = idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, g.trans_b ? 0u : 1u, TBM, TN);
             uint32_t it = 0, uc = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -214,17 +246,20 @@ __global__ void __launch_bounds__(TTHREADS, 1)
                 ++uc;
                 if (!mbar_wait_bounded(&S.tempty[acc], aph ^ 1, abort, status)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t dt = tbase + acc * TBN;
+                const uint32_t dt = tbase + acc * TN;
                 bool first = true;
                 for (int k = k0; k < k1; k += TBK, ++it) {
-                    const int s = it % TSTAGES;
-                    const uint32_t ph = (it / TSTAGES) & 1;
-                    if (!mbar_wait_bounded(&S.conv[s], ph, abort, status)) { ok = false; break; }
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait_bounded(PRELO ? &S.full[s] : &S.conv[s], ph, abort, status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t ahi = smem_u32(S.stage[s]);
-                    const uint32_t alo = ahi + TILE_BYTES;
-                    const uint32_t bhi = ahi + 2 * TILE_BYTES;
-                    const uint32_t blo = ahi + 3 * TILE_BYTES;
+                    const uint32_t alo = ahi + A_BYTES;
+                    const uint32_t bhi = ahi + 2 * A_BYTES;
+                    const uint32_t blo = bhi + B_BYTES;
 #pragma unroll
                     for (int k8 = 0; k8 < TBK / 8; ++k8) {
                         // A: K-major, 8 fp32 = 32 bytes further along the swizzled row
@@ -253,7 +288,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
             }
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
+    } else if (!PRELO && warp >= 4 && warp < 8) {
         // converters: lo = x - trunc_tf32(x); hi is the loaded tile itself
         const int ct = threadIdx.x - 128;
         uint32_t it = 0;
@@ -262,18 +297,22 @@ __global__ void __launch_bounds__(TTHREADS, 1)
             int b, mt, nt, k0, k1;
             if (!unit_info(g, u, b, mt, nt, k0, k1)) continue;
             for (int k = k0; k < k1; k += TBK, ++it) {
-                const int s = it % TSTAGES;
-                const uint32_t ph = (it / TSTAGES) & 1;
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
                 const bool got = mbar_wait_bounded(&S.full[s], ph, abort, status);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 float4* ah = reinterpret_cast<float4*>(S.stage[s]);
-                float4* al = reinterpret_cast<float4*>(S.stage[s] + TILE_BYTES);
-                float4* bh = reinterpret_cast<float4*>(S.stage[s] + 2 * TILE_BYTES);
-                float4* bl = reinterpret_cast<float4*>(S.stage[s] + 3 * TILE_BYTES);
+                float4* al = reinterpret_cast<float4*>(S.stage[s] + A_BYTES);
+                float4* bh = reinterpret_cast<float4*>(S.stage[s] + 2 * A_BYTES);
+                float4* bl = reinterpret_cast<float4*>(S.stage[s] + 2 * A_BYTES + B_BYTES);
 #pragma unroll 4
-                for (int i = ct; i < TILE_BYTES / 16; i += 128) {
-                    const float4 xa = ah[i], xb = bh[i];
+                for (int i = ct; i < A_BYTES / 16; i += 128) {
+                    const float4 xa = ah[i];
                     al[i] = make_float4(tf32_low(xa.x), tf32_low(xa.y), tf32_low(xa.z), tf32_low(xa.w));
+                }
+#pragma unroll 4
+                for (int i = ct; i < B_BYTES / 16; i += 128) {
+                    const float4 xb = bh[i];
                     bl[i] = make_float4(tf32_low(xb.x), tf32_low(xb.y), tf32_low(xb.z), tf32_low(xb.w));
                 }
                 fence_proxy_async_smem();
@@ -302,10 +341,10 @@ __global__ void __launch_bounds__(TTHREADS, 1)
             const bool have = k1 > k0;
             const int row0 = mt * TBM + q * 32;
 #pragma unroll 1
-            for (int c = 0; c < TBN / 32; ++c) {
-                const int col0 = nt * TBN + c * 32;
+            for (int c = 0; c < TN / 32; ++c) {
+                const int col0 = nt * TN + c * 32;
                 float v[32];
-                tmem_ld_32x32b_x32(tbase + lane_addr + acc * TBN + c * 32, v);
+                tmem_ld_32x32b_x32(tbase + lane_addr + acc * TN + c * 32, v);
                 tmem_ld_wait();
                 // nothing of this chunk inside C (or, lower C, all above the diagonal)
                 if (row0 >= g.M || col0 >= g.N || (lower && col0 > row0 + 31)) continue;
@@ -361,13 +400,13 @@ __global__ void __launch_bounds__(TTHREADS, 1)
             // chunk c takes the vector path when it lies inside C, above no
             // skipped (upper) element and 16-byte aligned
             auto vec_ok = [&](int c) {
-                const int col0 = nt * TBN + c * 32;
+                const int col0 = nt * TN + c * 32;
                 return row < g.M && col0 + 32 <= g.N && !(lower && col0 + 31 > row) &&
                        (reinterpret_cast<uintptr_t>(crow + col0) & 15) == 0;
             };
             float4 cn[8];
             if (read_c && vec_ok(0)) {
-                const float4* p = reinterpret_cast<const float4*>(crow + nt * TBN);
+                const float4* p = reinterpret_cast<const float4*>(crow + nt * TN);
 #pragma unroll
                 for (int m = 0; m < 8; ++m) cn[m] = p[m];
             }
@@ -377,20 +416,20 @@ __global__ void __launch_bounds__(TTHREADS, 1)
             tc_fence_after();
             const bool have = k1 > k0;   // an empty K range leaves the accumulator unwritten
 #pragma unroll 1
-            for (int c = 0; c < TBN / 32; ++c) {
+            for (int c = 0; c < TN / 32; ++c) {
                 float4 cc[8];
 #pragma unroll
                 for (int m = 0; m < 8; ++m) cc[m] = cn[m];
-                if (read_c && c + 1 < TBN / 32 && vec_ok(c + 1)) {
-                    const float4* p = reinterpret_cast<const float4*>(crow + nt * TBN + (c + 1) * 32);
+                if (read_c && c + 1 < TN / 32 && vec_ok(c + 1)) {
+                    const float4* p = reinterpret_cast<const float4*>(crow + nt * TN + (c + 1) * 32);
 #pragma unroll
                     for (int m = 0; m < 8; ++m) cn[m] = p[m];
                 }
                 float v[32];
                 __syncwarp();   // the loads above may diverge; tcgen05.ld is warp-aligned
-                tmem_ld_32x32b_x32(tbase + lane_addr + acc * TBN + c * 32, v);
+                tmem_ld_32x32b_x32(tbase + lane_addr + acc * TN + c * 32, v);
                 tmem_ld_wait();
-                const int col0 = nt * TBN + c * 32;
+                const int col0 = nt * TN + c * 32;
                 if (row >= g.M || col0 >= g.N) continue;
                 if (vec_ok(c)) {
                     float4* p = reinterpret_cast<float4*>(crow + col0);
@@ -426,7 +465,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, TMEM_COLS);
+        tmem_dealloc(tbase, Cfg::TMEM_COLS);
     }
 }
 
@@ -481,38 +520,57 @@ bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, 
     return true;
 }
 
-int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
-                   int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
-                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream, int max_ctas)
+template <int TN, bool PRELO>
+static int set_smem_attr()
 {
-    if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
     static bool attr_set[64] = {};
     int dev = 0;
     GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
     if (dev < 64 && !attr_set[dev]) {
-        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(GEMM_SMEM)));
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gemm_tc_kernel<TN, PRELO>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(gemm_smem_bytes<TN, PRELO>())));
         attr_set[dev] = true;
     }
+    return GPTQ_OK;
+}
+
+int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
+                   int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
+                   int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream, int max_ctas,
+                   const float* A_lo, const float* B_lo)
+{
+    if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
+    const bool prelo = A_lo && B_lo;
+    const int tn = prelo ? 256 : 128;
+    int rc = prelo ? set_smem_attr<256, true>() : set_smem_attr<128, false>();
+    if (rc) return rc;
     const int Kp = K > 0 ? K : 1;
-    CUtensorMap mA, mB, mC;
+    CUtensorMap mA, mB, mAlo, mBlo, mC;
+    memset(&mAlo, 0, sizeof mAlo);
+    memset(&mBlo, 0, sizeof mBlo);
     int c_mode = kCPlain;
     const bool c_tma = (reinterpret_cast<uintptr_t>(C) & 15) == 0 && (ldc & 3) == 0 &&
                        (batch == 1 || (sC & 3) == 0);
     if (c_tma && (beta == 1.f || beta == 0.f)) {
-        int rc = make_map_f32(&mC, C, N, M, ldc, batch, sC, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+        rc = make_map_f32(&mC, C, N, M, ldc, batch, sC, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
         c_mode = beta == 1.f ? kCReduce : kCStore;
     } else {
         memset(&mC, 0, sizeof mC);
     }
-    int rc = make_map_f32(&mA, A, Kp, M, lda, batch, sA, TBK, TBM, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc) return rc;
-    if (trans_b)
-        rc = make_map_f32(&mB, B, Kp, N, ldb, batch, sB, TBK, TBN, CU_TENSOR_MAP_SWIZZLE_128B);
-    else
-        rc = make_map_f32(&mB, B, N, Kp, ldb, batch, sB, 32, TBK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
-    if (rc) return rc;
+    // A: [M][K] K-major boxes of 32 x 128; B: [N][K] boxes 32 x tn (trans_b) or
+    // [K][N] boxes of 32 columns x 32 rows
+    auto map_a = [&](CUtensorMap* m, const float* p) {
+        return make_map_f32(m, p, Kp, M, lda, batch, sA, TBK, TBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    };
+    auto map_b = [&](CUtensorMap* m, const float* p) {
+        return trans_b ? make_map_f32(m, p, Kp, N, ldb, batch, sB, TBK, tn, CU_TENSOR_MAP_SWIZZLE_128B)
+                       : make_map_f32(m, p, N, Kp, ldb, batch, sB, 32, TBK,
+                                      CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+    };
+    if ((rc = map_a(&mA, A)) || (rc = map_b(&mB, B))) return rc;
+    if (prelo && ((rc = map_a(&mAlo, A_lo)) || (rc = map_b(&mBlo, B_lo)))) return rc;
     GemmArgs g;
     g.M = M;
     g.N = N;
@@ -521,19 +579,25 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     g.flags = flags;
     g.trans_b = trans_b ? 1 : 0;
     g.c_mode = c_mode;
+    g.tn = tn;
     g.alpha = alpha;
     g.beta = beta;
     g.C = C;
     g.ldc = ldc;
     g.sC = sC;
     g.n_mt = (M + TBM - 1) / TBM;
-    g.n_nt = (N + TBN - 1) / TBN;
+    g.n_nt = (N + tn - 1) / tn;
     g.status = device_status_ptr();
     const int64_t units = static_cast<int64_t>(g.n_mt) * g.n_nt * batch;
     int cap = sm_count();
     if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;
     const int grid = static_cast<int>(units < cap ? units : cap);
-    gemm_tc_kernel<<<grid, TTHREADS, GEMM_SMEM, stream>>>(mA, mB, mC, g);
+    if (prelo)
+        gemm_tc_kernel<256, true><<<grid, TTHREADS, gemm_smem_bytes<256, true>(), stream>>>(
+            mA, mB, mAlo, mBlo, mC, g);
+    else
+        gemm_tc_kernel<128, false><<<grid, TTHREADS, gemm_smem_bytes<128, false>(), stream>>>(
+            mA, mB, mAlo, mBlo, mC, g);
     GPTQ_LAUNCH_CHECK();
     return GPTQ_OK;
 }

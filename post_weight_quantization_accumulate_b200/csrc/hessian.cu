@@ -23,7 +23,8 @@
 //    swizzle, the canonical MN-major SW128 layout tcgen05.mma reads.  Each CTA
 //    loads its own boxes (no multicast); the loads of both CTAs complete on
 //    the first CTA's barrier, whose thread issues the MMAs.
-//  * Work units = (tile, token span of kSpanTokens).  A persistent grid of
+//  * Work units = (tile, token span of 4096 .. 32768 tokens, the longest that
+//    still gives each pair about eight units).  A persistent grid of
 //    one pair per two SMs walks the units span-major, so concurrently
 //    running units read the same token rows of X (L2 reuse).
 //  * Accumulation precision: the tensor core adds each MMA's result into the
@@ -66,7 +67,8 @@ constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr int kTmemCols = 512;    // two 256-column fp32 chain buffers
 constexpr int kChainTokens = 512; // tokens per TMEM accumulation chain
-constexpr int kSpanTokens = 16384;  // tokens per work unit (one flush into H)
+constexpr int kSpanMax = 32768;   // tokens per work unit (one flush into H), at most
+constexpr int kSpanMin = 4096;
 constexpr uint32_t kIdesc = idesc_f32acc(1 /*bf16*/, 1, 1, 2 * kBM, kBN);
 
 struct alignas(1024) HessSmem {
@@ -180,7 +182,7 @@ __device__ __forceinline__ void tile_coords(int tile, int n_t, int& ti, int& tj)
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int d,
-                      int n_tokens, int n_t, int n_tiles, int n_split, int* status)
+                      int n_tokens, int n_t, int n_tiles, int n_split, int span, int* status)
 {
     extern __shared__ uint8_t smem_raw[];
     HessSmem& S = *reinterpret_cast<HessSmem*>(
@@ -223,8 +225,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int u = pair; u < n_units && !*abort; u += n_pairs) {
                 int ti, tj;
                 tile_coords(u % n_tiles, n_t, ti, tj);
-                const int t0 = (u / n_tiles) * kSpanTokens;
-                const int t1 = min(n_tokens, t0 + kSpanTokens);
+                const int t0 = (u / n_tiles) * span;
+                const int t1 = min(n_tokens, t0 + span);
                 const int col_a = ti * kTile + static_cast<int>(rank) * kBM;
                 const int col_b = tj * kTile + static_cast<int>(rank) * (kBN / 2);
                 bool ok = true;
@@ -249,8 +251,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t it = 0, ch = 0;
             bool ok = true;
             for (int u = pair; u < n_units && ok && !*abort; u += n_pairs) {
-                const int t0 = (u / n_tiles) * kSpanTokens;
-                const int t1 = min(n_tokens, t0 + kSpanTokens);
+                const int t0 = (u / n_tiles) * span;
+                const int t1 = min(n_tokens, t0 + span);
                 for (int c0 = t0; c0 < t1 && ok; c0 += kChainTokens, ++ch) {
                     const int b = ch & 1;
                     const uint32_t cph = (ch >> 1) & 1;
@@ -289,8 +291,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t ch = 0;
         bool ok = true;
         for (int u = pair; u < n_units && ok; u += n_pairs) {
-            const int t0 = (u / n_tiles) * kSpanTokens;
-            const int t1 = min(n_tokens, t0 + kSpanTokens);
+            const int t0 = (u / n_tiles) * span;
+            const int t1 = min(n_tokens, t0 + span);
             float acc[kBN / 2];
 #pragma unroll
             for (int i = 0; i < kBN / 2; ++i) acc[i] = 0.f;
@@ -426,7 +428,12 @@ int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
     if (rc) return rc;
     const int n_t = static_cast<int>((d + kTile - 1) / kTile);
     const int n_tiles = n_t * (n_t + 1) / 2;
-    const int n_split = static_cast<int>((n_rows + kSpanTokens - 1) / kSpanTokens);
+    // the longest token span (fewest flushes of partial sums into H) that
+    // still gives every pair about eight units
+    const int64_t want = 8 * static_cast<int64_t>(sm_count() / 2);
+    int span = kSpanMax;
+    while (span > kSpanMin && n_tiles * ((n_rows + span - 1) / span) < want) span /= 2;
+    const int n_split = static_cast<int>((n_rows + span - 1) / span);
     const int64_t units = static_cast<int64_t>(n_tiles) * n_split;
     // pairs that can be resident at once (a GPC with an odd number of free
     // SMs holds one pair less than half its SMs)
@@ -449,7 +456,7 @@ int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
     }
     const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
     hessian_tc_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(
-        map, H, static_cast<int>(d), static_cast<int>(n_rows), n_t, n_tiles, n_split,
+        map, H, static_cast<int>(d), static_cast<int>(n_rows), n_t, n_tiles, n_split, span,
         device_status_ptr());
     GPTQ_LAUNCH_CHECK();
     return GPTQ_OK;

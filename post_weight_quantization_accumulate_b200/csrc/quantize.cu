@@ -55,6 +55,7 @@ struct QArgs {
     float* zeros;
     uint8_t* codes_p;     // [d_out][d_in], processing order
     float* E;             // [d_out][kOuterMax] errors of the current outer window
+    float* E_lo;          // their low parts e - trunc_tf32(e) (tensor-core operand)
     int e_off;            // column of this block inside the outer window
     float* err_sq;        // [d_out] or null
     int* status;
@@ -90,6 +91,27 @@ __global__ void u_layout_kernel(const float* __restrict__ U, int d_in, int block
             }
         }
         out[idx] = v;
+    }
+}
+
+// Low part of x below its tf32 truncation (exact in float32): the tensor core
+// reads an fp32 operand as tf32 by dropping the 13 low mantissa bits.
+__device__ __forceinline__ float tf32_low(float x)
+{
+    return x - __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+}
+
+// U_lo[i][j] = tf32_low(U[i][j]) on and above the diagonal (the part the
+// lazy-batch products read).
+__global__ void u_low_kernel(const float* __restrict__ U, int d, float* __restrict__ U_lo)
+{
+    const int64_t n4 = static_cast<int64_t>(d) * d / 4;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int row = static_cast<int>((4 * i) / d), col = static_cast<int>((4 * i) % d);
+        if (col + 3 < row) continue;
+        const float4 v = reinterpret_cast<const float4*>(U)[i];
+        reinterpret_cast<float4*>(U_lo)[i] = make_float4(tf32_low(v.x), tf32_low(v.y), tf32_low(v.z), tf32_low(v.w));
     }
 }
 
@@ -341,8 +363,9 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                     kw[h][0] = s[h] * (kq[h][0] - z[h]);
                     kw[h][1] = s[h] * (kq[h][1] - z[h]);
                 }
-                *reinterpret_cast<float2*>(a.E + static_cast<int64_t>(r[h]) * kOuterMax + a.e_off + col) =
-                    make_float2(ke[h][0], ke[h][1]);
+                const int64_t eo = static_cast<int64_t>(r[h]) * kOuterMax + a.e_off + col;
+                *reinterpret_cast<float2*>(a.E + eo) = make_float2(ke[h][0], ke[h][1]);
+                *reinterpret_cast<float2*>(a.E_lo + eo) = make_float2(tf32_low(ke[h][0]), tf32_low(ke[h][1]));
                 *reinterpret_cast<float2*>(a.Wp + rowoff[h] + j0 + col) = make_float2(kw[h][0], kw[h][1]);
                 const uint32_t q2 = static_cast<uint32_t>(kq[h][0]) | (static_cast<uint32_t>(kq[h][1]) << 8);
                 *reinterpret_cast<uint16_t*>(a.codes_p + rowoff[h] + j0 + col) = static_cast<uint16_t>(q2);
@@ -520,12 +543,17 @@ inline size_t u_layout_bytes(int64_t d_in)
     return static_cast<size_t>(d_in / 8 + 16) * UCH_BYTES;
 }
 
+// Workspace of the column loop, in this order: working weights Wp (d_out x d_in
+// f32), codes (d_out x d_in u8), errors E and their low parts E_lo (d_out x
+// 1024 f32 each), the inverse permutation (d_in i32), the U block layout, and
+// U's low parts (d_in x d_in f32).
 size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
 {
     const size_t n = static_cast<size_t>(d_out) * static_cast<size_t>(d_in);
-    return 256 + up256(n * sizeof(float)) + up256(n) +
-           up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)) +
-           up256(static_cast<size_t>(d_in) * sizeof(int32_t)) + up256(u_layout_bytes(d_in));
+    const size_t e = up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float));
+    return 256 + up256(n * sizeof(float)) + up256(n) + 2 * e +
+           up256(static_cast<size_t>(d_in) * sizeof(int32_t)) + up256(u_layout_bytes(d_in)) +
+           up256(static_cast<size_t>(d_in) * static_cast<size_t>(d_in) * sizeof(float));
 }
 
 static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
@@ -538,11 +566,13 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* Wp = reinterpret_cast<float*>(ws + 256);
     uint8_t* codes_p = ws + 256 + up256(n * sizeof(float));
+    const size_t e_bytes = up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float));
     float* E = reinterpret_cast<float*>(ws + 256 + up256(n * sizeof(float)) + up256(n));
-    int32_t* inv = reinterpret_cast<int32_t*>(ws + 256 + up256(n * sizeof(float)) + up256(n) +
-                                              up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)));
+    float* E_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(E) + e_bytes);
+    int32_t* inv = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(E_lo) + e_bytes);
     float* Ul = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(inv) +
                                          up256(static_cast<size_t>(d_in) * sizeof(int32_t)));
+    float* U_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(Ul) + up256(u_layout_bytes(d_in)));
     const int nsm = sm_count();
     int* status = device_status_ptr();
     const int n_groups = gs > 0 ? d_in / gs : 1;
@@ -566,6 +596,8 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     const int nch_blk = (block + QSUB - 1) / QSUB;
     const int n_blocks = (d_in + block - 1) / block;
     u_layout_kernel<<<n_blocks * nch_blk, 256, 0, stream>>>(U, d_in, block, nch_blk, Ul);
+    GPTQ_LAUNCH_CHECK();
+    u_low_kernel<<<nsm * 8, 256, 0, stream>>>(U, d_in, U_lo);
     GPTQ_LAUNCH_CHECK();
 
     float* work = W;
@@ -602,7 +634,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         for (int j0 = J0; j0 < J1; j0 += block) {
             const int bw = (J1 - j0 < block) ? J1 - j0 : block;
             QArgs a{work, Ul, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
-                    codes_p, E, j0 - J0, err_sq, status};
+                    codes_p, E, E_lo, j0 - J0, err_sq, status};
             if (groups_in_step)
                 gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
             else
@@ -610,17 +642,18 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
             GPTQ_LAUNCH_CHECK();
             const int rest_in = J1 - j0 - bw;
             if (rest_in > 0) {
+                const int64_t uo = static_cast<int64_t>(j0) * d_in + j0 + bw;
                 int rc = launch_sgemm(false, d_out, rest_in, bw, -1.f, E + (j0 - J0), kOuterMax, 0,
-                                      U + static_cast<int64_t>(j0) * d_in + j0 + bw, d_in, 0, 1.f,
-                                      work + j0 + bw, d_in, 0, 1, 0, stream);
+                                      U + uo, d_in, 0, 1.f, work + j0 + bw, d_in, 0, 1, 0, stream, 0,
+                                      E_lo + (j0 - J0), U_lo + uo);
                 if (rc) return rc;
             }
         }
         const int rest = d_in - J1;
         if (rest > 0) {
-            int rc = launch_sgemm(false, d_out, rest, J1 - J0, -1.f, E, kOuterMax, 0,
-                                  U + static_cast<int64_t>(J0) * d_in + J1, d_in, 0, 1.f,
-                                  work + J1, d_in, 0, 1, 0, stream);
+            const int64_t uo = static_cast<int64_t>(J0) * d_in + J1;
+            int rc = launch_sgemm(false, d_out, rest, J1 - J0, -1.f, E, kOuterMax, 0, U + uo, d_in, 0,
+                                  1.f, work + J1, d_in, 0, 1, 0, stream, 0, E_lo, U_lo + uo);
             if (rc) return rc;
         }
     }
