@@ -19,7 +19,7 @@
 //    bandwidth at the full MMA rate.
 //  * Both operands are slices of the same X rows: A = X[t, rows], B = X[t,
 //    cols].  Their contraction index (tokens) is the outer dimension of X, so
-//    both are MN-major; TMA brings 64-token x 64-column boxes with 128-byte
+//    both are MN-major; TMA brings 128-token x 64-column boxes with 128-byte
 //    swizzle, the canonical MN-major SW128 layout tcgen05.mma reads.  Each CTA
 //    loads its own boxes (no multicast); the loads of both CTAs complete on
 //    the first CTA's barrier, whose thread issues the MMAs.
@@ -38,8 +38,10 @@
 //    (warpgroup 0 gives its registers up to 64); warps 4-11 = epilogue (raised
 //    to 216 registers); warps w and w+4 share TMEM lanes 32*(w%4)..+31 and
 //    split the 256 columns in halves, 128 fp32 registers of running sum each.
-//    128 x 64 + 256 x 216 = 63488 fits the launch budget 384 x 168.  A 6-stage
-//    shared-memory ring (32 KB per stage) and two TMEM chain buffers (2 x 256
+//    128 x 64 + 256 x 216 = 63488 fits the launch budget 384 x 168.  A 3-stage
+//    shared-memory ring (64 KB per stage: few, large TMA batches per barrier
+//    round trip measured faster than more, smaller stages) and two TMEM chain
+//    buffers (2 x 256
 //    columns) let the promotion of one chain overlap the MMAs of the next.
 //  * Every mbarrier wait is bounded; a time-out records GPTQ_ERR_TIMEOUT and
 //    ends the role; both CTAs meet at a cluster barrier before the pair frees
@@ -56,13 +58,13 @@ namespace {
 constexpr int kBM = 128;          // H rows per CTA (half of the pair's M = 256)
 constexpr int kBN = 256;          // H cols per tile (MMA N)
 constexpr int kTile = 256;        // tile edge
-constexpr int kBK = 64;           // tokens per pipeline stage
-constexpr int kStages = 6;
+constexpr int kBK = 128;          // tokens per pipeline stage
+constexpr int kStages = 3;
 constexpr int kBoxCols = 64;      // 64 bf16 = 128 bytes = one swizzle row
-constexpr int kBoxBytes = kBK * kBoxCols * 2;           // 8 KB
-constexpr int kABytes = kBoxBytes * (kBM / kBoxCols);   // 16 KB: 128 rows of A
-constexpr int kBBytes = kBoxBytes * (kBN / 2 / kBoxCols);  // 16 KB: this CTA's 128 columns of B
-constexpr int kStageBytes = kABytes + kBBytes;          // 32 KB
+constexpr int kBoxBytes = kBK * kBoxCols * 2;           // 16 KB
+constexpr int kABytes = kBoxBytes * (kBM / kBoxCols);   // 32 KB: 128 rows of A
+constexpr int kBBytes = kBoxBytes * (kBN / 2 / kBoxCols);  // 32 KB: this CTA's 128 columns of B
+constexpr int kStageBytes = kABytes + kBBytes;          // 64 KB
 constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr int kTmemCols = 512;    // two 256-column fp32 chain buffers
@@ -229,21 +231,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int t1 = min(n_tokens, t0 + span);
                 const int col_a = ti * kTile + static_cast<int>(rank) * kBM;
                 const int col_b = tj * kTile + static_cast<int>(rank) * (kBN / 2);
+                const bool diag = ti == tj;
                 bool ok = true;
                 for (int t = t0; t < t1 && ok; t += kBK, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status)) { ok = false; break; }
-                    if (leader) mbar_arrive_expect_tx(&S.full[s], 2 * kStageBytes);
+                    // a diagonal tile's B half is this CTA's A rows: loaded once
+                    if (leader) mbar_arrive_expect_tx(&S.full[s], 2 * (diag ? kABytes : kStageBytes));
                     const uint32_t fb = cluster_addr(&S.full[s], 0);
                     uint8_t* a = S.stage[s];
                     uint8_t* b = a + kABytes;
 #pragma unroll
                     for (int m = 0; m < kBM / kBoxCols; ++m)
                         tma_load_2d_pair(a + m * kBoxBytes, &tmap, fb, col_a + m * kBoxCols, t);
+                    if (!diag) {
 #pragma unroll
-                    for (int m = 0; m < kBN / 2 / kBoxCols; ++m)
-                        tma_load_2d_pair(b + m * kBoxBytes, &tmap, fb, col_b + m * kBoxCols, t);
+                        for (int m = 0; m < kBN / 2 / kBoxCols; ++m)
+                            tma_load_2d_pair(b + m * kBoxBytes, &tmap, fb, col_b + m * kBoxCols, t);
+                    }
                 }
                 if (!ok) break;
             }
@@ -253,6 +259,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int u = pair; u < n_units && ok && !*abort; u += n_pairs) {
                 const int t0 = (u / n_tiles) * span;
                 const int t1 = min(n_tokens, t0 + span);
+                int ti, tj;
+                tile_coords(u % n_tiles, n_t, ti, tj);
+                const uint32_t b_off = ti == tj ? 0u : static_cast<uint32_t>(kABytes);
                 for (int c0 = t0; c0 < t1 && ok; c0 += kChainTokens, ++ch) {
                     const int b = ch & 1;
                     const uint32_t cph = (ch >> 1) & 1;
@@ -266,7 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         if (!mbar_wait_bounded(&S.full[s], ph, abort, status)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t a0 = smem_u32(S.stage[s]);
-                        const uint32_t b0 = a0 + kABytes;
+                        const uint32_t b0 = a0 + b_off;
 #pragma unroll
                         for (int k = 0; k < kBK / 16; ++k) {
                             // 16 tokens = two 8-row swizzle groups = 2048 bytes
