@@ -69,10 +69,17 @@ uint64_t gptq_launch_count(void);
 int gptq_device_status(void);
 
 /* Bytes of workspace gptq_prepare (d_in) and gptq_quantize (d_out, d_in,
- * block_size, with or without an activation order) need; the maximum of the
- * two is safe for both.  The workspace must be 256-byte aligned.  Returns 0
- * for invalid sizes. */
+ * block_size, with or without an activation order) need for their fastest
+ * path; the maximum of the two is safe for both.  The workspace must be
+ * 256-byte aligned.  Returns 0 for invalid sizes. */
 size_t gptq_workspace_bytes(int64_t d_out, int64_t d_in, int block_size);
+
+/* The smallest workspace the two calls accept (same arguments and rules).
+ * gptq_quantize with less than gptq_workspace_bytes but at least this much
+ * forms the tf32 low parts of its lazy-batch operands inside the products
+ * instead of keeping them in the workspace (same results, somewhat slower).
+ * Returns 0 for invalid sizes. */
+size_t gptq_workspace_min_bytes(int64_t d_out, int64_t d_in, int block_size);
 
 /*
  * H += 2 * X^T X   ("Jak działa": H = 2 X X^T; "Złożoność obliczeniowa":
@@ -186,10 +193,12 @@ int gptq_quantize(float *W, const float *Hinv_chol, const int32_t *perm, int64_t
  * Arguments, outputs and results are those of gptq_quantize.  The scratch is
  * a fixed array inside the library (GPTQ_STATIC_SCRATCH_BYTES), so the call
  * allocates nothing.  Limits and rules:
- *   - A layer whose working set exceeds the array (about 5 bytes per weight
- *     plus 4 KiB per output row: 4096 x 4096 needs about 96 MiB and fits,
- *     4096 x 11008 does not) is refused with GPTQ_ERR_WORKSPACE before the
- *     device is touched.
+ *   - A layer whose working set exceeds the array (the minimum workspace of
+ *     gptq_quantize: about 5 bytes per weight plus 4 KiB per output row;
+ *     4096 x 4096 needs about 102 MiB and fits, 4096 x 11008 does not) is
+ *     refused with GPTQ_ERR_WORKSPACE before the device is touched.  When the
+ *     array also holds the optional low-part buffers (small layers) they are
+ *     used.
  *   - The first call on each device looks up the array's device address with
  *     that device current (a one-time set-up); make that first call before any
  *     stream capture begins.

@@ -31,6 +31,7 @@ SIGNATURES = [
     ("gptq_launch_count", ctypes.c_uint64, []),
     ("gptq_device_status", _I, []),
     ("gptq_workspace_bytes", _SZ, [_I64, _I64, _I]),
+    ("gptq_workspace_min_bytes", _SZ, [_I64, _I64, _I]),
     ("gptq_hessian_accumulate", _I, [_P, _P, _I64, _I64, _P]),
     ("gptq_hessian_accumulate_host", _I, [_P, _P, _I64, _I64, _P, _I64, _P]),
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
@@ -116,6 +117,10 @@ def gptq_device_status() -> int:
 
 def gptq_workspace_bytes(d_out: int, d_in: int, block_size: int = 128) -> int:
     return int(lib().gptq_workspace_bytes(d_out, d_in, block_size))
+
+
+def gptq_workspace_min_bytes(d_out: int, d_in: int, block_size: int = 128) -> int:
+    return int(lib().gptq_workspace_min_bytes(d_out, d_in, block_size))
 
 
 def workspace(d_out: int, d_in: int, block_size: int = 128, device=None) -> torch.Tensor:

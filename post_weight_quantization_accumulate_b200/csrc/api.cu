@@ -14,12 +14,13 @@ int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
 int launch_mirror(float* H, int64_t d, cudaStream_t s);
 size_t prepare_workspace_bytes(int64_t d);
 size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in);
+size_t quantize_workspace_min_bytes(int64_t d_out, int64_t d_in);
 int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* perm, float* U,
                 void* ws, cudaStream_t s, int* host_status, bool graphed);
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
                  int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
-                 uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, cudaStream_t s,
-                 bool graphed);
+                 uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, size_t ws_bytes,
+                 cudaStream_t s, bool graphed);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
 
@@ -151,12 +152,12 @@ int quantize_entry(float* W, const float* Hinv_chol, const int32_t* perm, int64_
     }
     if (packed_int4 && bits > 4) return GPTQ_ERR_INVALID_ARG;
     if (static_cast<int64_t>(d_out) * d_in >= (int64_t(1) << 40)) return GPTQ_ERR_INVALID_ARG;
-    if (!workspace || !aligned(workspace, 256) || ws_bytes < quantize_workspace_bytes(d_out, d_in))
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < quantize_workspace_min_bytes(d_out, d_in))
         return GPTQ_ERR_WORKSPACE;
     int rc = check_device();
     if (rc) return rc;
     return run_quantize(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
-                        scales, zeros, packed_int4, g_idx, err_sq, workspace,
+                        scales, zeros, packed_int4, g_idx, err_sq, workspace, ws_bytes,
                         static_cast<cudaStream_t>(stream), graphed);
 }
 
@@ -206,6 +207,16 @@ size_t gptq_workspace_bytes(int64_t d_out, int64_t d_in, int block_size)
         return 0;
     size_t a = prepare_workspace_bytes(d_in);
     size_t b = quantize_workspace_bytes(d_out, d_in);
+    return a > b ? a : b;
+}
+
+size_t gptq_workspace_min_bytes(int64_t d_out, int64_t d_in, int block_size)
+{
+    if (d_in <= 0 || d_in > kMaxDim || d_out < 0 || d_out > (int64_t(1) << 31) / 2 ||
+        block_size < 0)
+        return 0;
+    size_t a = prepare_workspace_bytes(d_in);
+    size_t b = quantize_workspace_min_bytes(d_out, d_in);
     return a > b ? a : b;
 }
 

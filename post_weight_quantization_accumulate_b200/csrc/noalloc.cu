@@ -13,7 +13,7 @@
 #include <mutex>
 
 namespace gptq {
-size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in);
+size_t quantize_workspace_min_bytes(int64_t d_out, int64_t d_in);
 }
 
 namespace {
@@ -65,7 +65,7 @@ extern "C" int gptq_quantize_static_scratch(float* W, const float* Hinv_chol,
     if (d_out <= 0 || d_in <= 0) return GPTQ_ERR_INVALID_ARG;
     // A layer whose working set does not fit the fixed array is refused
     // before anything touches the device.
-    if (gptq::quantize_workspace_bytes(d_out, d_in) > GPTQ_STATIC_SCRATCH_BYTES)
+    if (gptq::quantize_workspace_min_bytes(d_out, d_in) > GPTQ_STATIC_SCRATCH_BYTES)
         return GPTQ_ERR_WORKSPACE;
     void* scratch = nullptr;
     int rc = scratch_address(&scratch);

@@ -55,7 +55,7 @@ struct QArgs {
     float* zeros;
     uint8_t* codes_p;     // [d_out][d_in], processing order
     float* E;             // [d_out][kOuterMax] errors of the current outer window
-    float* E_lo;          // their low parts e - trunc_tf32(e) (tensor-core operand)
+    float* E_lo;          // their low parts e - trunc_tf32(e) (tensor-core operand) or null
     int e_off;            // column of this block inside the outer window
     float* err_sq;        // [d_out] or null
     int* status;
@@ -365,7 +365,8 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                 }
                 const int64_t eo = static_cast<int64_t>(r[h]) * kOuterMax + a.e_off + col;
                 *reinterpret_cast<float2*>(a.E + eo) = make_float2(ke[h][0], ke[h][1]);
-                *reinterpret_cast<float2*>(a.E_lo + eo) = make_float2(tf32_low(ke[h][0]), tf32_low(ke[h][1]));
+                if (a.E_lo)
+                    *reinterpret_cast<float2*>(a.E_lo + eo) = make_float2(tf32_low(ke[h][0]), tf32_low(ke[h][1]));
                 *reinterpret_cast<float2*>(a.Wp + rowoff[h] + j0 + col) = make_float2(kw[h][0], kw[h][1]);
                 const uint32_t q2 = static_cast<uint32_t>(kq[h][0]) | (static_cast<uint32_t>(kq[h][1]) << 8);
                 *reinterpret_cast<uint16_t*>(a.codes_p + rowoff[h] + j0 + col) = static_cast<uint16_t>(q2);
@@ -544,22 +545,29 @@ inline size_t u_layout_bytes(int64_t d_in)
 }
 
 // Workspace of the column loop, in this order: working weights Wp (d_out x d_in
-// f32), codes (d_out x d_in u8), errors E and their low parts E_lo (d_out x
-// 1024 f32 each), the inverse permutation (d_in i32), the U block layout, and
-// U's low parts (d_in x d_in f32).
-size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
+// f32), codes (d_out x d_in u8), errors E (d_out x 1024 f32), the inverse
+// permutation (d_in i32), the U block layout -- the minimum -- then the tf32
+// low parts of E (d_out x 1024 f32) and of U (d_in x d_in f32).  With the low
+// parts present the lazy-batch products skip their conversion pass.
+size_t quantize_workspace_min_bytes(int64_t d_out, int64_t d_in)
 {
     const size_t n = static_cast<size_t>(d_out) * static_cast<size_t>(d_in);
-    const size_t e = up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float));
-    return 256 + up256(n * sizeof(float)) + up256(n) + 2 * e +
-           up256(static_cast<size_t>(d_in) * sizeof(int32_t)) + up256(u_layout_bytes(d_in)) +
+    return 256 + up256(n * sizeof(float)) + up256(n) +
+           up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)) +
+           up256(static_cast<size_t>(d_in) * sizeof(int32_t)) + up256(u_layout_bytes(d_in));
+}
+
+size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
+{
+    return quantize_workspace_min_bytes(d_out, d_in) +
+           up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float)) +
            up256(static_cast<size_t>(d_in) * static_cast<size_t>(d_in) * sizeof(float));
 }
 
 static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
                             int64_t d_in64, int bits, int gs, int block, uint8_t* codes,
                             float* scales, float* zeros, uint8_t* packed, int32_t* g_idx,
-                            float* err_sq, void* workspace, cudaStream_t stream)
+                            float* err_sq, void* workspace, bool with_low_parts, cudaStream_t stream)
 {
     const int d_out = static_cast<int>(d_out64), d_in = static_cast<int>(d_in64);
     const size_t n = static_cast<size_t>(d_out) * d_in;
@@ -568,11 +576,15 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     uint8_t* codes_p = ws + 256 + up256(n * sizeof(float));
     const size_t e_bytes = up256(static_cast<size_t>(d_out) * kOuterMax * sizeof(float));
     float* E = reinterpret_cast<float*>(ws + 256 + up256(n * sizeof(float)) + up256(n));
-    float* E_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(E) + e_bytes);
-    int32_t* inv = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(E_lo) + e_bytes);
+    int32_t* inv = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(E) + e_bytes);
     float* Ul = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(inv) +
                                          up256(static_cast<size_t>(d_in) * sizeof(int32_t)));
-    float* U_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(Ul) + up256(u_layout_bytes(d_in)));
+    float* E_lo = nullptr;
+    float* U_lo = nullptr;
+    if (with_low_parts) {
+        E_lo = reinterpret_cast<float*>(ws + quantize_workspace_min_bytes(d_out, d_in));
+        U_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(E_lo) + e_bytes);
+    }
     const int nsm = sm_count();
     int* status = device_status_ptr();
     const int n_groups = gs > 0 ? d_in / gs : 1;
@@ -597,8 +609,10 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     const int n_blocks = (d_in + block - 1) / block;
     u_layout_kernel<<<n_blocks * nch_blk, 256, 0, stream>>>(U, d_in, block, nch_blk, Ul);
     GPTQ_LAUNCH_CHECK();
-    u_low_kernel<<<nsm * 8, 256, 0, stream>>>(U, d_in, U_lo);
-    GPTQ_LAUNCH_CHECK();
+    if (with_low_parts) {
+        u_low_kernel<<<nsm * 8, 256, 0, stream>>>(U, d_in, U_lo);
+        GPTQ_LAUNCH_CHECK();
+    }
 
     float* work = W;
     if (perm) {
@@ -645,7 +659,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                 const int64_t uo = static_cast<int64_t>(j0) * d_in + j0 + bw;
                 int rc = launch_sgemm(false, d_out, rest_in, bw, -1.f, E + (j0 - J0), kOuterMax, 0,
                                       U + uo, d_in, 0, 1.f, work + j0 + bw, d_in, 0, 1, 0, stream, 0,
-                                      E_lo + (j0 - J0), U_lo + uo);
+                                      E_lo ? E_lo + (j0 - J0) : nullptr, U_lo ? U_lo + uo : nullptr);
                 if (rc) return rc;
             }
         }
@@ -653,7 +667,8 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         if (rest > 0) {
             const int64_t uo = static_cast<int64_t>(J0) * d_in + J1;
             int rc = launch_sgemm(false, d_out, rest, J1 - J0, -1.f, E, kOuterMax, 0, U + uo, d_in, 0,
-                                  1.f, work + J1, d_in, 0, 1, 0, stream, 0, E_lo, U_lo + uo);
+                                  1.f, work + J1, d_in, 0, 1, 0, stream, 0, E_lo,
+                                  U_lo ? U_lo + uo : nullptr);
             if (rc) return rc;
         }
     }
@@ -671,11 +686,13 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
 
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in, int bits,
                  int gs, int block, uint8_t* codes, float* scales, float* zeros, uint8_t* packed,
-                 int32_t* g_idx, float* err_sq, void* workspace, cudaStream_t stream, bool graphed)
+                 int32_t* g_idx, float* err_sq, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                 bool graphed)
 {
+    const bool low = ws_bytes >= quantize_workspace_bytes(d_out, d_in);
     auto enq = [&](cudaStream_t s, int*) {
         return enqueue_quantize(W, U, perm, d_out, d_in, bits, gs, block, codes, scales, zeros,
-                                packed, g_idx, err_sq, workspace, s);
+                                packed, g_idx, err_sq, workspace, low, s);
     };
     if (!graphed) return enq(stream, nullptr);
     auto P = [](const void* p) { return static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p)); };
@@ -683,7 +700,8 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                                        static_cast<uint64_t>(d_in), static_cast<uint64_t>(bits),
                                        static_cast<uint64_t>(static_cast<int64_t>(gs)),
                                        static_cast<uint64_t>(block), P(codes), P(scales), P(zeros),
-                                       P(packed), P(g_idx), P(err_sq), P(workspace)};
+                                       P(packed), P(g_idx), P(err_sq), P(workspace),
+                                       static_cast<uint64_t>(low)};
     return run_graphed(key, false, enq, stream, nullptr);
 }
 

@@ -1,7 +1,7 @@
 """Comparison helpers shared by the GPU parity tests (no arithmetic of the
 method lives here: only element-wise comparisons and the tolerances).
 
-Tolerances (spec bar for this path):
+Tolerances of this path (the stated parity bar):
   H          relative Frobenius error <= 1e-5 (fp32 accumulation of exact bf16 products)
   codes      identical on >= 99.9% of entries (2-4 bits; the stated widths);
              every mismatch exactly one level.  For wider codes the bar scales

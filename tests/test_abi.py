@@ -48,6 +48,9 @@ def test_workspace_bytes(lib):
     w = B.gptq_workspace_bytes(4096, 4096, 128)
     assert w >= 2 * 4096 * 4096 * 4          # factorisation: working copy and inverse
     assert w >= 4096 * 4096 * 5              # working weights + codes
+    m = B.gptq_workspace_min_bytes(4096, 4096, 128)
+    assert 4096 * 4096 * 5 <= m < w          # the low parts of the operands are optional
+    assert B.gptq_workspace_min_bytes(4096, 0, 128) == 0
     assert B.gptq_workspace_bytes(4096, 0, 128) == 0
     assert B.gptq_workspace_bytes(4096, -5, 128) == 0
 

@@ -274,3 +274,32 @@ def test_division_free_quotient_matches_ieee_division():
     division instruction; on the device it must agree with IEEE division on
     random, all-ones-significand and near-tie operands."""
     assert B.gptq_selftest_quotient(3 << 26, seed=7) == 0
+
+
+def test_minimum_workspace_gives_the_same_results():
+    """gptq_quantize with the smallest accepted workspace forms the tf32 low
+    parts inside the lazy-batch products instead of keeping them in the
+    workspace; the per-element accumulation order is the same, so the results
+    match the full-workspace call."""
+    d_out, d_in, bits, gs = 256, 1024, 4, 128
+    W, xb = synth.random_layer(21, d_out, d_in, 2 * d_in, correlated=True)
+    H = torch.zeros(d_in, d_in, dtype=torch.float32, device=DEV)
+    B.gptq_hessian_accumulate(H, torch.from_numpy(xb.view(np.int16)).to(DEV).view(torch.bfloat16))
+    U = torch.empty(d_in, d_in, dtype=torch.float32, device=DEV)
+    perm = torch.empty(d_in, dtype=torch.int32, device=DEV)
+    B.gptq_prepare(H, 0.01, 1, perm, U, B.workspace(d_out, d_in, 128))
+    outs = []
+    for n in (B.gptq_workspace_bytes(d_out, d_in, 128), B.gptq_workspace_min_bytes(d_out, d_in, 128)):
+        ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+        Wt = torch.from_numpy(W.astype(np.float32)).to(DEV)
+        ng = d_in // gs
+        sc = torch.empty(d_out, ng, device=DEV)
+        zr = torch.empty(d_out, ng, device=DEV)
+        codes = torch.empty(d_out, d_in, dtype=torch.uint8, device=DEV)
+        B.gptq_quantize(Wt, U, perm, bits, gs, 128, sc, zr, ws, codes=codes)
+        torch.cuda.synchronize()
+        outs.append((Wt.cpu().numpy(), sc.cpu().numpy(), codes.cpu().numpy()))
+    assert B.gptq_device_status() == 0
+    np.testing.assert_array_equal(outs[0][2], outs[1][2])
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+    np.testing.assert_allclose(outs[0][0], outs[1][0], rtol=1e-6, atol=1e-8)
