@@ -153,7 +153,34 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
 // Inverse Z = L^{-1} by recursive doubling: the 16 diagonal 4 x 4 inverses,
 // then Z21 = -Z22 (L21 Z11) for block sizes 8, 16, 32, 64.
 typedef float Tile64[kNB + 1];
-constexpr size_t kPanelSmem = (4 * kNB * (kNB + 1) + 32 * 33) * sizeof(float) + 16;
+constexpr size_t kPanelSmem = (5 * kNB * (kNB + 1) + 32 * 33) * sizeof(float) + 16;
+
+// 4-byte asynchronous copy global -> shared; `valid` false writes a zero.
+__device__ __forceinline__ void cp_async4(void* dst, const float* src, bool valid)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 4 : 0)
+                 : "memory");
+}
+
+// 64 x 64 tile of A (rows r_begin.., columns c_begin..) into smem by
+// asynchronous copies (one commit group); rows >= nrows or columns >= ncols
+// read as 0.  Completes at cp.async.wait_group.
+__device__ __forceinline__ void load_tile_async(Tile64* dst, const float* A, int d, int r_begin, int nrows,
+                                                int c_begin, int ncols)
+{
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        const bool valid = i < nrows && j < ncols;
+        cp_async4(&dst[i][j], valid ? A + static_cast<int64_t>(r_begin + i) * d + c_begin + j : A, valid);
+    }
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // acc[i][j] (tile rows 4ty.., cols 4tx..) -= X[rows] . Y[cols] over 64 columns:
 // the rank-64 correction of the previous panel applied on the fly.
@@ -206,11 +233,28 @@ __global__ void __launch_bounds__(256)
     Tile64* Zs = As + kNB;
     Tile64* Pd = Zs + kNB;       // previous panel, rows of this diagonal block
     Tile64* Pr = Pd + kNB;       // previous panel, rows of this CTA's panel block
-    float* Ys = reinterpret_cast<float*>(Pr + kNB);
+    Tile64* Ts = Pr + kNB;       // this CTA's operand tile (panel rows, or a block of M^{-1})
+    float* Ys = reinterpret_cast<float*>(Ts + kNB);
     int& bad_any = *reinterpret_cast<int*>(Ys + 32 * 33);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
+    const int n_trsm = (d - k0 - kb + kNB - 1) / kNB;
+    const bool y_cta = static_cast<int>(blockIdx.x) > n_trsm;
+    const int pr0 = k0 + kb + (static_cast<int>(blockIdx.x) - 1) * kNB;   // TRSM CTAs
+    const int prn = min(kNB, d - pr0);
+    const int cb = (static_cast<int>(blockIdx.x) - 1 - n_trsm) * kNB;      // M^{-1} CTAs
+
+    // The operand tiles of the second phase do not depend on the diagonal
+    // block: they are fetched asynchronously while it is factored.
+    if (y_cta) {
+        load_tile_async(Ts, Minv, d, k0, kb, cb, kNB);   // Y~_k
+        load_tile_async(Pr, Minv, d, pk0, kNB, cb, kNB); // Y_{k-1}
+    } else if (blockIdx.x > 0) {
+        load_tile_async(Ts, A, d, pr0, prn, k0, kb);
+        if (pk0 >= 0) load_tile_async(Pr, A, d, pr0, prn, pk0, kNB);
+    }
+    cp_async_commit();
 
     // diagonal block (lower part); padding beyond kb is the identity
     load_tile(As, A, d, k0, kb, k0, kb, true, true);
@@ -421,18 +465,15 @@ __global__ void __launch_bounds__(256)
             }
         return;
     }
-    const int n_trsm = (d - k0 - kb + kNB - 1) / kNB;
-    if (static_cast<int>(blockIdx.x) > n_trsm) {
+    if (y_cta) {
         // column block cb of row block k of M^{-1} (pk0 >= 0 here)
-        const int cb = (blockIdx.x - 1 - n_trsm) * kNB;
-        load_tile(As, Minv, d, k0, kb, cb, kNB, false, false);   // Y~_k
-        load_tile(Pr, Minv, d, pk0, kNB, cb, kNB, false, false); // Y_{k-1}
+        cp_async_wait_all();
         __syncthreads();
         float t4[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) t4[i][j] = As[r0 + i][c0 + j];
+            for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
         for (int k = 0; k < kNB; ++k) {
             float a4[4], b4[4];
 #pragma unroll
@@ -472,30 +513,27 @@ __global__ void __launch_bounds__(256)
 
     // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k], with
     // T = A[rows][block] - P_prev[rows] P_prev,kk^T
-    const int pr0 = k0 + kb + (blockIdx.x - 1) * kNB;
-    const int prn = min(kNB, d - pr0);
-    load_tile(As, A, d, pr0, prn, k0, kb, false, false);
-    if (pk0 >= 0) load_tile(Pr, A, d, pr0, prn, pk0, kNB, false, false);
+    cp_async_wait_all();
     __syncthreads();
     if (pk0 >= 0) {
         float t4[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) t4[i][j] = As[r0 + i][c0 + j];
+            for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
         tile_minus_xyT(t4, Pr, Pd, r0, c0);
         __syncthreads();
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = (c0 + j < kb) ? t4[i][j] : 0.f;
+            for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = (c0 + j < kb) ? t4[i][j] : 0.f;
         __syncthreads();
     }
     float acc[4][4] = {};
     for (int k = 0; k < kNB; ++k) {
         float t[4], xv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = As[r0 + i][k];
+        for (int i = 0; i < 4; ++i) t[i] = Ts[r0 + i][k];
 #pragma unroll
         for (int j = 0; j < 4; ++j) xv[j] = Zs[c0 + j][k];
 #pragma unroll
