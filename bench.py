@@ -110,6 +110,57 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+PROFILE_TF32 = os.path.join(ROOT, "profiles", "tf32_peak_cublas.md")
+
+
+def tf32_peak():
+    """Measured dense tf32 throughput of the vendor GEMM (sustained), from the
+    committed measurement; None if it is missing."""
+    try:
+        for line in open(PROFILE_TF32):
+            if line.startswith("tf32_tflops_sustained:"):
+                return float(line.split(":", 1)[1].split()[0])
+    except OSError:
+        pass
+    return None
+
+
+def lazy_flops(spec) -> float:
+    """fp32 flops of all lazy-batch products of one layer: every (j, k) column
+    pair in different blocks, per row: d_out (d_in^2 - sum of block widths^2)."""
+    bw = [min(spec.block_size, spec.d_in - j) for j in range(0, spec.d_in, spec.block_size)]
+    return float(spec.d_out) * (spec.d_in ** 2 - sum(b * b for b in bw))
+
+
+def lazy_batch_line(spec, stage):
+    if not stage or not stage.get("lazy_batch_ms"):
+        return None
+    fl = lazy_flops(spec)
+    rate = fl / (stage["lazy_batch_ms"] / 1e3) / 1e12
+    peak = tf32_peak()
+    return {"flops_fp32": fl, "ms": stage["lazy_batch_ms"], "achieved_fp32_tflops": rate,
+            "tf32_rate_tflops": 3 * rate, "peak": peak, "unit": "TFLOP/s",
+            "frac": (3 * rate / peak) if peak else None,
+            "note": "3xTF32: three tf32 MMAs per fp32-accurate product; peak = measured cuBLAS tf32, sustained"}
+
+
+def layer_roofline(spec, ms, bf16_peak, stage):
+    """Ideal time of the layer's tensor work at the measured peaks (Hessian on
+    bf16, factorisation and lazy batch as 3xTF32) against the measured step;
+    the column loop's chain of dependent column steps has no flop roofline and
+    is not in the ideal."""
+    peak = tf32_peak()
+    if not peak:
+        return None
+    d = spec.d_in
+    t_h = spec.n_tokens * d * (d + 1) / (bf16_peak * 1e12) * 1e3
+    t_f = 3 * (2.0 / 3.0) * d ** 3 / (peak * 1e12) * 1e3
+    t_l = 3 * lazy_flops(spec) / (peak * 1e12) * 1e3
+    ideal = t_h + t_f + t_l
+    return {"ideal_ms": ideal, "measured_ms": ms, "frac": ideal / ms,
+            "terms_ms": {"hessian": t_h, "factorisation": t_f, "lazy_batch": t_l}}
+
+
 def profiled_traffic(kernel_src: str):
     """dram read+write bytes per launch of the Hessian kernel from the committed
     ncu summary, or None when the kernel source changed since the capture."""
@@ -301,6 +352,9 @@ def main():
         torch.cuda.synchronize()
         stage = {"hessian_ms": evs[0].elapsed_time(evs[1]), "prepare_ms": evs[1].elapsed_time(evs[2]),
                  "quantize_ms": evs[2].elapsed_time(evs[3])}
+        # the column-loop stage split into its kernel classes (events between launches)
+        qt = q.quantize_timed(Wd)
+        stage.update({"column_loop_ms": qt[0], "lazy_batch_ms": qt[1], "quantize_other_ms": qt[2]})
 
     # end to end through the public API with host buffers: X and W copied in
     # (overlapped chunked copy of X), packed codes + scales + zeros + g_idx out
@@ -362,6 +416,8 @@ def main():
                          "peak_source": f"{peak_kind} bf16_tflops_sustained",
                          "flops_per_launch": alg_flops, "launch_ms": h_ms},
             "hessian_tflops_dense_equiv": 2 * spec.n_tokens * spec.d_in ** 2 / (h_ms / 1e3) / 1e12,
+            "lazy_batch": lazy_batch_line(spec, stage),
+            "layer_roofline": layer_roofline(spec, ms, peak, stage),
             "stages_ms": stage,
             "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
             "e2e": e2e, "cpu_baseline": cpu,

@@ -214,6 +214,18 @@ int gptq_quantize_static_scratch(float *W, const float *Hinv_chol, const int32_t
                                  uint8_t *packed_int4, int32_t *g_idx, float *err_sq,
                                  void *stream);
 
+/* Diagnostic: gptq_quantize (same arguments, rules and results) enqueued
+ * directly on `stream` with a CUDA event after every launch; synchronises
+ * the stream and returns the summed device time of the column-loop kernels
+ * (*loop_ms), of the lazy-batch products (*update_ms) and of everything else
+ * (*other_ms: layout, gathers, unpermute/packing).  For measurement only:
+ * the events add small gaps between launches. */
+int gptq_quantize_timed(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
+                        int64_t d_in, int bits, int group_size, int block_size, uint8_t* codes,
+                        float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,
+                        float* err_sq, void* workspace, size_t ws_bytes, void* stream,
+                        float* loop_ms, float* update_ms, float* other_ms);
+
 /* Diagnostic of the bounded waits the tensor-core kernels use: launches one
  * warp that waits on an mbarrier nothing completes, with a limit of
  * `limit_cycles` SM clocks (0 < limit <= about 2e9), and returns what the

@@ -37,6 +37,8 @@ SIGNATURES = [
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize_static_scratch", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    ("gptq_quantize_timed", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                 _P, _P, _P, _P]),
     ("gptq_selftest_bounded_wait", _I, [_I64]),
     ("gptq_selftest_quotient", _I, [_I64, ctypes.c_uint64, _P]),
     ("gptq_bf16_to_f32", _I, [_P, _P, _I64, _P]),
@@ -183,6 +185,24 @@ def gptq_quantize(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor |
                                group_size, block_size, _ptr(codes), _ptr(scales), _ptr(zeros),
                                _ptr(packed_int4), _ptr(g_idx), _ptr(err_sq), _ptr(ws),
                                ws.numel(), _stream(W, stream)))
+
+
+def gptq_quantize_timed(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor | None, bits: int,
+                        group_size: int, block_size: int, scales: torch.Tensor, zeros: torch.Tensor,
+                        ws: torch.Tensor, codes: torch.Tensor | None = None,
+                        packed_int4: torch.Tensor | None = None, g_idx: torch.Tensor | None = None,
+                        err_sq: torch.Tensor | None = None, stream=None):
+    """gptq_quantize with per-class device times: returns (column-loop ms,
+    lazy-batch product ms, other ms) of this call (synchronises the stream)."""
+    _need(W, torch.float32, "W")
+    d_out, d_in = W.shape
+    out = [ctypes.c_float(0.0) for _ in range(3)]
+    _check("gptq_quantize_timed",
+           lib().gptq_quantize_timed(_ptr(W), _ptr(Hinv_chol), _ptr(perm), d_out, d_in, bits,
+                                     group_size, block_size, _ptr(codes), _ptr(scales), _ptr(zeros),
+                                     _ptr(packed_int4), _ptr(g_idx), _ptr(err_sq), _ptr(ws),
+                                     ws.numel(), _stream(W, stream), *(ctypes.byref(o) for o in out)))
+    return tuple(o.value for o in out)
 
 
 def gptq_quantize_static_scratch(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor | None,

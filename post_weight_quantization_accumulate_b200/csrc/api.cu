@@ -23,6 +23,10 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                  cudaStream_t s, bool graphed);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
+int run_quantize_timed(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
+                       int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
+                       uint8_t* packed, int32_t* g_idx, float* err_sq, void* workspace,
+                       size_t ws_bytes, cudaStream_t stream, float* ms_by_class);
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
@@ -139,7 +143,8 @@ __global__ void bounded_wait_selftest_kernel(long long limit_cycles, int* status
 int quantize_entry(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
                    int64_t d_in, int bits, int group_size, int block_size, uint8_t* codes,
                    float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,
-                   float* err_sq, void* workspace, size_t ws_bytes, void* stream, bool graphed)
+                   float* err_sq, void* workspace, size_t ws_bytes, void* stream, bool graphed,
+                   float* ms_by_class = nullptr)
 {
     if (!W || !Hinv_chol || !scales || !zeros || d_out <= 0 || d_in <= 0 || d_in > kMaxDim ||
         d_out > (int64_t(1) << 31) / 2 || d_in % 8 != 0 || bits < 1 || bits > 8 ||
@@ -156,6 +161,10 @@ int quantize_entry(float* W, const float* Hinv_chol, const int32_t* perm, int64_
         return GPTQ_ERR_WORKSPACE;
     int rc = check_device();
     if (rc) return rc;
+    if (ms_by_class)
+        return run_quantize_timed(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size,
+                                  codes, scales, zeros, packed_int4, g_idx, err_sq, workspace,
+                                  ws_bytes, static_cast<cudaStream_t>(stream), ms_by_class);
     return run_quantize(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
                         scales, zeros, packed_int4, g_idx, err_sq, workspace, ws_bytes,
                         static_cast<cudaStream_t>(stream), graphed);
@@ -308,6 +317,23 @@ int gptq_quantize(float* W, const float* Hinv_chol, const int32_t* perm, int64_t
     return quantize_entry(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size, codes,
                           scales, zeros, packed_int4, g_idx, err_sq, workspace, ws_bytes, stream,
                           true);
+}
+
+int gptq_quantize_timed(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
+                        int64_t d_in, int bits, int group_size, int block_size, uint8_t* codes,
+                        float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,
+                        float* err_sq, void* workspace, size_t ws_bytes, void* stream,
+                        float* loop_ms, float* update_ms, float* other_ms)
+{
+    if (!loop_ms || !update_ms || !other_ms) return GPTQ_ERR_INVALID_ARG;
+    float ms[3] = {0.f, 0.f, 0.f};
+    const int rc = quantize_entry(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size,
+                                  codes, scales, zeros, packed_int4, g_idx, err_sq, workspace,
+                                  ws_bytes, stream, false, ms);
+    *other_ms = ms[0];
+    *loop_ms = ms[1];
+    *update_ms = ms[2];
+    return rc;
 }
 
 int gptq_selftest_bounded_wait(int64_t limit_cycles)

@@ -52,7 +52,8 @@ namespace gptq {
 int quantize_entry(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
                    int64_t d_in, int bits, int group_size, int block_size, uint8_t* codes,
                    float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,
-                   float* err_sq, void* workspace, size_t ws_bytes, void* stream, bool graphed);
+                   float* err_sq, void* workspace, size_t ws_bytes, void* stream, bool graphed,
+                   float* ms_by_class);
 }
 
 extern "C" int gptq_quantize_static_scratch(float* W, const float* Hinv_chol,
@@ -75,5 +76,5 @@ extern "C" int gptq_quantize_static_scratch(float* W, const float* Hinv_chol,
     // launches are enqueued directly (no graph is instantiated for this path).
     return gptq::quantize_entry(W, Hinv_chol, perm, d_out, d_in, bits, group_size, block_size,
                                 codes, scales, zeros, packed_int4, g_idx, err_sq, scratch,
-                                GPTQ_STATIC_SCRATCH_BYTES, stream, false);
+                                GPTQ_STATIC_SCRATCH_BYTES, stream, false, nullptr);
 }

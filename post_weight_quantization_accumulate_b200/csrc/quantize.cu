@@ -23,6 +23,8 @@
 #include "common.cuh"
 #include "gemm.cuh"
 
+#include <vector>
+
 namespace gptq {
 
 namespace {
@@ -564,11 +566,35 @@ size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
            up256(static_cast<size_t>(d_in) * static_cast<size_t>(d_in) * sizeof(float));
 }
 
+// Optional CUDA-event marks between the launches of one enqueue (the
+// diagnostic entry point): an event after every launch, tagged with the class
+// of the launch it ends (0 = other, 1 = column loop, 2 = lazy-batch product).
+struct QuantizeMarks {
+    std::vector<cudaEvent_t> ev;
+    std::vector<int> cls;
+    int mark(cudaStream_t s, int c)
+    {
+        cudaEvent_t e = nullptr;
+        GPTQ_CUDA_CHECK(cudaEventCreate(&e));
+        ev.push_back(e);
+        cls.push_back(c);
+        GPTQ_CUDA_CHECK(cudaEventRecord(e, s));
+        return GPTQ_OK;
+    }
+    ~QuantizeMarks()
+    {
+        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    }
+};
+
 static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out64,
                             int64_t d_in64, int bits, int gs, int block, uint8_t* codes,
                             float* scales, float* zeros, uint8_t* packed, int32_t* g_idx,
-                            float* err_sq, void* workspace, bool with_low_parts, cudaStream_t stream)
+                            float* err_sq, void* workspace, bool with_low_parts, cudaStream_t stream,
+                            QuantizeMarks* marks = nullptr)
 {
+    auto mark = [&](int c) { return marks ? marks->mark(stream, c) : GPTQ_OK; };
+    if (int rc = mark(0)) return rc;
     const int d_out = static_cast<int>(d_out64), d_in = static_cast<int>(d_in64);
     const size_t n = static_cast<size_t>(d_out) * d_in;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -649,11 +675,13 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
             const int bw = (J1 - j0 < block) ? J1 - j0 : block;
             QArgs a{work, Ul, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
                     codes_p, E, E_lo, j0 - J0, err_sq, status};
+            if (int rc = mark(0)) return rc;
             if (groups_in_step)
                 gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
             else
                 gptq_block_kernel<false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
             GPTQ_LAUNCH_CHECK();
+            if (int rc = mark(1)) return rc;
             const int rest_in = J1 - j0 - bw;
             if (rest_in > 0) {
                 const int64_t uo = static_cast<int64_t>(j0) * d_in + j0 + bw;
@@ -661,6 +689,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                                       U + uo, d_in, 0, 1.f, work + j0 + bw, d_in, 0, 1, 0, stream, 0,
                                       E_lo ? E_lo + (j0 - J0) : nullptr, U_lo ? U_lo + uo : nullptr);
                 if (rc) return rc;
+                if ((rc = mark(2))) return rc;
             }
         }
         const int rest = d_in - J1;
@@ -670,6 +699,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                                   1.f, work + J1, d_in, 0, 1, 0, stream, 0, E_lo,
                                   U_lo ? U_lo + uo : nullptr);
             if (rc) return rc;
+            if ((rc = mark(2))) return rc;
         }
     }
     if (codes || packed || perm) {
@@ -681,7 +711,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         g_idx_kernel<<<(d_in + 255) / 256, 256, 0, stream>>>(perm, d_in, gs, g_idx);
         GPTQ_LAUNCH_CHECK();
     }
-    return GPTQ_OK;
+    return mark(0);
 }
 
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in, int bits,
@@ -703,6 +733,26 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                                        P(packed), P(g_idx), P(err_sq), P(workspace),
                                        static_cast<uint64_t>(low)};
     return run_graphed(key, false, enq, stream, nullptr);
+}
+
+int run_quantize_timed(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
+                       int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
+                       uint8_t* packed, int32_t* g_idx, float* err_sq, void* workspace,
+                       size_t ws_bytes, cudaStream_t stream, float* ms_by_class)
+{
+    QuantizeMarks marks;
+    const bool low = ws_bytes >= quantize_workspace_bytes(d_out, d_in);
+    int rc = enqueue_quantize(W, U, perm, d_out, d_in, bits, gs, block, codes, scales, zeros, packed,
+                              g_idx, err_sq, workspace, low, stream, &marks);
+    if (rc) return rc;
+    GPTQ_CUDA_CHECK(cudaStreamSynchronize(stream));
+    for (int c = 0; c < 3; ++c) ms_by_class[c] = 0.f;
+    for (size_t i = 1; i < marks.ev.size(); ++i) {
+        float ms = 0.f;
+        GPTQ_CUDA_CHECK(cudaEventElapsedTime(&ms, marks.ev[i - 1], marks.ev[i]));
+        ms_by_class[marks.cls[i]] += ms;
+    }
+    return GPTQ_OK;
 }
 
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches)

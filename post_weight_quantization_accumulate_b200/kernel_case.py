@@ -25,13 +25,50 @@ from post_weight_quantization_accumulate_b200 import synth  # noqa: E402
 from post_weight_quantization_accumulate_b200.layer import LayerQuantizer  # noqa: E402
 
 
+def tf32_peak(n: int = 8192, seconds: float = 3.0):
+    """Dense tf32 tensor-core throughput of the vendor GEMM (cuBLAS through
+    torch.matmul on float32 with tf32 allowed): a burst (3 products after
+    warm-up) and a sustained figure (back-to-back products for `seconds`), the
+    denominators of the lazy-batch products' roofline."""
+    torch.backends.cuda.matmul.allow_tf32 = True
+    dev = torch.device("cuda", 0)
+    a = torch.randn(n, n, device=dev)
+    b = torch.randn(n, n, device=dev)
+    c = torch.empty(n, n, device=dev)
+    flop = 2.0 * n ** 3
+    for _ in range(3):
+        torch.matmul(a, b, out=c)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        torch.matmul(a, b, out=c)
+    e1.record()
+    torch.cuda.synchronize()
+    burst = 3 * flop / (e0.elapsed_time(e1) / 1e3) / 1e12
+    reps = max(3, int(seconds / (e0.elapsed_time(e1) / 3e3)))
+    e0.record()
+    for _ in range(reps):
+        torch.matmul(a, b, out=c)
+    e1.record()
+    torch.cuda.synchronize()
+    sustained = reps * flop / (e0.elapsed_time(e1) / 1e3) / 1e12
+    print(f"tf32_tflops: {burst:.1f}")
+    print(f"tf32_tflops_sustained: {sustained:.1f}")
+    print(f"(n = {n}, {reps} products in the sustained loop)")
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--call", default="hessian", choices=["hessian", "prepare", "quantize", "layer"])
+    ap.add_argument("--call", default="hessian",
+                    choices=["hessian", "prepare", "quantize", "layer", "tf32_peak"])
     ap.add_argument("--workload", default="q_proj_4096")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
     a = ap.parse_args()
+    if a.call == "tf32_peak":
+        tf32_peak()
+        return
     spec = synth.WORKLOADS[a.workload]
     if a.tokens:
         spec = synth.scaled(spec, n_tokens=a.tokens)

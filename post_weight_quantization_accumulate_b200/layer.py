@@ -88,6 +88,18 @@ class LayerQuantizer:
         return QuantizedLayer(self.packed, self.codes, self.scales, self.zeros, self.g_idx,
                               self.perm, self.W, self.err_sq)
 
+    def quantize_timed(self, W: torch.Tensor):
+        """As quantize, enqueued directly with CUDA events between launches;
+        returns (column-loop ms, lazy-batch product ms, other ms)."""
+        if W.dtype == torch.bfloat16:
+            B.gptq_bf16_to_f32(self.W, W)
+        else:
+            self.W.copy_(W)
+        return B.gptq_quantize_timed(self.W, self.U, self.perm if self.act_order else None, self.bits,
+                                     self.group_size, self.block_size, self.scales, self.zeros, self.ws,
+                                     codes=self.codes, packed_int4=self.packed, g_idx=self.g_idx,
+                                     err_sq=self.err_sq)
+
     def run(self, W: torch.Tensor) -> QuantizedLayer:
         self.prepare()
         return self.quantize(W)

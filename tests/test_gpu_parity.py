@@ -303,3 +303,31 @@ def test_minimum_workspace_gives_the_same_results():
     np.testing.assert_array_equal(outs[0][2], outs[1][2])
     np.testing.assert_array_equal(outs[0][1], outs[1][1])
     np.testing.assert_allclose(outs[0][0], outs[1][0], rtol=1e-6, atol=1e-8)
+
+
+def test_timed_quantize_matches_and_reports_times():
+    """The timing diagnostic runs the same launches as gptq_quantize (direct
+    enqueue instead of a graph replay): identical codes, and positive times
+    for the column loop and the lazy-batch products."""
+    d_out, d_in, bits, gs = 256, 1024, 4, 128
+    W, xb = synth.random_layer(22, d_out, d_in, 2 * d_in, correlated=True)
+    H = torch.zeros(d_in, d_in, dtype=torch.float32, device=DEV)
+    B.gptq_hessian_accumulate(H, torch.from_numpy(xb.view(np.int16)).to(DEV).view(torch.bfloat16))
+    U = torch.empty(d_in, d_in, dtype=torch.float32, device=DEV)
+    perm = torch.empty(d_in, dtype=torch.int32, device=DEV)
+    ws = B.workspace(d_out, d_in, 128)
+    B.gptq_prepare(H, 0.01, 0, perm, U, ws)
+    res = []
+    for timed in (False, True):
+        Wt = torch.from_numpy(W.astype(np.float32)).to(DEV)
+        sc = torch.empty(d_out, d_in // gs, device=DEV)
+        zr = torch.empty(d_out, d_in // gs, device=DEV)
+        codes = torch.empty(d_out, d_in, dtype=torch.uint8, device=DEV)
+        if timed:
+            loop_ms, upd_ms, other_ms = B.gptq_quantize_timed(Wt, U, None, bits, gs, 128, sc, zr, ws, codes=codes)
+            assert loop_ms > 0 and upd_ms > 0 and other_ms >= 0
+        else:
+            B.gptq_quantize(Wt, U, None, bits, gs, 128, sc, zr, ws, codes=codes)
+        torch.cuda.synchronize()
+        res.append(codes.cpu().numpy())
+    np.testing.assert_array_equal(res[0], res[1])
