@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="decoder_layer: bits {2,3,4} x group_size {64,128,per-channel}")
     return ap.parse_args()
 
 
@@ -252,6 +254,49 @@ def config_of(spec, n):
 
 # ------------------------------------------------------------------ our arm
 
+def run_decoder_layer(args, rank) -> int:
+    """Layer-sequential calibration of a Llama-2-7B-shaped decoder layer (all
+    seven linears, one Hessian per input group, each group's input produced by
+    the quantized earlier groups) on one GPU; one JSON line, rank 0 only."""
+    if rank != 0:
+        return 0
+    import torch
+    from post_weight_quantization_accumulate_b200 import build as build_mod
+    from post_weight_quantization_accumulate_b200 import decoder as D
+
+    build_mod.build()
+    torch.cuda.set_device(0)
+    shape = D.LLAMA2_7B
+    W, X = D.synthetic_layer(shape)
+    combos = [(b, g) for b in (2, 3, 4) for g in (64, 128, -1)] if args.sweep else [(4, 128)]
+    for _ in range(max(1, min(args.warmup, 1))):
+        D.calibrate(X, W, shape, bits=4, group_size=128)
+    torch.cuda.synchronize()
+    rows = []
+    for bits, gs in combos:
+        ms = []
+        for _ in range(max(1, min(args.steps, 3))):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            r = D.calibrate(X, W, shape, bits=bits, group_size=gs)
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        rows.append({"bits": bits, "group_size": gs, "ms": min(ms), "groups_ms": r.ms})
+        del r
+    n_w = D.quantized_weights(shape)
+    best = rows[-1] if not args.sweep else next(r for r in rows if r["bits"] == 4 and r["group_size"] == 128)
+    print(json.dumps({
+        "metric": "GPTQ quantized weights/s, full decoder layer (7 linears, layer-sequential)",
+        "value": n_w / (best["ms"] / 1e3), "unit": "weights/s", "n_gpus": 1,
+        "ms_per_layer": best["ms"], "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "llama2_7b_decoder_layer", "d_model": shape.d_model, "d_ff": shape.d_ff,
+                   "n_tokens": shape.n_tokens, "weights": n_w,
+                   "glue": "vendor bf16 GEMM between groups (not a GPTQ step)"},
+        "sweep": rows}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -259,6 +304,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload == "decoder_layer":
+        return run_decoder_layer(args, rank)
 
     import numpy as np
     import torch

@@ -32,6 +32,7 @@ struct PrepHeader {
 };
 
 constexpr int kNB = 64;  // panel width of the blocked Cholesky / leaf of the inverse
+constexpr int kPanelMaxCtas = 64;
 
 size_t prepare_workspace_bytes(int64_t d)
 {
@@ -239,21 +240,38 @@ __global__ void __launch_bounds__(256)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
+    // Second-phase work items: n_trsm blocks of 64 panel rows, then (from the
+    // second panel on) k0/64 column blocks of M^{-1}'s row block; CTA b >= 1
+    // takes items b-1, b-1 + (G-1), ...
     const int n_trsm = (d - k0 - kb + kNB - 1) / kNB;
-    const bool y_cta = static_cast<int>(blockIdx.x) > n_trsm;
-    const int pr0 = k0 + kb + (static_cast<int>(blockIdx.x) - 1) * kNB;   // TRSM CTAs
-    const int prn = min(kNB, d - pr0);
-    const int cb = (static_cast<int>(blockIdx.x) - 1 - n_trsm) * kNB;      // M^{-1} CTAs
+    const int n_items = n_trsm + (pk0 >= 0 ? k0 / kNB : 0);
+    const int stride = static_cast<int>(gridDim.x) - 1;
+    auto fetch_item = [&](int it, bool async) {
+        if (it >= n_trsm) {
+            const int cb = (it - n_trsm) * kNB;
+            if (async) {
+                load_tile_async(Ts, Minv, d, k0, kb, cb, kNB);   // Y~_k
+                load_tile_async(Pr, Minv, d, pk0, kNB, cb, kNB); // Y_{k-1}
+            } else {
+                load_tile(Ts, Minv, d, k0, kb, cb, kNB, false, false);
+                load_tile(Pr, Minv, d, pk0, kNB, cb, kNB, false, false);
+            }
+        } else {
+            const int pr0 = k0 + kb + it * kNB;
+            const int prn = min(kNB, d - pr0);
+            if (async) {
+                load_tile_async(Ts, A, d, pr0, prn, k0, kb);
+                if (pk0 >= 0) load_tile_async(Pr, A, d, pr0, prn, pk0, kNB);
+            } else {
+                load_tile(Ts, A, d, pr0, prn, k0, kb, false, false);
+                if (pk0 >= 0) load_tile(Pr, A, d, pr0, prn, pk0, kNB, false, false);
+            }
+        }
+    };
 
-    // The operand tiles of the second phase do not depend on the diagonal
+    // The operand tiles of the first item do not depend on the diagonal
     // block: they are fetched asynchronously while it is factored.
-    if (y_cta) {
-        load_tile_async(Ts, Minv, d, k0, kb, cb, kNB);   // Y~_k
-        load_tile_async(Pr, Minv, d, pk0, kNB, cb, kNB); // Y_{k-1}
-    } else if (blockIdx.x > 0) {
-        load_tile_async(Ts, A, d, pr0, prn, k0, kb);
-        if (pk0 >= 0) load_tile_async(Pr, A, d, pr0, prn, pk0, kNB);
-    }
+    if (blockIdx.x > 0 && static_cast<int>(blockIdx.x) - 1 < n_items) fetch_item(blockIdx.x - 1, true);
     cp_async_commit();
 
     // diagonal block (lower part); padding beyond kb is the identity
@@ -465,89 +483,94 @@ __global__ void __launch_bounds__(256)
             }
         return;
     }
-    if (y_cta) {
-        // column block cb of row block k of M^{-1} (pk0 >= 0 here)
-        cp_async_wait_all();
-        __syncthreads();
-        float t4[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
-        for (int k = 0; k < kNB; ++k) {
-            float a4[4], b4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a4[i] = Pd[r0 + i][k];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) b4[j] = Pr[k][c0 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) t4[i][j] = fmaf(-a4[i], b4[j], t4[i][j]);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = t4[i][j];
-        __syncthreads();
-        float y4[4][4] = {};
-        for (int k = 0; k < kNB; ++k) {
-            float a4[4], b4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a4[i] = Zs[r0 + i][k];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) b4[j] = As[k][c0 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) y4[i][j] = fmaf(a4[i], b4[j], y4[i][j]);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (r0 + i < kb) Minv[static_cast<int64_t>(k0 + r0 + i) * d + cb + c0 + j] = y4[i][j];
-        return;
-    }
-
-    // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k], with
-    // T = A[rows][block] - P_prev[rows] P_prev,kk^T
     cp_async_wait_all();
-    __syncthreads();
-    if (pk0 >= 0) {
-        float t4[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
-        tile_minus_xyT(t4, Pr, Pd, r0, c0);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = (c0 + j < kb) ? t4[i][j] : 0.f;
-        __syncthreads();
-    }
-    float acc[4][4] = {};
-    for (int k = 0; k < kNB; ++k) {
-        float t[4], xv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = Ts[r0 + i][k];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) xv[j] = Zs[c0 + j][k];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(t[i], xv[j], acc[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = pr0 + r0 + i, cj = c0 + j;
-            if (r < d && cj < kb) A[static_cast<int64_t>(r) * d + k0 + cj] = acc[i][j];
+    for (int it = blockIdx.x - 1; it < n_items; it += stride) {
+        if (it != static_cast<int>(blockIdx.x) - 1) {
+            __syncthreads();   // the previous item is done with Ts, Pr and As
+            fetch_item(it, false);
         }
+        __syncthreads();
+        if (it >= n_trsm) {
+            // column block cb of row block k of M^{-1} (pk0 >= 0 here)
+            const int cb = (it - n_trsm) * kNB;
+            float t4[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
+            for (int k = 0; k < kNB; ++k) {
+                float a4[4], b4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a4[i] = Pd[r0 + i][k];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) b4[j] = Pr[k][c0 + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) t4[i][j] = fmaf(-a4[i], b4[j], t4[i][j]);
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = t4[i][j];
+            __syncthreads();
+            float y4[4][4] = {};
+            for (int k = 0; k < kNB; ++k) {
+                float a4[4], b4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a4[i] = Zs[r0 + i][k];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) b4[j] = As[k][c0 + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) y4[i][j] = fmaf(a4[i], b4[j], y4[i][j]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (r0 + i < kb) Minv[static_cast<int64_t>(k0 + r0 + i) * d + cb + c0 + j] = y4[i][j];
+            continue;
+        }
+        // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k], with
+        // T = A[rows][block] - P_prev[rows] P_prev,kk^T
+        const int pr0 = k0 + kb + it * kNB;
+        if (pk0 >= 0) {
+            float t4[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
+            tile_minus_xyT(t4, Pr, Pd, r0, c0);
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = (c0 + j < kb) ? t4[i][j] : 0.f;
+            __syncthreads();
+        }
+        float acc[4][4] = {};
+        for (int k = 0; k < kNB; ++k) {
+            float t[4], xv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) t[i] = Ts[r0 + i][k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xv[j] = Zs[c0 + j][k];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(t[i], xv[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = pr0 + r0 + i, cj = c0 + j;
+                if (r < d && cj < kb) A[static_cast<int64_t>(r) * d + k0 + cj] = acc[i][j];
+            }
+    }
 }
 
 // U[i][j] = Minv[d-1-i][d-1-j] for i <= j, 0 below the diagonal.
@@ -672,7 +695,9 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
         const int kb = std::min(kNB, d - k0);
         const int rest = d - k0 - kb;
         const int n_trsm = (rest + kNB - 1) / kNB;
-        const int n_cta = 1 + n_trsm + p;
+        // CTA 0 writes L_kk^{-1}; the others share the panel's work items, at
+        // most kPanelMaxCtas of them so the side products keep enough SMs
+        const int n_cta = std::min(1 + n_trsm + p, kPanelMaxCtas);
         // SMs the side products may hold: the rest after this panel's CTAs,
         // split between the two side streams in proportion to their flops
         // (rest2^2 / 2 for the symmetric update, rest2 (k0 + kb) for M^{-1})
