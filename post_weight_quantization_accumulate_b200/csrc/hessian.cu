@@ -165,18 +165,26 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
                  : "memory");
 }
 
-// Upper-triangle tile number -> (ti, tj), tj >= ti.
+// Upper-triangle tile number -> (ti, tj), tj >= ti, in bands of kBand tile
+// rows enumerated column by column: the pairs running at the same time (same
+// token span, consecutive tile numbers) then cover a compact block of tiles
+// and share both operand slices of X in L2, instead of one tile row sharing A
+// and streaming a different B slice each.
+constexpr int kBand = 8;
 __device__ __forceinline__ void tile_coords(int tile, int n_t, int& ti, int& tj)
 {
     int idx = tile;
-    for (int i = 0; i < n_t; ++i) {
-        const int cnt = n_t - i;
-        if (idx < cnt) {
-            ti = i;
-            tj = i + idx;
-            return;
+    for (int b0 = 0; b0 < n_t; b0 += kBand) {
+        const int b1 = min(b0 + kBand, n_t);
+        for (int c = b0; c < n_t; ++c) {
+            const int cnt = min(c + 1, b1) - b0;   // rows b0 .. min(c, b1-1)
+            if (idx < cnt) {
+                ti = b0 + idx;
+                tj = c;
+                return;
+            }
+            idx -= cnt;
         }
-        idx -= cnt;
     }
     ti = n_t - 1;
     tj = n_t - 1;
