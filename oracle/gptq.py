@@ -201,6 +201,42 @@ def g_idx(perm: np.ndarray, group_size: int) -> np.ndarray:
     return g
 
 
+def unpack_int4(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_int4: codes [..., 2 * bytes], low nibble first."""
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 15
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def dequant_int4(packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray,
+                 g_idx: np.ndarray | None, group_size: int) -> np.ndarray:
+    """W^[n][k] = scales[n][g] * (q[n][k] - zeros[n][g]) from the packed 4-bit
+    storage (AutoGPTQ page, "Mixed Precision Scheme": int4 weights dequantized
+    with their group's scale at inference), g = g_idx[k] when given, else
+    k // group_size (group_size -1: one group per row).  The exact product of
+    the binary32 scale and the integer q - z, in float64 (as the column loop
+    here forms W^)."""
+    q = unpack_int4(packed).astype(np.float32)
+    K = q.shape[1]
+    if g_idx is not None:
+        g = np.asarray(g_idx, dtype=np.int64)
+    else:
+        g = (np.arange(K) // group_size) if group_size > 0 else np.zeros(K, dtype=np.int64)
+    s = np.asarray(scales, dtype=np.float32)[:, g].astype(np.float64)
+    z = np.asarray(zeros, dtype=np.float32)[:, g].astype(np.float64)
+    return s * (q.astype(np.float64) - z)
+
+
+def w4a16(x_bits: np.ndarray, packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray,
+          g_idx: np.ndarray | None, group_size: int) -> np.ndarray:
+    """Y = X W^T in float64 for bf16 activations X [M, K] (bits) and the packed
+    4-bit weights [N, K/2] (the inference-side use of the quantized layer)."""
+    x = bf16_bits_to_f64(x_bits)
+    return x @ dequant_int4(packed, scales, zeros, g_idx, group_size).T
+
+
 def pack_int4(codes: np.ndarray) -> np.ndarray:
     """Two codes per byte: column 2i in the low nibble, 2i+1 in the high one."""
     c = np.asarray(codes, dtype=np.uint8)

@@ -372,3 +372,41 @@ def test_codes_in_range_and_packing_roundtrip():
     s = np.take_along_axis(r["scales"], np.broadcast_to(r["g_idx"], r["codes"].shape), axis=1)
     z = np.take_along_axis(r["zeros"], np.broadcast_to(r["g_idx"], r["codes"].shape), axis=1)
     np.testing.assert_array_equal(s.astype(np.float64) * (r["codes"] - z.astype(np.float64)), r["W_hat"])
+
+
+# ---- P-l: the packed-format consumer (W4A16 product) -------------------------
+
+def test_unpack_inverts_pack():
+    g = np.random.default_rng(11)
+    c = g.integers(0, 16, size=(5, 64), dtype=np.uint8)
+    np.testing.assert_array_equal(oracle.unpack_int4(oracle.pack_int4(c)), c)
+
+
+@pytest.mark.parametrize("act_order,gs", [(False, 32), (True, 32), (False, -1)])
+def test_dequant_of_packed_output_is_the_quantizers_w_hat(act_order, gs):
+    """Dequantizing the packed codes with the scales, zeros and g_idx reproduces
+    the W^ the column loop formed column by column (an independent path
+    through the storage format: packing, group map, zero points)."""
+    W, xb = synth.random_layer(12, 16, 64, 256, correlated=True)
+    r = oracle.layer(W, xb, 4, gs, act_order=act_order)
+    Wd = oracle.dequant_int4(r["packed"], r["scales"], r["zeros"],
+                             r["g_idx"] if act_order else None, gs)
+    np.testing.assert_array_equal(Wd, r["W_hat"])
+
+
+def test_w4a16_matches_brute_force_sum():
+    g = np.random.default_rng(13)
+    M, N, K, gs = 3, 4, 16, 8
+    codes = g.integers(0, 16, size=(N, K), dtype=np.uint8)
+    scales = g.uniform(0.01, 0.1, size=(N, K // gs)).astype(np.float32)
+    zeros = g.integers(0, 16, size=(N, K // gs)).astype(np.float32)
+    gidx = g.permutation(np.repeat(np.arange(K // gs), gs)).astype(np.int32)
+    xb = synth.f32_to_bf16_bits(g.standard_normal((M, K)).astype(np.float32))
+    x = synth.bf16_bits_to_f32(xb).astype(np.float64)
+    Y = oracle.w4a16(xb, oracle.pack_int4(codes), scales, zeros, gidx, gs)
+    for m, n in itertools.product(range(M), range(N)):
+        ref = 0.0
+        for k in range(K):
+            w = float(scales[n, gidx[k]]) * (float(codes[n, k]) - float(zeros[n, gidx[k]]))
+            ref += x[m, k] * w
+        assert abs(Y[m, n] - ref) <= 1e-12 * (1 + abs(ref))
