@@ -241,6 +241,41 @@ int gptq_selftest_bounded_wait(int64_t limit_cycles);
  * Expected 0.  Uses the default stream and synchronises the device. */
 int gptq_selftest_quotient(int64_t n_pairs, uint64_t seed, int64_t* mismatches);
 
+/* Paths of gptq_w4a16_gemm. */
+enum { GPTQ_W4A16_AUTO = 0, GPTQ_W4A16_TENSOR_CORE = 1, GPTQ_W4A16_GENERAL = 2 };
+
+/*
+ * Y = X W^T with W^ the dequantized 4-bit weights gptq_quantize writes: the
+ * consumer of its packed format (AutoGPTQ page, "Mixed Precision Scheme":
+ * 4-bit weights, 16-bit activations, dequantized on the fly inside the
+ * product).  W^[n][k] = scales[n][g] * (q[n][k] - zeros[n][g]) with
+ * g = g_idx[k] when g_idx is given, else k / group_size (0 for group_size
+ * -1); q[n][k] is nibble k of row n of `packed`.
+ *   Y           float32 [M, N] OUT, row-major.
+ *   X           bf16 [M, K] row-major (uint16 bit patterns), 16-byte aligned.
+ *   packed      uint8 [N, K / 2]: column 2i in the low nibble of byte i,
+ *               2i + 1 in the high nibble; 16-byte aligned.
+ *   scales      float32 [N, n_groups], zeros float32 [N, n_groups] with
+ *               integer values 0..15; n_groups = K / group_size (1 for -1).
+ *   g_idx       int32 [K] or NULL (groups contiguous along K).
+ *   M >= 0, N >= 0, K > 0 with K % 8 == 0; group_size -1 or dividing K.
+ *   path        GPTQ_W4A16_AUTO picks the tensor-core path when it applies:
+ *               g_idx NULL, K % 32 == 0, group_size dividing 128 (a multiple
+ *               of 16) or a multiple of 128 or -1.  GPTQ_W4A16_TENSOR_CORE
+ *               asks for it (GPTQ_ERR_INVALID_ARG when it does not apply);
+ *               GPTQ_W4A16_GENERAL takes the SIMT path for any layout.
+ * Tensor-core path: Y = sum_g s * (sum over the group's columns of
+ * (q - z) x), the inner sums exact bf16 products accumulated in fp32 on
+ * tcgen05 (q - z is exact in bf16), the scale applied per group; split-K
+ * partial sums are added in a fixed order, so results are deterministic.
+ * General path: fp32 W^ = s * (q - z) and fp32 dot products.  Both are
+ * X W^T up to fp32 rounding of the sums.  Stream-ordered; allocates nothing.
+ * Y must not overlap the inputs.
+ */
+int gptq_w4a16_gemm(float *Y, const uint16_t *X, const uint8_t *packed, const float *scales,
+                    const float *zeros, const int32_t *g_idx, int64_t M, int64_t N, int64_t K,
+                    int group_size, int path, void *stream);
+
 /* dst[i] = (float) bf16 src[i] (exact widening), n >= 0 elements. */
 int gptq_bf16_to_f32(float *dst, const uint16_t *src, int64_t n, void *stream);
 

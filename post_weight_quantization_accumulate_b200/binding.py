@@ -41,8 +41,11 @@ SIGNATURES = [
                                  _P, _P, _P, _P]),
     ("gptq_selftest_bounded_wait", _I, [_I64]),
     ("gptq_selftest_quotient", _I, [_I64, ctypes.c_uint64, _P]),
+    ("gptq_w4a16_gemm", _I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P]),
     ("gptq_bf16_to_f32", _I, [_P, _P, _I64, _P]),
 ]
+
+W4A16_AUTO, W4A16_TENSOR_CORE, W4A16_GENERAL = 0, 1, 2
 
 _lib = None
 _lock = threading.Lock()
@@ -233,6 +236,23 @@ def gptq_selftest_quotient(n_pairs: int, seed: int = 0) -> int:
     _check("gptq_selftest_quotient",
            lib().gptq_selftest_quotient(int(n_pairs), ctypes.c_uint64(seed), ctypes.byref(out)))
     return out.value
+
+
+def gptq_w4a16_gemm(Y: torch.Tensor, X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                    zeros: torch.Tensor, g_idx: torch.Tensor | None, group_size: int,
+                    path: int = W4A16_AUTO, stream=None):
+    """Y float32 [M, N] = X (bf16 [M, K]) times the dequantized packed 4-bit
+    weights (uint8 [N, K/2]) transposed."""
+    _need(Y, torch.float32, "Y")
+    _need(X, torch.bfloat16, "X")
+    _need(packed, torch.uint8, "packed")
+    M, K = X.shape
+    N = packed.shape[0]
+    if Y.shape != (M, N) or packed.shape[1] * 2 != K:
+        raise ValueError("shape mismatch")
+    _check("gptq_w4a16_gemm",
+           lib().gptq_w4a16_gemm(_ptr(Y), _ptr(X), _ptr(packed), _ptr(scales), _ptr(zeros),
+                                 _ptr(g_idx), M, N, K, group_size, path, _stream(Y, stream)))
 
 
 def gptq_bf16_to_f32(dst: torch.Tensor, src: torch.Tensor, stream=None):

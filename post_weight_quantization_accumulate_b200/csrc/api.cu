@@ -23,6 +23,11 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                  cudaStream_t s, bool graphed);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
+bool w4a16_tc_supported(const uint16_t* X, const uint8_t* packed, const int32_t* g_idx,
+                        int64_t K, int gs);
+int run_w4a16(float* Y, const uint16_t* X, const uint8_t* packed, const float* scales,
+              const float* zeros, const int32_t* g_idx, int64_t M, int64_t N, int64_t K, int gs,
+              int path, cudaStream_t stream);
 int run_quantize_timed(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
                        int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
                        uint8_t* packed, int32_t* g_idx, float* err_sq, void* workspace,
@@ -68,6 +73,13 @@ uint64_t launch_count() { return t_launches; }
 int cuda_fail(cudaError_t e)
 {
     snprintf(g_last_error, sizeof g_last_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return GPTQ_ERR_CUDA;
+}
+
+int cuda_fail_msg(const char* where, cudaError_t e)
+{
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s: %s", where, cudaGetErrorName(e),
+             cudaGetErrorString(e));
     return GPTQ_ERR_CUDA;
 }
 
@@ -354,6 +366,27 @@ int gptq_selftest_quotient(int64_t n_pairs, uint64_t seed, int64_t* mismatches)
     int rc = check_device();
     if (rc) return rc;
     return run_quotient_selftest(n_pairs, seed, mismatches);
+}
+
+int gptq_w4a16_gemm(float* Y, const uint16_t* X, const uint8_t* packed, const float* scales,
+                    const float* zeros, const int32_t* g_idx, int64_t M, int64_t N, int64_t K,
+                    int group_size, int path, void* stream)
+{
+    if (M < 0 || N < 0 || K <= 0 || K % 8 != 0 || K > (int64_t(1) << 30) ||
+        M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || M * N > (int64_t(1) << 40) ||
+        path < GPTQ_W4A16_AUTO || path > GPTQ_W4A16_GENERAL)
+        return GPTQ_ERR_INVALID_ARG;
+    if (group_size != -1 && (group_size <= 0 || K % group_size != 0)) return GPTQ_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return GPTQ_OK;
+    if (!Y || !X || !packed || !scales || !zeros || !aligned(X, 16) || !aligned(packed, 16) ||
+        !aligned(Y, 4) || !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(g_idx, 4))
+        return GPTQ_ERR_INVALID_ARG;
+    if (path == GPTQ_W4A16_TENSOR_CORE && !w4a16_tc_supported(X, packed, g_idx, K, group_size))
+        return GPTQ_ERR_INVALID_ARG;
+    int rc = check_device();
+    if (rc) return rc;
+    return run_w4a16(Y, X, packed, scales, zeros, g_idx, M, N, K, group_size, path,
+                     static_cast<cudaStream_t>(stream));
 }
 
 int gptq_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, void* stream)

@@ -8,6 +8,7 @@
 
 #include "../../include/gptq.h"
 
+#include <algorithm>
 #include <functional>
 #include <vector>
 
@@ -28,6 +29,7 @@ int run_graphed(const std::vector<uint64_t>& key, bool want_status,
                 const std::function<int(cudaStream_t, int*)>& enqueue, cudaStream_t stream,
                 int** status_out);
 int cuda_fail(cudaError_t e);          // stores the message, returns GPTQ_ERR_CUDA
+int cuda_fail_msg(const char* where, cudaError_t e);   // same, naming the failing step
 int* device_status_ptr();              // status word of the current device (device memory)
 int sm_count();                        // SMs of the current device
 

@@ -214,3 +214,26 @@ def random_layer(seed: int, d_out: int, d_in: int, n_tokens: int, *, correlated:
         m += np.eye(d_in, dtype=np.float32)
         z = z @ m
     return w, f32_to_bf16_bits(z)
+
+
+def w4a16_operands(seed: int, M: int, N: int, K: int, group_size: int, *, act_order: bool = False):
+    """Seeded operands of the 4-bit linear: X bf16 bits [M, K] (the q_proj
+    activation recipe: N(0, 1) with 1% of the channels scaled lognormally),
+    packed codes uint8 [N, K/2] (uniform random bytes = uniform 4-bit codes),
+    float32 scales [N, n_groups] around the size a 0.02-std weight row gives
+    at 4 bits (lognormal, median 0.008), integer zeros uniform in 0..15, and
+    with act_order a group map g_idx [K] that assigns each group's columns
+    to random positions (as the act_order permutation does)."""
+    g = _rng(seed, 4016, M, N, K, max(group_size, 0))
+    ng = K // group_size if group_size > 0 else 1
+    x = g.standard_normal((M, K)).astype(np.float32)
+    ch = g.choice(K, size=max(1, K // 100), replace=False)
+    x[:, ch] *= np.exp(g.normal(1.5, 0.5, size=ch.size)).astype(np.float32)
+    packed = g.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = (0.008 * np.exp(g.normal(0.0, 0.3, size=(N, ng)))).astype(np.float32)
+    zeros = g.integers(0, 16, size=(N, ng)).astype(np.float32)
+    g_idx = None
+    if act_order:
+        gs = group_size if group_size > 0 else K
+        g_idx = g.permutation(np.arange(K) // gs).astype(np.int32)
+    return f32_to_bf16_bits(x), packed, scales, zeros, g_idx

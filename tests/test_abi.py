@@ -97,3 +97,28 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.gptq_selftest_bounded_wait(1 << 40) == 1
     assert lib.gptq_selftest_quotient(0, 0, fake) == 1
     assert lib.gptq_selftest_quotient(16, 0, None) == 1
+
+
+def test_w4a16_arguments_rejected_on_host(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+
+    def w(M=4, N=64, K=256, gs=128, path=0, X=fake, packed=fake, g_idx=None, Y=fake):
+        return lib.gptq_w4a16_gemm(Y, X, packed, fake, fake, g_idx, M, N, K, gs, path, None)
+    assert w(K=250) == 1             # K not a multiple of 8
+    assert w(K=0) == 1
+    assert w(M=-1) == 1
+    assert w(gs=100) == 1            # does not divide K
+    assert w(gs=0) == 1
+    assert w(path=3) == 1
+    assert w(X=None) == 1
+    assert w(Y=None) == 1
+    assert w(X=P((1 << 20) + 2)) == 1       # X not 16-byte aligned
+    assert w(packed=P((1 << 20) + 8)) == 1  # packed rows not 16-byte aligned
+    # the tensor-core path refuses layouts it does not cover
+    assert w(path=1, g_idx=fake) == 1       # groups given per column
+    assert w(path=1, K=264, gs=-1) == 1     # K not a multiple of 32
+    assert w(path=1, K=192, gs=48) == 1     # group neither divides nor is a multiple of 128
+    # empty products are done without a device
+    assert w(M=0) == 0
+    assert w(N=0) == 0
