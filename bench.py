@@ -3,6 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload q_proj_4096]
                     [--impl ours|reference] [--no-cpu-baseline]
 
+--workload decoder_layer times the layer-sequential calibration of a whole
+decoder layer; --workload w4a16 times the product of bf16 activations with the
+packed 4-bit output (the inference-side consumer of the format).
+
 One step = the whole per-layer path on one synthetic layer: Hessian over all
 calibration tokens (H = 2 X^T X), damping + Cholesky factor of the inverse,
 the blocked GPTQ column loop with lazy-batch updates, unpermute and int4
@@ -297,6 +301,83 @@ def run_decoder_layer(args, rank) -> int:
     return 0
 
 
+W4A16_SHAPES = (("qkv", 12288, 4096), ("o", 4096, 4096), ("gate_up", 22016, 4096), ("down", 4096, 11008))
+
+
+def run_w4a16(args, rank) -> int:
+    """The inference-side consumer of the packed output: one decode step of a
+    Llama-2-7B-shaped model's linears (per layer q/k/v fused, o, gate/up
+    fused, down; 4-bit codes, group 128) through gptq_w4a16_gemm, over L
+    distinct layers whose weights (about 0.46 GB) do not fit in L2.  The
+    4 L launches of a step are replayed from a CUDA graph.  value = weight
+    bytes streamed per second (codes + scales + zeros); the roofline is HBM."""
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    from post_weight_quantization_accumulate_b200 import binding as B
+    from post_weight_quantization_accumulate_b200 import build as build_mod
+    from post_weight_quantization_accumulate_b200 import synth
+
+    build_mod.build()
+    torch.cuda.set_device(0)
+    L, gs = 4, 128
+    peaks, src = measured_peaks()
+    out = {"metric": "W4A16 decode: packed-weight bytes streamed per second (Llama-2-7B linears)",
+           "unit": "GB/s", "n_gpus": 1, "higher_is_better": True, "dtype": "bf16 x int4 -> f32",
+           "data": "synthetic", "steps": max(args.steps, 400), "warmup": max(3, args.warmup),
+           "config": {"workload": "w4a16_llama2_7b_decode", "layers": L, "group_size": gs,
+                      "shapes": [list(x) for x in W4A16_SHAPES], "l2": "weights > L2 (0.46 GB)"}}
+    lines = {}
+    for M in (1, 16):
+        for path, pname in ((B.W4A16_TENSOR_CORE, "tensor_core"), (B.W4A16_GENERAL, "general")):
+            ops, wbytes = [], 0
+            for name, N, K in W4A16_SHAPES:
+                x, p, sc, z, _ = synth.w4a16_operands(11, M, N, K, gs)
+                X = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+                P0, S0, Z0 = (torch.from_numpy(a).cuda() for a in (p, sc, z))
+                for _ in range(L):
+                    Y = torch.empty(M, N, device="cuda")
+                    ops.append((Y, X, P0.clone(), S0.clone(), Z0.clone()))
+                    wbytes += P0.numel() + 4 * (S0.numel() + Z0.numel())
+                del P0, S0, Z0
+            for o in ops[:4]:
+                B.gptq_w4a16_gemm(*o, None, gs, path)
+            torch.cuda.synchronize()
+            n0 = B.gptq_launch_count()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for o in ops:
+                    B.gptq_w4a16_gemm(*o, None, gs, path)
+            launches = B.gptq_launch_count() - n0
+            for _ in range(max(3, args.warmup)):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(args.steps, 400)    # long enough for the 100 ms clock samples
+            with ClockSampler(0) as clk:
+                e0.record()
+                for _ in range(reps):
+                    g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            assert B.gptq_device_status() == 0
+            gbs = wbytes / (ms / 1e3) / 1e9
+            lines[f"M{M}_{pname}"] = {"ms_per_step": ms, "gbs": gbs, "tokens_per_s": M / (ms / 1e3),
+                                      "weight_bytes": wbytes, "launches_per_step": launches,
+                                      "frac_of_hbm": gbs / peaks["hbm_gbs"], "clocks": clk.summary()}
+            del g, ops
+            torch.cuda.empty_cache()
+    head = lines["M1_tensor_core"]
+    out.update({"value": head["gbs"], "ms_per_step": head["ms_per_step"], "gpu_launches": head["launches_per_step"] * max(args.steps, 400),
+                "roofline": {"bound": "hbm", "achieved": head["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": head["frac_of_hbm"], "peak_source": src, "traffic": None},
+                "clocks": head["clocks"], "vs_baseline": None, "by_case": lines})
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -306,6 +387,8 @@ def main():
         return run_reference(args, rank, world)
     if args.workload == "decoder_layer":
         return run_decoder_layer(args, rank)
+    if args.workload == "w4a16":
+        return run_w4a16(args, rank)
 
     import numpy as np
     import torch

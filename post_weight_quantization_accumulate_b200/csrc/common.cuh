@@ -97,15 +97,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 
 // Waits for the phase of `bar` with the given parity.  Gives up when *abort
 // becomes non-zero or after `limit` cycles; on a time-out it raises *abort
-// and records GPTQ_ERR_TIMEOUT.  Returns false when it gave up.
+// and records GPTQ_ERR_TIMEOUT.  Returns false when it gave up.  The abort
+// flag and the clock are read once per 32 polls of the barrier: waiting warps
+// share the SM's issue slots and load/store queues with the working ones.
+// With sleep_ns > 0 the waiting warp sleeps that long between polls and
+// leaves its scheduler's issue slots to the warps that have work.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, int* status,
-                                                  long long limit = kWaitLimitCycles)
+                                                  long long limit = kWaitLimitCycles,
+                                                  unsigned sleep_ns = 0)
 {
     if (mbar_try_wait(bar, parity)) return true;
     long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i) {
+            if (mbar_try_wait(bar, parity)) return true;
+            if (sleep_ns) __nanosleep(sleep_ns);
+        }
         if (*abort) return false;
         if (clock64() - t0 > limit) {
             *abort = 1;
@@ -113,6 +122,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
             return false;
         }
     }
+}
+
+// mbar_wait_bounded for a whole warp (all 32 lanes call it): lane 0 polls and
+// the others wait at the warp barrier, which also orders what lane 0 observed
+// before their own accesses.  Polls from every lane of many waiting warps
+// fill the SM's shared-memory pipe that the working warps' loads, special-
+// function and tcgen05 instructions go through as well.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               int* status, long long limit = kWaitLimitCycles,
+                                               unsigned sleep_ns = 0)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait_bounded(bar, parity, abort, status, limit, sleep_ns) ? 1 : 0;
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // 2-D tiled TMA load into shared memory, completing on `bar` (tx bytes).

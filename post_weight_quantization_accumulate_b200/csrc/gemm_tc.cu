@@ -158,8 +158,12 @@ template <int TN, bool PRELO>
 __global__ void __launch_bounds__(TTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const __grid_constant__ CUtensorMap mapAlo, const __grid_constant__ CUtensorMap mapBlo,
-                   const __grid_constant__ CUtensorMap mapC, const GemmArgs g)
+                   const __grid_constant__ CUtensorMap mapC, const GemmArgs g_param)
 {
+    // a register copy of the arguments: the parameter struct itself, reached
+    // through a reference, would be reloaded with generic loads after every
+    // asm statement with a memory clobber inside the loops
+    const GemmArgs g = g_param;
     using Cfg = GemmCfg<TN, PRELO>;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int B_BYTES = Cfg::B_BYTES;

@@ -18,8 +18,9 @@
 // 16-bit rounding of s (q - z)), differing only in the order of the fp32
 // additions.
 //   * A tile is 128 weight rows (the MMA's M) by a K range.  Stages of 128
-//     columns: TMA brings the packed bytes (128 x 64 B), the X tile (M padded
-//     to NP rows, 128B-swizzled) and cp.async the stage's scales and zeros.
+//     columns: TMA brings the packed bytes (128 x 64 B) and the X tile (M
+//     padded to NP rows, 128B-swizzled).  Each converter thread reads its own
+//     row's zero and scale through L1 (one 32-byte sector serves 8 groups).
 //   * Eight converter warps turn a row's nibbles into bf16 pairs (128 + q
 //     from the exponent trick, minus 128 + z) and store them with
 //     tcgen05.st straight into tensor memory, which is the MMA's A operand:
@@ -124,13 +125,22 @@ __global__ void __launch_bounds__(kWThreads)
 // ------------------------------------------------------- tensor-core path
 constexpr int kRows = 128;          // weight rows per tile = MMA M
 constexpr int kStageCols = 128;     // K columns per stage
-constexpr int kStages = 4;
+constexpr int kMaxStages = 6;
+// pipeline depth per accumulator width: two CTAs fit on an SM for NP <= 32
+template <int NP>
+__host__ __device__ constexpr int stages_for()
+{
+    return NP <= 16 ? 6 : (NP <= 32 ? 5 : 4);
+}
 constexpr int kTcThreads = 320;     // warp 0 loads, warp 1 issues MMAs, 2..9 convert
 constexpr int kConvWarps = 8;
 constexpr int kTmemCols = 256;      // 2 A buffers of 64 columns + 128 accumulator columns
 constexpr int kAcols = 64;          // TMEM columns of one stage's A (128 bf16 per lane)
 constexpr int kWBytes = kRows * kStageCols / 2;   // packed bytes of a stage
 constexpr int kMinSmem = 78 * 1024;  // at most two CTAs per SM (TMEM holds two)
+// sleeps between polls of a barrier (ns): waiting warps give their issue slots
+// to the converters and to the MMA thread
+constexpr unsigned kSleepLoad = 200, kSleepMma = 20, kSleepConv = 60;
 
 struct TcArgs {
     float* Y;
@@ -140,15 +150,15 @@ struct TcArgs {
     int M, N, K;
     int m0;       // first X row of this pass
     int gs;       // group length along K (K for one group per row)
+    int gs_shift; // log2(gs) when gs is a power of two, else -1
     int ng;       // row length of scales / zeros
-    int gps;      // group slots per stage in shared memory
     int stage_bytes;
     int splits;   // CTAs along K (the cluster)
 };
 
 struct TcShared {
-    uint64_t full[kStages];     // TMA bytes + 32 cp.async arrivals + 1
-    uint64_t empty[kStages];    // MMA commit + 8 converter warps (after the epilogue)
+    uint64_t full[kMaxStages];  // TMA bytes
+    uint64_t empty[kMaxStages]; // MMA commit
     uint64_t a_full[2];         // 8 converter warps
     uint64_t a_empty[2];        // MMA commit
     uint64_t slot_full[8];      // MMA commit after a group's last K step
@@ -194,28 +204,14 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
-
-// Arrives on `bar` when the calling thread's earlier cp.async copies land
-// (counted as one of the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all()
-{
-    asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
 __device__ __forceinline__ void fence_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* p)
+{
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ uint32_t cta_rank_in_cluster()
@@ -255,6 +251,12 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zz, uint32_t* 
     for (int i = 0; i < 4; ++i) out[i] = bf16x2_sub(((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u, zz);
 }
 
+// Group of column c (a shift when the group length is a power of two).
+__device__ __forceinline__ int group_of(int c, int gs, int gs_shift)
+{
+    return gs_shift >= 0 ? c >> gs_shift : c / gs;
+}
+
 // Column range and groups of stage `t` (local index) of a CTA whose K range
 // is [kb, ke).
 struct StageGroups {
@@ -263,14 +265,14 @@ struct StageGroups {
     int fin;         // groups that end inside the stage (the first `fin` of them)
 };
 
-__device__ __forceinline__ StageGroups stage_groups(int t, int kb, int ke, int gs)
+__device__ __forceinline__ StageGroups stage_groups(int t, int kb, int ke, int gs, int gs_shift)
 {
     StageGroups r;
     r.c0 = kb + t * kStageCols;
     r.ce = min(r.c0 + kStageCols, ke);
-    r.g0 = r.c0 / gs;
+    r.g0 = group_of(r.c0, gs, gs_shift);
     if (gs <= kStageCols) {   // gs divides the stage width: every group ends inside
-        r.count = (r.ce - r.c0 + gs - 1) / gs;
+        r.count = group_of(r.ce - r.c0 + gs - 1, gs, gs_shift);
         r.fin = r.count;
     } else {                  // one group spans the stage
         r.count = 1;
@@ -285,42 +287,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const TcArgs a)
 {
     constexpr int R = 128 / NP;                 // accumulator slots
+    constexpr int kStages = stages_for<NP>();
     constexpr int XBOX = NP * 128;              // bytes of one 64-column X box
     constexpr int XBYTES = 2 * XBOX;
     constexpr uint32_t kIdesc = idesc_f32acc(1 /*bf16*/, 0, 0, kRows, NP);
+    // the arguments as scalars: the kernel never reads the parameter struct
+    // through a reference, which after each asm statement with a memory
+    // clobber would be reloaded with generic loads inside the loops
+    const int K = a.K, N = a.N, M = a.M, m0 = a.m0, gs = a.gs, gs_shift = a.gs_shift;
+    const int ng = a.ng, splits = a.splits, stage_bytes = a.stage_bytes;
+    float* const Yout = a.Y;
+    const float* const scales = a.scales;
+    const float* const zeros = a.zeros;
+    int* const status = a.status;
     __shared__ TcShared S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    // stage layout: X tile (1024-aligned) | packed weights | scales | zeros
-    auto xs = [&](int s) { return base + s * a.stage_bytes; };
-    auto ws = [&](int s) { return base + s * a.stage_bytes + XBYTES; };
-    auto sc = [&](int s) {
-        return reinterpret_cast<float*>(base + s * a.stage_bytes + XBYTES + kWBytes);
-    };
-    auto zr = [&](int s) {
-        return reinterpret_cast<float*>(base + s * a.stage_bytes + XBYTES + kWBytes) +
-               a.gps * kRows;
-    };
-    float* red = reinterpret_cast<float*>(base + kStages * a.stage_bytes);   // [NP][128]
+    // stage layout: X tile (1024-aligned) | packed weights
+    auto xs = [base, stage_bytes](int s) { return base + s * stage_bytes; };
+    auto ws = [base, stage_bytes](int s) { return base + s * stage_bytes + XBYTES; };
+    float* red = reinterpret_cast<float*>(base + kStages * stage_bytes);   // [NP][128]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cta_rank_in_cluster();
     const int n0 = blockIdx.y * kRows;
     // this CTA's stages of the K range
-    const int T = (a.K + kStageCols - 1) / kStageCols;
-    const int t_begin = static_cast<int>((static_cast<int64_t>(T) * rank) / a.splits);
-    const int t_end = static_cast<int>((static_cast<int64_t>(T) * (rank + 1)) / a.splits);
+    const int T = (K + kStageCols - 1) / kStageCols;
+    const int t_begin = static_cast<int>((static_cast<int64_t>(T) * rank) / splits);
+    const int t_end = static_cast<int>((static_cast<int64_t>(T) * (rank + 1)) / splits);
     const int nt = t_end - t_begin;
     const int kb = t_begin * kStageCols;
-    const int ke = min(t_end * kStageCols, a.K);
-    const int g_first = kb / a.gs;
+    const int ke = min(t_end * kStageCols, K);
+    const int g_first = group_of(kb, gs, gs_shift);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&S.full[s], 33);
-            mbar_init(&S.empty[s], 1 + kConvWarps);
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&S.a_full[b], kConvWarps);
@@ -345,47 +350,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tA = S.tmem_base;              // A buffers: columns 0..127
     const uint32_t tAcc = S.tmem_base + 2 * kAcols;   // accumulator slots: 128..255
     volatile int* abort = &S.abort;
-    int* status = a.status;
     float y[NP / 2];
 #pragma unroll
     for (int j = 0; j < NP / 2; ++j) y[j] = 0.f;
 
     if (warp == 0) {
-        // ---- loads: TMA (lane 0) for X and the packed weights, cp.async (all
-        // lanes) for the stage's scales and zeros
-        int issued = 0;
-        for (int t = 0; t < nt; ++t) {
-            const int s = t % kStages;
-            const uint32_t ph = (t / kStages) & 1;
-            const bool got = mbar_wait_bounded(&S.empty[s], ph ^ 1, abort, status);
-            if (!__all_sync(0xffffffffu, got)) break;
-            const StageGroups sg = stage_groups(t, kb, ke, a.gs);
-            if (lane == 0) {
+        // ---- loads: TMA for X and the packed weights
+        if (lane == 0) {
+            int issued = 0;
+            for (int t = 0; t < nt; ++t) {
+                const int s = t % kStages;
+                if (!mbar_wait_bounded(&S.empty[s], ((t / kStages) & 1) ^ 1, abort, status, kWaitLimitCycles, kSleepLoad)) break;
+                const int c0 = kb + t * kStageCols;
                 mbar_arrive_expect_tx(&S.full[s], XBYTES + kWBytes);
-                tma_load_2d(xs(s), &mapX, &S.full[s], sg.c0, a.m0);
-                tma_load_2d(xs(s) + XBOX, &mapX, &S.full[s], sg.c0 + 64, a.m0);
-                tma_load_2d(ws(s), &mapW, &S.full[s], sg.c0 / 2, n0);
+                tma_load_2d(xs(s), &mapX, &S.full[s], c0, m0);
+                tma_load_2d(xs(s) + XBOX, &mapX, &S.full[s], c0 + 64, m0);
+                tma_load_2d(ws(s), &mapW, &S.full[s], c0 / 2, n0);
+                ++issued;
             }
-            const int items = sg.count * kRows;
-            for (int i = lane; i < 2 * items; i += 32) {
-                const int arr = i >= items;
-                const int rem = arr ? i - items : i;
-                const int gi = rem / kRows, r = rem % kRows;
-                if (n0 + r < a.N) {
-                    const int64_t off = static_cast<int64_t>(n0 + r) * a.ng + sg.g0 + gi;
-                    cp_async_4((arr ? zr(s) : sc(s)) + gi * kRows + r, (arr ? a.zeros : a.scales) + off);
-                }
+            // after a time-out, let the copies already issued land before the
+            // CTA's shared memory goes away
+            if (*abort) {
+                for (int t = max(0, issued - kStages); t < issued; ++t)
+                    mbar_wait_bounded(&S.full[t % kStages], (t / kStages) & 1, abort, nullptr,
+                                      kWaitLimitCycles / 16);
             }
-            cp_async_arrive(&S.full[s]);
-            ++issued;
-        }
-        cp_async_wait_all();
-        // after a time-out, let the copies already issued land before the
-        // CTA's shared memory goes away
-        if (*abort && lane == 0) {
-            for (int t = max(0, issued - kStages); t < issued; ++t)
-                mbar_wait_bounded(&S.full[t % kStages], (t / kStages) & 1, abort, nullptr,
-                                  kWaitLimitCycles / 16);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -395,20 +384,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int t = 0; t < nt && ok; ++t) {
                 const int s = t % kStages;
                 const int b = t & 1;
-                if (!mbar_wait_bounded(&S.a_full[b], (t >> 1) & 1, abort, status)) break;
+                if (!mbar_wait_bounded(&S.a_full[b], (t >> 1) & 1, abort, status, kWaitLimitCycles, kSleepMma)) break;
                 tc_fence_after();
-                const StageGroups sg = stage_groups(t, kb, ke, a.gs);
+                const StageGroups sg = stage_groups(t, kb, ke, gs, gs_shift);
                 const uint32_t xaddr = smem_u32(xs(s));
 #pragma unroll 1
                 for (int j = 0; j < kStageCols / 16; ++j) {
                     const int c = sg.c0 + 16 * j;
                     if (c >= sg.ce) break;
-                    const int g = c / a.gs;
+                    const int g = group_of(c, gs, gs_shift);
                     const int u = g - g_first;
                     const int slot = u % R;
-                    const bool first = c == max(g * a.gs, kb);
+                    const bool first = c == max(g * gs, kb);
                     if (first && u >= R) {
-                        if (!mbar_wait_bounded(&S.slot_empty[slot], ((u / R) - 1) & 1, abort, status)) {
+                        if (!mbar_wait_bounded(&S.slot_empty[slot], ((u / R) - 1) & 1, abort, status, kWaitLimitCycles, kSleepMma)) {
                             ok = false;
                             break;
                         }
@@ -418,7 +407,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         sdesc_sw128(xaddr + (j >> 2) * XBOX + (j & 3) * 32, 16, 1024);
                     umma_f16_ts(tAcc + slot * NP, tA + b * kAcols + 8 * j, bdesc, kIdesc,
                                 first ? 0u : 1u);
-                    if (c + 16 == min((g + 1) * a.gs, ke)) umma_commit(&S.slot_full[slot]);
+                    if (c + 16 == min((g + 1) * gs, ke)) umma_commit(&S.slot_full[slot]);
                 }
                 if (!ok) break;
                 umma_commit(&S.a_empty[b]);
@@ -435,18 +424,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int rl = q * 32 + lane;                  // tile row
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
         const int ct = threadIdx.x - 64;               // 0..255
+        // this row's scales and zeros (rows past N read row N - 1; unused)
+        const int64_t roff = static_cast<int64_t>(min(n0 + rl, N - 1)) * ng;
+        const float* srow = scales + roff;
+        const float* zrow = zeros + roff;
 
         // epilogue of the groups that end in stage tp (local index)
         auto drain = [&](int tp) -> bool {
-            const StageGroups sg = stage_groups(tp, kb, ke, a.gs);
-            const float* scl = sc(tp % kStages);
+            const StageGroups sg = stage_groups(tp, kb, ke, gs, gs_shift);
             for (int gi = 0; gi < sg.fin; ++gi) {
                 const int u = sg.g0 + gi - g_first;
                 const int slot = u % R;
-                const bool got = mbar_wait_bounded(&S.slot_full[slot], (u / R) & 1, abort, status);
-                if (!__all_sync(0xffffffffu, got)) return false;
+                if (!mbar_wait_warp(&S.slot_full[slot], (u / R) & 1, abort, status, kWaitLimitCycles, kSleepConv)) return false;
                 tc_fence_after();
-                const float sv = scl[gi * kRows + rl];
+                const float sv = __ldg(srow + sg.g0 + gi);
 #pragma unroll
                 for (int c8 = 0; c8 < NP / 16; ++c8) {
                     float v[8];
@@ -459,20 +450,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.slot_empty[slot]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.empty[tp % kStages]);
             return true;
         };
 
         bool ok = true;
+        prefetch_l1(zrow + g_first);
+        prefetch_l1(srow + g_first);
         for (int t = 0; t < nt; ++t) {
             const int s = t % kStages;
             const int b = t & 1;
-            bool got = mbar_wait_bounded(&S.full[s], (t / kStages) & 1, abort, status);
-            if (got && t >= 2) got = mbar_wait_bounded(&S.a_empty[b], ((t >> 1) - 1) & 1, abort, status);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            {   // the next stage's zero and scale, into L1 ahead of use
+                const int gn = min(group_of(kb + (t + 1) * kStageCols, gs, gs_shift), ng - 1);
+                prefetch_l1(zrow + gn);
+                prefetch_l1(srow + gn);
+            }
+            bool got = mbar_wait_warp(&S.full[s], (t / kStages) & 1, abort, status, kWaitLimitCycles, kSleepConv);
+            if (got && t >= 2) got = mbar_wait_warp(&S.a_empty[b], ((t >> 1) - 1) & 1, abort, status, kWaitLimitCycles, kSleepConv);
+            if (!got) { ok = false; break; }
             tc_fence_after();
-            const StageGroups sg = stage_groups(t, kb, ke, a.gs);
+            const StageGroups sg = stage_groups(t, kb, ke, gs, gs_shift);
             // X tile: within each 16-byte chunk (8 columns) order the columns
             // (0, 4, 1, 5, 2, 6, 3, 7) like the converted weight pairs
             uint4* xc = reinterpret_cast<uint4*>(xs(s));
@@ -495,14 +491,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint4 r1 = *reinterpret_cast<const uint4*>(wrow + 16 * (rot ^ 1));
             const uint4 wv0 = rot ? r1 : r0;
             const uint4 wv1 = rot ? r0 : r1;
-            const float* zrs = zr(s);
+            int gz = -1;
+            float zf = 0.f;
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const int j = 4 * h + jj;
                 const int c = sg.c0 + 16 * j;
                 if (c >= sg.ce) break;   // warp-uniform
-                const int gi = c / a.gs - sg.g0;
-                const float zf = 128.f + zrs[gi * kRows + rl];
+                const int g = group_of(c, gs, gs_shift);
+                if (g != gz) {           // warp-uniform
+                    zf = 128.f + __ldg(zrow + g);
+                    gz = g;
+                }
                 const uint32_t zb = __float_as_uint(zf) >> 16;   // exact: 128 + z, z in 0..15
                 const uint32_t zz = zb | (zb << 16);
                 const uint32_t w0 = jj < 2 ? (jj == 0 ? wv0.x : wv0.z) : (jj == 2 ? wv1.x : wv1.z);
@@ -528,16 +528,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     cluster_barrier();
     {
-        const int mv = min(NP, a.M - a.m0);
+        const int mv = min(NP, M - m0);
         const int E = mv * kRows;
-        const int e0 = static_cast<int>((static_cast<int64_t>(E) * rank) / a.splits);
-        const int e1 = static_cast<int>((static_cast<int64_t>(E) * (rank + 1)) / a.splits);
+        const int e0 = static_cast<int>((static_cast<int64_t>(E) * rank) / splits);
+        const int e1 = static_cast<int>((static_cast<int64_t>(E) * (rank + 1)) / splits);
         for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kTcThreads) {
             const int m = e / kRows, r = e % kRows;
-            if (n0 + r >= a.N) continue;
+            if (n0 + r >= N) continue;
             float v = 0.f;
-            for (int p = 0; p < a.splits; ++p) v += ld_cluster_f32(red + e, static_cast<uint32_t>(p));
-            a.Y[static_cast<int64_t>(a.m0 + m) * a.N + n0 + r] = v;
+            for (int p = 0; p < splits; ++p) v += ld_cluster_f32(red + e, static_cast<uint32_t>(p));
+            Yout[static_cast<int64_t>(m0 + m) * N + n0 + r] = v;
         }
     }
     cluster_barrier();
@@ -589,9 +589,8 @@ template <int NP>
 int launch_tc(float* Y, const uint16_t* X, const uint8_t* packed, const float* scales,
               const float* zeros, int M, int N, int K, int gs_e, int ng, cudaStream_t stream)
 {
-    const int gps = gs_e <= kStageCols ? kStageCols / gs_e : 1;
-    const int stage_bytes = 2 * NP * 128 + kWBytes + ((2 * gps * kRows * 4 + 1023) / 1024) * 1024;
-    const int smem = std::max(1024 + kStages * stage_bytes + NP * kRows * 4, kMinSmem);
+    const int stage_bytes = 2 * NP * 128 + kWBytes;
+    const int smem = std::max(1024 + stages_for<NP>() * stage_bytes + NP * kRows * 4, kMinSmem);
     // the opt-in limit is raised to what this call needs (once per size and device)
     static int attr_bytes[64] = {};
     int dev = 0;
@@ -612,7 +611,8 @@ int launch_tc(float* Y, const uint16_t* X, const uint8_t* packed, const float* s
 
     const int tiles = (N + kRows - 1) / kRows;
     const int T = (K + kStageCols - 1) / kStageCols;
-    const int per_sm = smem * 2 + 2 * static_cast<int>(sizeof(TcShared)) <= 228 * 1024 ? 2 : 1;
+    // two CTAs per SM when both fit (each also holds 1 KB the system reserves)
+    const int per_sm = 2 * (smem + static_cast<int>(sizeof(TcShared)) + 1024) <= 228 * 1024 ? 2 : 1;
     int splits = (per_sm * sm_count()) / tiles;
     splits = std::max(1, std::min({splits, 8, T}));
 
@@ -625,8 +625,8 @@ int launch_tc(float* Y, const uint16_t* X, const uint8_t* packed, const float* s
     args.N = N;
     args.K = K;
     args.gs = gs_e;
+    args.gs_shift = (gs_e & (gs_e - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(gs_e)) : -1;
     args.ng = ng;
-    args.gps = gps;
     args.stage_bytes = stage_bytes;
     args.splits = splits;
 

@@ -2,6 +2,8 @@
 
     python -m post_weight_quantization_accumulate_b200.kernel_case \
         --call hessian|prepare|quantize|layer --workload q_proj_4096 [--tokens N] [--reps R]
+    python -m post_weight_quantization_accumulate_b200.kernel_case \
+        --call w4a16 [--m M] [--n N] [--k K] [--group-size G] [--path 0|1|2] [--reps R]
 
 The inputs follow the workload's recipe (see synth.py) with `--tokens`
 overriding the calibration size, so a profiler can capture a launch on a case
@@ -58,16 +60,46 @@ def tf32_peak(n: int = 8192, seconds: float = 3.0):
     print(f"(n = {n}, {reps} products in the sustained loop)")
 
 
+def w4a16_case(a):
+    """gptq_w4a16_gemm on seeded operands; a 256 MB buffer is rewritten before
+    every call so that the weights come from HBM, not L2."""
+    dev = torch.device("cuda", 0)
+    x, p, sc, z, _ = synth.w4a16_operands(7, a.m, a.n, a.k, a.group_size)
+    X = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    P, S, Z = (torch.from_numpy(t).to(dev) for t in (p, sc, z))
+    Y = torch.empty(a.m, a.n, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ms = []
+    for _ in range(a.reps + 1):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.gptq_w4a16_gemm(Y, X, P, S, Z, None, a.group_size, a.path)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    print(f"w4a16 M={a.m} N={a.n} K={a.k} g={a.group_size} path={a.path}: "
+          f"{min(ms[1:]) * 1e3:.1f} us/call (cold L2, single launch), status {B.gptq_device_status()}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--call", default="hessian",
-                    choices=["hessian", "prepare", "quantize", "layer", "tf32_peak"])
+                    choices=["hessian", "prepare", "quantize", "layer", "tf32_peak", "w4a16"])
     ap.add_argument("--workload", default="q_proj_4096")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--m", type=int, default=1)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--group-size", type=int, default=128)
+    ap.add_argument("--path", type=int, default=0)
     a = ap.parse_args()
     if a.call == "tf32_peak":
         tf32_peak()
+        return
+    if a.call == "w4a16":
+        w4a16_case(a)
         return
     spec = synth.WORKLOADS[a.workload]
     if a.tokens:
