@@ -387,27 +387,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!mbar_wait_bounded(&S.a_full[b], (t >> 1) & 1, abort, status, kWaitLimitCycles, kSleepMma)) break;
                 tc_fence_after();
                 const StageGroups sg = stage_groups(t, kb, ke, gs, gs_shift);
-                const uint32_t xaddr = smem_u32(xs(s));
-#pragma unroll 1
-                for (int j = 0; j < kStageCols / 16; ++j) {
-                    const int c = sg.c0 + 16 * j;
-                    if (c >= sg.ce) break;
-                    const int g = group_of(c, gs, gs_shift);
+                const int nk = (sg.ce - sg.c0) >> 4;              // K steps in the stage
+                // B descriptor of K step 0; step j starts (j / 4) boxes and
+                // (j % 4) * 32 bytes further (address field in 16-byte units)
+                const uint64_t bdesc0 = sdesc_sw128(smem_u32(xs(s)), 16, 1024);
+                const uint32_t a0 = tA + b * kAcols;
+                int j = 0;
+                // the groups touching the stage, in order; per K step only the
+                // MMA itself is issued
+                for (int gi = 0; gi < sg.count && ok; ++gi) {
+                    const int g = sg.g0 + gi;
+                    const int gstart = max(g * gs, kb);        // group's first column in this CTA
+                    const int gend = min((g + 1) * gs, ke);
+                    const int j1 = min(nk, (gend - sg.c0) >> 4);
                     const int u = g - g_first;
                     const int slot = u % R;
-                    const bool first = c == max(g * gs, kb);
-                    if (first && u >= R) {
-                        if (!mbar_wait_bounded(&S.slot_empty[slot], ((u / R) - 1) & 1, abort, status, kWaitLimitCycles, kSleepMma)) {
+                    const int jfirst = gstart >= sg.c0 ? (gstart - sg.c0) >> 4 : -1;
+                    if (jfirst >= 0 && u >= R) {
+                        if (!mbar_wait_bounded(&S.slot_empty[slot], ((u / R) - 1) & 1, abort, status,
+                                               kWaitLimitCycles, kSleepMma)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                     }
-                    const uint64_t bdesc =
-                        sdesc_sw128(xaddr + (j >> 2) * XBOX + (j & 3) * 32, 16, 1024);
-                    umma_f16_ts(tAcc + slot * NP, tA + b * kAcols + 8 * j, bdesc, kIdesc,
-                                first ? 0u : 1u);
-                    if (c + 16 == min((g + 1) * gs, ke)) umma_commit(&S.slot_full[slot]);
+                    const uint32_t d = tAcc + slot * NP;
+                    if (j == 0 && j1 == kStageCols / 16) {
+                        // a whole stage inside one group: eight MMAs, straight line
+#pragma unroll
+                        for (int jj = 0; jj < kStageCols / 16; ++jj)
+                            umma_f16_ts(d, a0 + 8 * jj,
+                                        bdesc0 + static_cast<uint64_t>(((jj >> 2) * XBOX + (jj & 3) * 32) >> 4),
+                                        kIdesc, jj == jfirst ? 0u : 1u);
+                        j = j1;
+                    }
+#pragma unroll 1
+                    for (; j < j1; ++j) {
+                        const uint64_t bdesc =
+                            bdesc0 + static_cast<uint64_t>(((j >> 2) * XBOX + (j & 3) * 32) >> 4);
+                        umma_f16_ts(d, a0 + 8 * j, bdesc, kIdesc, j == jfirst ? 0u : 1u);
+                    }
+                    if (gend <= sg.ce) umma_commit(&S.slot_full[slot]);
                 }
                 if (!ok) break;
                 umma_commit(&S.a_empty[b]);
@@ -491,26 +511,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint4 r1 = *reinterpret_cast<const uint4*>(wrow + 16 * (rot ^ 1));
             const uint4 wv0 = rot ? r1 : r0;
             const uint4 wv1 = rot ? r0 : r1;
-            int gz = -1;
-            float zf = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = 4 * h + jj;
-                const int c = sg.c0 + 16 * j;
-                if (c >= sg.ce) break;   // warp-uniform
-                const int g = group_of(c, gs, gs_shift);
-                if (g != gz) {           // warp-uniform
-                    zf = 128.f + __ldg(zrow + g);
-                    gz = g;
-                }
+            // this warp's 64 columns lie in one group when the stage is whole
+            // and groups are at least 64 columns long: one zero, no checks
+            if (sg.ce - sg.c0 == kStageCols && gs >= 64) {
+                const float zf = 128.f + __ldg(zrow + group_of(sg.c0 + 64 * h, gs, gs_shift));
                 const uint32_t zb = __float_as_uint(zf) >> 16;   // exact: 128 + z, z in 0..15
                 const uint32_t zz = zb | (zb << 16);
-                const uint32_t w0 = jj < 2 ? (jj == 0 ? wv0.x : wv0.z) : (jj == 2 ? wv1.x : wv1.z);
-                const uint32_t w1 = jj < 2 ? (jj == 0 ? wv0.y : wv0.w) : (jj == 2 ? wv1.y : wv1.w);
-                uint32_t v[8];
-                dequant_word(w0, zz, v);
-                dequant_word(w1, zz, v + 4);
-                tmem_st_32x32b_x8(tA + lane_addr + b * kAcols + 8 * j, v);
+                const uint32_t wq[8] = {wv0.x, wv0.y, wv0.z, wv0.w, wv1.x, wv1.y, wv1.z, wv1.w};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t v[8];
+                    dequant_word(wq[2 * jj], zz, v);
+                    dequant_word(wq[2 * jj + 1], zz, v + 4);
+                    tmem_st_32x32b_x8(tA + lane_addr + b * kAcols + 8 * (4 * h + jj), v);
+                }
+            } else {
+                int gz = -1;
+                float zf = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = 4 * h + jj;
+                    const int c = sg.c0 + 16 * j;
+                    if (c >= sg.ce) break;   // warp-uniform
+                    const int g = group_of(c, gs, gs_shift);
+                    if (g != gz) {           // warp-uniform
+                        zf = 128.f + __ldg(zrow + g);
+                        gz = g;
+                    }
+                    const uint32_t zb = __float_as_uint(zf) >> 16;   // exact: 128 + z, z in 0..15
+                    const uint32_t zz = zb | (zb << 16);
+                    const uint32_t w0 = jj < 2 ? (jj == 0 ? wv0.x : wv0.z) : (jj == 2 ? wv1.x : wv1.z);
+                    const uint32_t w1 = jj < 2 ? (jj == 0 ? wv0.y : wv0.w) : (jj == 2 ? wv1.y : wv1.w);
+                    uint32_t v[8];
+                    dequant_word(w0, zz, v);
+                    dequant_word(w1, zz, v + 4);
+                    tmem_st_32x32b_x8(tA + lane_addr + b * kAcols + 8 * j, v);
+                }
             }
             tmem_st_wait();
             tc_fence_before();
