@@ -105,6 +105,21 @@ def hessian(x_bits: np.ndarray, H: np.ndarray | None = None) -> np.ndarray:
     return H
 
 
+def hessian_f32(x: np.ndarray, H: np.ndarray | None = None, chunk: int = 4096) -> np.ndarray:
+    """H (+)= 2 * sum_t x_t x_t^T for float32 activations X [n, d] (GPTQ
+    overview, "Złożoność obliczeniowa": H = 2 X X^T), in float64.  The binary32
+    values are widened exactly; the token sum is a float64 matrix product over
+    chunks of rows."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    n, d = x.shape
+    if H is None:
+        H = np.zeros((d, d), dtype=np.float64)
+    for t0 in range(0, n, chunk):
+        xc = x[t0:t0 + chunk].astype(np.float64)
+        H += 2.0 * (xc.T @ xc)
+    return H
+
+
 def hessian_block(x_bits: np.ndarray, rows, cols) -> np.ndarray:
     """Entries H[rows][:, cols] of 2 X^T X, each summed directly over tokens."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)

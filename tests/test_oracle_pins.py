@@ -410,3 +410,20 @@ def test_w4a16_matches_brute_force_sum():
             w = float(scales[n, gidx[k]]) * (float(codes[n, k]) - float(zeros[n, gidx[k]]))
             ref += x[m, k] * w
         assert abs(Y[m, n] - ref) <= 1e-12 * (1 + abs(ref))
+
+
+def test_hessian_f32_matches_brute_force_and_the_bf16_checker():
+    """fp32-activation Hessian: a literal triple loop on a tiny case, and on
+    bf16-representable values the independent bf16 checker (same exact sums)."""
+    g = np.random.default_rng(17)
+    x = g.standard_normal((9, 5)).astype(np.float32)
+    H = oracle.hessian_f32(x, chunk=4)
+    for i in range(5):
+        for j in range(5):
+            ref = 0.0
+            for t in range(9):
+                ref += 2.0 * float(x[t, i]) * float(x[t, j])
+            assert abs(H[i, j] - ref) <= 1e-12 * (1.0 + abs(ref))
+    xb = synth.f32_to_bf16_bits(g.standard_normal((300, 24)).astype(np.float32))
+    xf = synth.bf16_bits_to_f32(xb)
+    np.testing.assert_allclose(oracle.hessian_f32(xf, chunk=64), oracle.hessian(xb), rtol=1e-13, atol=0)
