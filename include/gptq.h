@@ -116,6 +116,32 @@ int gptq_hessian_accumulate_host(float *H, const uint16_t *X_host, int64_t n_tok
                                  int64_t d_in, uint16_t *staging, int64_t chunk_tokens,
                                  void *stream);
 
+/* Workspace bytes of gptq_hessian_accumulate_f32 for d_in and chunk_tokens
+ * (0 for invalid sizes): 16 d_in^2 + 4 chunk_tokens d_in, rounded up. */
+size_t gptq_hessian_f32_workspace_bytes(int64_t d_in, int64_t chunk_tokens);
+
+/*
+ * gptq_hessian_accumulate for float32 activations: H += 2 X^T X with X
+ * float32 [n_tokens, d_in] on the device.  Each value is split into two bf16
+ * parts, x = hi + lo + r with |r| <= 2^-18 |x|, and the bf16 tensor-core
+ * Hessian of [hi | lo] (n_tokens x 2 d_in) gives every term of (hi + lo)^T
+ * (hi + lo): products exact, sums in float32, so the result matches the
+ * float64 2 X^T X to about 1e-5 relative (four times the tensor work of the
+ * bf16 call).
+ *   H             float32 [d_in, d_in], IN/OUT, symmetric; stays bitwise
+ *                 symmetric.  16-byte aligned.
+ *   X             float32 [n_tokens, d_in], 16-byte aligned.
+ *   d_in          > 0, multiple of 8, <= 32768.
+ *   chunk_tokens  tokens per pass through the workspace, 1 .. 2^30.
+ *   workspace     >= gptq_hessian_f32_workspace_bytes(d_in, chunk_tokens)
+ *                 bytes of device memory, 256-byte aligned, not used by
+ *                 anything else until `stream` has finished this call.
+ * Stream-ordered.  GPTQ_ERR_WORKSPACE when the workspace is missing or small.
+ */
+int gptq_hessian_accumulate_f32(float *H, const float *X, int64_t n_tokens, int64_t d_in,
+                                int64_t chunk_tokens, void *workspace, size_t ws_bytes,
+                                void *stream);
+
 /*
  * Damping, activation order and the Cholesky factor of the inverse Hessian
  * ("Hiperparametry": value added to the diagonal, quantizing columns in order

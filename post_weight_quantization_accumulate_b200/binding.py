@@ -34,6 +34,8 @@ SIGNATURES = [
     ("gptq_workspace_min_bytes", _SZ, [_I64, _I64, _I]),
     ("gptq_hessian_accumulate", _I, [_P, _P, _I64, _I64, _P]),
     ("gptq_hessian_accumulate_host", _I, [_P, _P, _I64, _I64, _P, _I64, _P]),
+    ("gptq_hessian_f32_workspace_bytes", _SZ, [_I64, _I64]),
+    ("gptq_hessian_accumulate_f32", _I, [_P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize_static_scratch", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
@@ -161,6 +163,21 @@ def gptq_hessian_accumulate_host(H: torch.Tensor, X_host: torch.Tensor, staging:
            lib().gptq_hessian_accumulate_host(_ptr(H), _ptr(X_host), n, d, _ptr(staging),
                                               chunk_tokens, _stream(H, stream)))
     return H
+
+
+def gptq_hessian_f32_workspace_bytes(d_in: int, chunk_tokens: int) -> int:
+    return int(lib().gptq_hessian_f32_workspace_bytes(d_in, chunk_tokens))
+
+
+def gptq_hessian_accumulate_f32(H: torch.Tensor, X: torch.Tensor, ws: torch.Tensor,
+                                chunk_tokens: int = 8192, stream=None):
+    """H float32 [d, d] += 2 X^T X for float32 X [n, d] on the device."""
+    _need(H, torch.float32, "H")
+    _need(X, torch.float32, "X")
+    n, d = X.shape
+    _check("gptq_hessian_accumulate_f32",
+           lib().gptq_hessian_accumulate_f32(_ptr(H), _ptr(X), n, d, chunk_tokens, _ptr(ws),
+                                             ws.numel() * ws.element_size(), _stream(H, stream)))
 
 
 def gptq_prepare(H: torch.Tensor, damp: float, act_order: bool, perm: torch.Tensor,

@@ -23,6 +23,9 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                  cudaStream_t s, bool graphed);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
+size_t hessian_f32_workspace_bytes(int64_t d, int64_t chunk);
+int run_hessian_f32(float* H, const float* X, int64_t n, int64_t d, int64_t chunk, void* ws,
+                    cudaStream_t s);
 bool w4a16_tc_supported(const uint16_t* X, const uint8_t* packed, const int32_t* g_idx,
                         int64_t K, int gs);
 int run_w4a16(float* Y, const uint16_t* X, const uint8_t* packed, const float* scales,
@@ -254,6 +257,32 @@ int gptq_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tokens, int64
     rc = hessian_device(H, X, n_tokens, d_in, s);
     if (rc) return rc;
     return launch_mirror(H, d_in, s);
+}
+
+size_t gptq_hessian_f32_workspace_bytes(int64_t d_in, int64_t chunk_tokens)
+{
+    if (d_in <= 0 || d_in > kMaxDim / 2 || d_in % 8 != 0 || chunk_tokens <= 0 ||
+        chunk_tokens > (int64_t(1) << 30))
+        return 0;
+    return hessian_f32_workspace_bytes(d_in, chunk_tokens);
+}
+
+int gptq_hessian_accumulate_f32(float* H, const float* X, int64_t n_tokens, int64_t d_in,
+                                int64_t chunk_tokens, void* workspace, size_t ws_bytes,
+                                void* stream)
+{
+    if (!H || (!X && n_tokens > 0) || n_tokens < 0 || d_in <= 0 || d_in > kMaxDim / 2 ||
+        d_in % 8 != 0 || chunk_tokens <= 0 || chunk_tokens > (int64_t(1) << 30) ||
+        !aligned(H, 16) || !aligned(X, 16))
+        return GPTQ_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) ||
+        ws_bytes < hessian_f32_workspace_bytes(d_in, chunk_tokens))
+        return GPTQ_ERR_WORKSPACE;
+    if (n_tokens == 0) return GPTQ_OK;
+    int rc = check_device();
+    if (rc) return rc;
+    return run_hessian_f32(H, X, n_tokens, d_in, chunk_tokens, workspace,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int gptq_hessian_accumulate_host(float* H, const uint16_t* X_host, int64_t n_tokens,

@@ -122,3 +122,24 @@ def test_w4a16_arguments_rejected_on_host(lib):
     # empty products are done without a device
     assert w(M=0) == 0
     assert w(N=0) == 0
+
+
+def test_hessian_f32_arguments_rejected_on_host(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    assert B.gptq_hessian_f32_workspace_bytes(4096, 8192) >= 16 * 4096 * 4096 + 4 * 8192 * 4096
+    assert B.gptq_hessian_f32_workspace_bytes(100, 16) == 0       # d_in not a multiple of 8
+    assert B.gptq_hessian_f32_workspace_bytes(40000, 16) == 0     # above 32768
+    assert B.gptq_hessian_f32_workspace_bytes(64, 0) == 0
+
+    def f(n=16, d=64, chunk=8, ws=fake, ws_bytes=1 << 40, H=fake, X=fake):
+        return lib.gptq_hessian_accumulate_f32(H, X, n, d, chunk, ws, ws_bytes, None)
+    assert f(d=60) == 1
+    assert f(chunk=0) == 1
+    assert f(n=-1) == 1
+    assert f(H=None) == 1
+    assert f(X=P((1 << 20) + 4)) == 1     # X not 16-byte aligned
+    assert f(ws=None) == 6
+    assert f(ws=P((1 << 20) + 16)) == 6   # workspace not 256-byte aligned
+    assert f(ws_bytes=100) == 6
+    assert f(n=0) == 0                    # nothing to do, device untouched
