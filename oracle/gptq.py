@@ -71,8 +71,10 @@ def _load():
             lib.orc_inverse_gauss_jordan.argtypes = [P, I64]
             lib.orc_obs_upper.argtypes = [P, I64, P]
             lib.orc_gptq_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64, I64, P, P, P, P, P, P]
+            lib.orc_gptq_rows_q4k.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, P]
             for f in (lib.orc_hessian_accumulate, lib.orc_hessian_block,
-                      lib.orc_inverse_gauss_jordan, lib.orc_obs_upper, lib.orc_gptq_rows):
+                      lib.orc_inverse_gauss_jordan, lib.orc_obs_upper, lib.orc_gptq_rows,
+                      lib.orc_gptq_rows_q4k):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -314,6 +316,61 @@ def rtn(W: np.ndarray, bits: int, group_size: int) -> dict:
         zeros[:, g] = z
         What[:, sl] = s[:, None].astype(np.float64) * (q.astype(np.float64) - z[:, None])
     return dict(codes=codes, scales=scales, zeros=zeros, W_hat=What)
+
+
+# --- GPTQ onto the two-level Q4_K grid -----------------------------------------
+
+Q4K_BLOCK, Q4K_SUPER = 32, 256
+
+
+def gptq_rows_q4k(Wp: np.ndarray, U: np.ndarray, block: int = 0) -> dict:
+    """Column loop onto the Q4_K grid (torchao pull request "Add gguf q4_k
+    quantization": w = q * block_scale + block_min, 6-bit block scales and
+    mins, a super-block scale above them) for W in processing order; see
+    orc_gptq_rows_q4k for the parameter choice.  Returns W^ (float64), codes,
+    sc6 and m6 [d_out, d_in/32], d and dmin [d_out, d_in/256], E, all in
+    processing order."""
+    W = np.array(Wp, dtype=np.float64, copy=True, order="C")
+    d_out, d_in = W.shape
+    U = np.ascontiguousarray(U, dtype=np.float64)
+    assert U.shape == (d_in, d_in) and d_in % Q4K_SUPER == 0
+    codes = np.empty((d_out, d_in), dtype=np.uint8)
+    sc6 = np.empty((d_out, d_in // Q4K_BLOCK), dtype=np.uint8)
+    m6 = np.empty((d_out, d_in // Q4K_BLOCK), dtype=np.uint8)
+    d = np.empty((d_out, d_in // Q4K_SUPER), dtype=np.float32)
+    dmin = np.empty((d_out, d_in // Q4K_SUPER), dtype=np.float32)
+    E = np.empty((d_out, d_in), dtype=np.float64)
+    _check(_load().orc_gptq_rows_q4k(_ptr(W), _ptr(U), d_out, d_in, block, _ptr(codes),
+                                     _ptr(sc6), _ptr(m6), _ptr(d), _ptr(dmin), _ptr(E)),
+           "gptq_rows_q4k")
+    return dict(W_hat=W, codes=codes, sc6=sc6, m6=m6, d=d, dmin=dmin, E=E)
+
+
+def dequant_q4k(codes: np.ndarray, sc6: np.ndarray, m6: np.ndarray, d: np.ndarray,
+                dmin: np.ndarray) -> np.ndarray:
+    """w^ = d sc q - dmin m for every column (processing order), float64, with
+    the products of the binary32 levels formed in binary32 as the grid does."""
+    blk = np.arange(codes.shape[1]) // Q4K_BLOCK
+    sup = np.arange(codes.shape[1]) // Q4K_SUPER
+    s = (d[:, sup] * sc6[:, blk].astype(np.float32)).astype(np.float32)
+    o = (dmin[:, sup] * m6[:, blk].astype(np.float32)).astype(np.float32)
+    return s.astype(np.float64) * codes.astype(np.float64) - o.astype(np.float64)
+
+
+def quantize_q4k(W: np.ndarray, U: np.ndarray, perm: np.ndarray | None, block: int = 0) -> dict:
+    """GPTQ onto the Q4_K grid for one layer, W in original column order (the
+    blocks and super-blocks run over processing order, as groups do)."""
+    W = np.asarray(W, dtype=np.float64)
+    d_in = W.shape[1]
+    perm = np.arange(d_in, dtype=np.int64) if perm is None else np.asarray(perm, dtype=np.int64)
+    r = gptq_rows_q4k(W[:, perm], U, block)
+    codes = np.empty_like(r["codes"])
+    codes[:, perm] = r["codes"]
+    What = np.empty_like(r["W_hat"])
+    What[:, perm] = r["W_hat"]
+    r.update(codes_perm=r["codes"], codes=codes, W_hat_perm=r["W_hat"], W_hat=What,
+             perm=perm.astype(np.int32), block_of=g_idx(perm, Q4K_BLOCK))
+    return r
 
 
 # --- metrics -----------------------------------------------------------------

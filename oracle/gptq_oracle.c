@@ -272,3 +272,111 @@ int orc_gptq_rows(double *W, const double *U, int64_t d_out, int64_t d_in, int b
     }
     return status;
 }
+
+/* ---- GPTQ onto the two-level Q4_K grid ---------------------------------
+ *
+ * The gguf Q4_K layout as the torchao pull request "Add gguf q4_k
+ * quantization" describes it: w = q * block_scale + block_min with 4-bit q,
+ * a 6-bit scale and a 6-bit min per block, and a second level (super-block
+ * scales) that quantizes those.  Blocks of 32 columns, super-blocks of 8
+ * blocks (256 columns), in processing order:
+ *     w^ = d sc q - dmin m,   q in 0..15,  sc in 1..63,  m in 0..63.
+ * Parameter choice (the simple min/max choice of the pull request), decided
+ * in binary32 like the one-level grid:
+ *   - range of a block: [min(0, min v), max(0, max v)], an all-zero block
+ *     taking [-1, 1]; raw scale = (max - min) / 15, raw offset = -min >= 0;
+ *   - at a super-block's first column, from the row's current values of its
+ *     256 columns: d = max raw scale / 63, dmin = max raw offset / 63;
+ *   - at a block's first column, from the row's current values of its 32
+ *     columns: sc = clamp(rint(scale / d), 1, 63), m = rint(offset / dmin)
+ *     clamped to 0..63 (0 when dmin = 0).
+ * Both levels use the values as updated by every earlier column, as the
+ * one-level grid does at its group starts.  Per column:
+ *     q = clamp(rint((w + dmin m) / (d sc)), 0, 15), w^ = d sc q - dmin m,
+ *     e = (w - w^) / U[c][c], compensation as in orc_gptq_rows.
+ * d_in must be a multiple of 256.  Outputs: codes [d_out][d_in]; sc6, m6
+ * [d_out][d_in / 32]; dsup, dmin [d_out][d_in / 256]; E (optional). */
+static void q4k_block_range(const double *v, int64_t n, float *scale, float *offset)
+{
+    float xmin = 0.0f, xmax = 0.0f;
+    for (int64_t k = 0; k < n; k++) {
+        float f = (float)v[k];
+        if (f < xmin) xmin = f;
+        if (f > xmax) xmax = f;
+    }
+    if (xmin == xmax) { xmin = -1.0f; xmax = 1.0f; }
+    *scale = (xmax - xmin) / 15.0f;
+    *offset = -xmin;
+}
+
+int orc_gptq_rows_q4k(double *W, const double *U, int64_t d_out, int64_t d_in, int64_t block,
+                      uint8_t *codes, uint8_t *sc6, uint8_t *m6, float *dsup, float *dmin,
+                      double *E)
+{
+    if (!W || !U || !codes || !sc6 || !m6 || !dsup || !dmin || d_out < 0 || d_in <= 0 ||
+        d_in % 256 != 0)
+        return ORC_ERR_ARG;
+    const int64_t nb = d_in / 32, ns = d_in / 256;
+    int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < d_out; r++) {
+        double *w = W + r * d_in;
+        double *e_row = (double *)malloc((size_t)d_in * sizeof(double));
+        if (!e_row) { status = ORC_ERR_ARG; continue; }
+        float d = 1.0f, dm = 0.0f, s = 1.0f, o = 0.0f;
+        for (int64_t c = 0; c < d_in; c++) {
+            if (c % 256 == 0) {
+                float smax = 0.0f, omax = 0.0f;
+                for (int b = 0; b < 8; b++) {
+                    float sc, of;
+                    q4k_block_range(w + c + 32 * b, 32, &sc, &of);
+                    if (sc > smax) smax = sc;
+                    if (of > omax) omax = of;
+                }
+                d = smax / 63.0f;
+                dm = omax / 63.0f;
+                dsup[r * ns + c / 256] = d;
+                dmin[r * ns + c / 256] = dm;
+            }
+            if (c % 32 == 0) {
+                float sc, of;
+                q4k_block_range(w + c, 32, &sc, &of);
+                float qs = rintf(sc / d);
+                if (qs < 1.0f) qs = 1.0f;
+                if (qs > 63.0f) qs = 63.0f;
+                float qm = dm > 0.0f ? rintf(of / dm) : 0.0f;
+                if (qm < 0.0f) qm = 0.0f;
+                if (qm > 63.0f) qm = 63.0f;
+                sc6[r * nb + c / 32] = (uint8_t)qs;
+                m6[r * nb + c / 32] = (uint8_t)qm;
+                s = d * qs;
+                o = dm * qm;
+            }
+            float q = rintf(((float)w[c] + o) / s);
+            if (q < 0.0f) q = 0.0f;
+            if (q > 15.0f) q = 15.0f;
+            double what = (double)s * (double)q - (double)o;
+            double e = (w[c] - what) / U[c * d_in + c];
+            codes[r * d_in + c] = (uint8_t)q;
+            w[c] = what;
+            e_row[c] = e;
+            if (block <= 0) {
+                for (int64_t k = c + 1; k < d_in; k++) w[k] -= e * U[c * d_in + k];
+            } else {
+                int64_t b0 = (c / block) * block;
+                int64_t b1 = (b0 + block < d_in) ? b0 + block : d_in;
+                for (int64_t k = c + 1; k < b1; k++) w[k] -= e * U[c * d_in + k];
+                if (c == b1 - 1) {
+                    for (int64_t k = b1; k < d_in; k++) {
+                        double acc = 0.0;
+                        for (int64_t i = b0; i < b1; i++) acc += e_row[i] * U[i * d_in + k];
+                        w[k] -= acc;
+                    }
+                }
+            }
+        }
+        if (E) memcpy(E + r * d_in, e_row, (size_t)d_in * sizeof(double));
+        free(e_row);
+    }
+    return status;
+}

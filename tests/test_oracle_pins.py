@@ -427,3 +427,70 @@ def test_hessian_f32_matches_brute_force_and_the_bf16_checker():
     xb = synth.f32_to_bf16_bits(g.standard_normal((300, 24)).astype(np.float32))
     xf = synth.bf16_bits_to_f32(xb)
     np.testing.assert_allclose(oracle.hessian_f32(xf, chunk=64), oracle.hessian(xb), rtol=1e-13, atol=0)
+
+
+# --- GPTQ onto the two-level Q4_K grid -----------------------------------------
+
+def _q4k_layer(seed, d_out=12, d_in=512, n=2048):
+    W, xb = synth.random_layer(seed, d_out, d_in, n, correlated=True)
+    H = oracle.hessian(xb)
+    perm, U, _, _ = oracle.prepare(H, 0.01, False)
+    return W, H, U
+
+
+def test_q4k_dequant_identity_and_level_ranges():
+    W, H, U = _q4k_layer(31)
+    r = oracle.quantize_q4k(W, U, None)
+    np.testing.assert_array_equal(
+        oracle.dequant_q4k(r["codes_perm"], r["sc6"], r["m6"], r["d"], r["dmin"]), r["W_hat_perm"])
+    assert r["codes"].max() <= 15
+    assert r["sc6"].min() >= 1 and r["sc6"].max() <= 63 and r["m6"].max() <= 63
+    assert (r["d"] > 0).all() and (r["dmin"] >= 0).all()
+
+
+def test_q4k_without_compensation_picks_the_nearest_grid_point():
+    """U = I turns off the error feedback: every code must be the nearest of
+    the 16 points s q - o of its block (brute force over q)."""
+    g = np.random.default_rng(5)
+    W = g.standard_normal((6, 256)) * 0.02
+    W[:, 40:72] *= 6.0                      # one wide block, so the others sit below sc = 63
+    r = oracle.quantize_q4k(W, np.eye(256), None)
+    s = (r["d"][:, [0]] * r["sc6"].astype(np.float32)).astype(np.float32).astype(np.float64)
+    o = (r["dmin"][:, [0]] * r["m6"].astype(np.float32)).astype(np.float32).astype(np.float64)
+    qs = np.arange(16, dtype=np.float64)
+    for i in range(W.shape[0]):
+        for c in range(256):
+            b = c // 32
+            pts = s[i, b] * qs - o[i, b]
+            dist = np.abs(W[i, c] - pts)
+            chosen = dist[r["codes"][i, c]]
+            assert chosen <= dist.min() + 1e-6 * s[i, b], (i, c)
+
+
+def test_q4k_super_block_scale_is_attained():
+    """d = (largest block scale) / 63, so without compensation the widest
+    block of every super-block gets sc = 63 (and the deepest min m = 63)."""
+    g = np.random.default_rng(6)
+    W = g.standard_normal((5, 512)) * 0.02
+    r = oracle.quantize_q4k(W, np.eye(512), None)
+    sc = r["sc6"].reshape(5, 2, 8)
+    m = r["m6"].reshape(5, 2, 8)
+    assert (sc.max(axis=2) == 63).all()
+    assert (m.max(axis=2) == 63).all()
+
+
+def test_q4k_lazy_batch_invariance():
+    W, H, U = _q4k_layer(32)
+    a = oracle.quantize_q4k(W, U, None, block=0)
+    b = oracle.quantize_q4k(W, U, None, block=128)
+    assert (a["codes"] == b["codes"]).mean() >= 0.999
+    assert np.abs(a["W_hat"] - b["W_hat"]).max() <= 1e-3 * np.abs(W).max()
+
+
+def test_q4k_gptq_lowers_the_output_error_of_round_to_nearest():
+    """The method's purpose on this grid too: the error feedback lowers the
+    layer-output MSE against rounding to nearest on the same grid (U = I)."""
+    W, H, U = _q4k_layer(33, d_out=16, d_in=512, n=4096)
+    gq = oracle.quantize_q4k(W, U, None)
+    rt = oracle.quantize_q4k(W, np.eye(W.shape[1]), None)
+    assert oracle.output_mse(W, gq["W_hat"], H, 4096) < 0.8 * oracle.output_mse(W, rt["W_hat"], H, 4096)
