@@ -203,6 +203,36 @@ int gptq_quantize(float *W, const float *Hinv_chol, const int32_t *perm, int64_t
                   float *scales, float *zeros, uint8_t *packed_int4, int32_t *g_idx,
                   float *err_sq, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * gptq_quantize onto the two-level Q4_K grid (torchao pull request "Add gguf
+ * q4_k quantization": w = q * block_scale + block_min with a 4-bit q, 6-bit
+ * block scales and mins, and super-block scales above them).  Blocks of 32
+ * columns and super-blocks of 256, both in processing order:
+ *     w^ = d sc q - dmin m,   q in 0..15,  sc in 1..63,  m in 0..63.
+ * At a super-block's first column, from each row's current (compensated)
+ * values of its 256 columns: per 32-column block the range [min(0, min),
+ * max(0, max)] (an all-zero block takes [-1, 1]) gives a raw scale
+ * (max - min) / 15 and offset -min; d = max raw scale / 63, dmin = max raw
+ * offset / 63.  At each block's first column, from the current values of its
+ * 32 columns: sc = clamp(rint(scale / d), 1, 63), m = clamp(rint(offset /
+ * dmin), 0, 63) (0 when dmin = 0).  Per column q = clamp(rint((w + dmin m) /
+ * (d sc)), 0, 15), then the usual error feedback (lazy batch of 128).
+ * Arguments as gptq_quantize (bits 4, group 32, block 128 implied), and
+ *   d_in     a multiple of 256.
+ *   codes    uint8 [d_out, d_in] OUT or NULL (original column order).
+ *   sc6, m6  uint8 [d_out, d_in / 32] OUT, blocks in processing order.
+ *   dsup, dmin  float32 [d_out, d_in / 256] OUT, super-blocks in processing order.
+ *   scales, offsets  float32 [d_out, d_in / 32] OUT: the block's d sc and
+ *            dmin m (w^ = scales * q - offsets).
+ *   packed_int4, g_idx (block of each original column), err_sq: as gptq_quantize.
+ * W holds W^ on return.
+ */
+int gptq_quantize_q4k(float *W, const float *Hinv_chol, const int32_t *perm, int64_t d_out,
+                      int64_t d_in, uint8_t *codes, uint8_t *sc6, uint8_t *m6, float *dsup,
+                      float *dmin, float *scales, float *offsets, uint8_t *packed_int4,
+                      int32_t *g_idx, float *err_sq, void *workspace, size_t ws_bytes,
+                      void *stream);
+
 /* Size of the fixed device array that gptq_quantize_static_scratch works in:
  * 128 MiB.  Every GPU on which the library's device code is loaded holds it
  * from then until the process exits. */

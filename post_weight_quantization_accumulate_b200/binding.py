@@ -38,6 +38,8 @@ SIGNATURES = [
     ("gptq_hessian_accumulate_f32", _I, [_P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    ("gptq_quantize_q4k", _I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                               _SZ, _P]),
     ("gptq_quantize_static_scratch", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     ("gptq_quantize_timed", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ,
                                  _P, _P, _P, _P]),
@@ -223,6 +225,23 @@ def gptq_quantize_timed(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Te
                                      _ptr(packed_int4), _ptr(g_idx), _ptr(err_sq), _ptr(ws),
                                      ws.numel(), _stream(W, stream), *(ctypes.byref(o) for o in out)))
     return tuple(o.value for o in out)
+
+
+def gptq_quantize_q4k(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor | None,
+                      out: dict, ws: torch.Tensor, codes: torch.Tensor | None = None,
+                      packed_int4: torch.Tensor | None = None, g_idx: torch.Tensor | None = None,
+                      err_sq: torch.Tensor | None = None, stream=None):
+    """GPTQ onto the Q4_K grid; `out` holds the device tensors sc6, m6
+    (uint8 [d_out, d_in/32]), dsup, dmin (float32 [d_out, d_in/256]) and
+    scales, offsets (float32 [d_out, d_in/32])."""
+    _need(W, torch.float32, "W")
+    d_out, d_in = W.shape
+    _check("gptq_quantize_q4k",
+           lib().gptq_quantize_q4k(_ptr(W), _ptr(Hinv_chol), _ptr(perm), d_out, d_in, _ptr(codes),
+                                   _ptr(out["sc6"]), _ptr(out["m6"]), _ptr(out["dsup"]),
+                                   _ptr(out["dmin"]), _ptr(out["scales"]), _ptr(out["offsets"]),
+                                   _ptr(packed_int4), _ptr(g_idx), _ptr(err_sq), _ptr(ws),
+                                   ws.numel(), _stream(W, stream)))
 
 
 def gptq_quantize_static_scratch(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor | None,

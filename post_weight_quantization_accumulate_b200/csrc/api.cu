@@ -20,7 +20,7 @@ int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* p
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
                  int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
                  uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, size_t ws_bytes,
-                 cudaStream_t s, bool graphed);
+                 cudaStream_t s, bool graphed, const Q4KOut* q4k = nullptr);
 int run_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, cudaStream_t s);
 int run_quotient_selftest(int64_t n, uint64_t seed, int64_t* mismatches);
 size_t hessian_f32_workspace_bytes(int64_t d, int64_t chunk);
@@ -416,6 +416,25 @@ int gptq_w4a16_gemm(float* Y, const uint16_t* X, const uint8_t* packed, const fl
     if (rc) return rc;
     return run_w4a16(Y, X, packed, scales, zeros, g_idx, M, N, K, group_size, path,
                      static_cast<cudaStream_t>(stream));
+}
+
+int gptq_quantize_q4k(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
+                      int64_t d_in, uint8_t* codes, uint8_t* sc6, uint8_t* m6, float* dsup,
+                      float* dmin, float* scales, float* offsets, uint8_t* packed_int4,
+                      int32_t* g_idx, float* err_sq, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!W || !Hinv_chol || !sc6 || !m6 || !dsup || !dmin || !scales || !offsets || d_out <= 0 ||
+        d_in <= 0 || d_in > kMaxDim || d_in % 256 != 0 || d_out > (int64_t(1) << 31) / 2 ||
+        !aligned(W, 16) || static_cast<int64_t>(d_out) * d_in >= (int64_t(1) << 40))
+        return GPTQ_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < quantize_workspace_min_bytes(d_out, d_in))
+        return GPTQ_ERR_WORKSPACE;
+    int rc = check_device();
+    if (rc) return rc;
+    const Q4KOut q4k{sc6, m6, dsup, dmin};
+    return run_quantize(W, Hinv_chol, perm, d_out, d_in, 4, 32, 128, codes, scales, offsets,
+                        packed_int4, g_idx, err_sq, workspace, ws_bytes,
+                        static_cast<cudaStream_t>(stream), true, &q4k);
 }
 
 int gptq_bf16_to_f32(float* dst, const uint16_t* src, int64_t n, void* stream)

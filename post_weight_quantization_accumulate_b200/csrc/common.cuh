@@ -46,6 +46,14 @@ int sm_count();                        // SMs of the current device
         if (_e != cudaSuccess) return ::gptq::cuda_fail(_e);  \
     } while (0)
 
+// Outputs of the two-level Q4_K grid (gptq_quantize_q4k).
+struct Q4KOut {
+    uint8_t* sc6;    // [d_out][d_in / 32] 6-bit block scales
+    uint8_t* m6;     // [d_out][d_in / 32] 6-bit block mins
+    float* dsup;     // [d_out][d_in / 256] super-block scale of the scales
+    float* dmin;     // [d_out][d_in / 256] super-block scale of the mins
+};
+
 // Upper bound on one device-side wait, in SM clock cycles (about 1 s).
 constexpr long long kWaitLimitCycles = 2000000000LL;
 

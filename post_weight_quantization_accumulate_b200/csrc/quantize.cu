@@ -61,6 +61,12 @@ struct QArgs {
     int e_off;            // column of this block inside the outer window
     float* err_sq;        // [d_out] or null
     int* status;
+    // two-level Q4_K grid (null otherwise): 6-bit scale and min per 32-column
+    // block [d_out][d_in / 32], super-block scales [d_out][d_in / 256]
+    uint8_t* sc6;
+    uint8_t* m6;
+    float* dsup;
+    float* dmin;
 };
 
 // Sub-block layout of U's diagonal blocks: chunk (b, S) covers rows
@@ -150,10 +156,11 @@ __device__ __forceinline__ float div_rn(float w, float s, float rs)
 // Scale and zero of the group starting at in-block column c, from one row's
 // current values: each part reduces its registers whose column lies in
 // [c, c + gs) and below bw, then the QTPR parts of the row pair combine.
-__device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int c, int gs, int bw,
-                                           float maxq, float& s, float& z)
+__device__ __forceinline__ void group_range(const float (&w)[QCPT], int part, int c, int gs, int bw,
+                                            float& mn, float& mx)
 {
-    float mn = 0.f, mx = 0.f;
+    mn = 0.f;
+    mx = 0.f;
 #pragma unroll
     for (int k = 0; k < QCPT; ++k) {
         const int col = QCPT * part + k;
@@ -167,7 +174,41 @@ __device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
+}
+
+__device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int c, int gs, int bw,
+                                           float maxq, float& s, float& z)
+{
+    float mn, mx;
+    group_range(w, part, c, gs, bw, mn, mx);
     grid_from_range(mn, mx, maxq, s, z);
+}
+
+// Q4_K (torchao pull request "Add gguf q4_k quantization": w = q * block_scale
+// + block_min, 6-bit block scales and mins under a super-block scale): the
+// raw scale and offset of a 32-column block from its range (an all-zero
+// range taking [-1, 1]).
+__device__ __forceinline__ void q4k_raw(float mn, float mx, float& scale, float& off)
+{
+    if (mn == mx) {
+        mn = -1.f;
+        mx = 1.f;
+    }
+    scale = __fdiv_rn(mx - mn, 15.f);
+    off = -mn;
+}
+
+// The block's 6-bit scale and min against the super-block's d and dmin, and
+// the grid they give: w^ = s q - o, s = d sc, o = dmin m.
+__device__ __forceinline__ void q4k_block_grid(float mn, float mx, float d, float dmin, float& s,
+                                               float& o, float& sc, float& m)
+{
+    float scale, off;
+    q4k_raw(mn, mx, scale, off);
+    sc = fminf(fmaxf(rintf(__fdiv_rn(scale, d)), 1.f), 63.f);
+    m = dmin > 0.f ? fminf(fmaxf(rintf(__fdiv_rn(off, dmin)), 0.f), 63.f) : 0.f;
+    s = d * sc;
+    o = dmin * m;
 }
 
 // One lazy-batch block [j0, j0 + bw) of the column loop for QROWS rows.
@@ -182,7 +223,7 @@ __device__ __forceinline__ void group_grid(const float (&w)[QCPT], int part, int
 // kGroupsInStep: a group may start inside a 16-column sub-block (group sizes
 // that are not multiples of 16); otherwise groups start at sub-block starts
 // and w^ is formed from the code at the store.
-template <bool kGroupsInStep>
+template <bool kGroupsInStep, bool kQ4K>
 __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
 {
     extern __shared__ __align__(128) uint8_t qsm_raw[];
@@ -270,6 +311,72 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
             }
         }
     }
+    // Q4_K super-block scales: at a super-block's first block from the current
+    // values of its 256 columns (this block's in registers, the next block's
+    // in the working copy, already corrected by every earlier block), else
+    // those the first block stored.  Part p holds columns 16p .. 16p + 15 of
+    // a block, i.e. half of 32-column block p / 2.
+    float qd[2] = {1.f, 1.f}, qdm[2] = {0.f, 0.f};
+    if (kQ4K) {
+        const int64_t sidx = j0 / 256;
+        const int ns = d_in / 256;
+        if (j0 % 256 == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float smax = 0.f, omax = 0.f;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float v[QCPT];
+                    if (half == 0) {
+#pragma unroll
+                        for (int k = 0; k < QCPT; ++k) v[k] = w[h][k];
+                    } else {
+#pragma unroll
+                        for (int m4 = 0; m4 < QCPT / 4; ++m4) {
+                            float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (valid[h])
+                                t4 = *reinterpret_cast<const float4*>(a.Wp + rowoff[h] + j0 + a.block +
+                                                                      QCPT * part + 4 * m4);
+                            v[4 * m4] = t4.x;
+                            v[4 * m4 + 1] = t4.y;
+                            v[4 * m4 + 2] = t4.z;
+                            v[4 * m4 + 3] = t4.w;
+                        }
+                    }
+                    float mn = 0.f, mx = 0.f;
+#pragma unroll
+                    for (int k = 0; k < QCPT; ++k) {
+                        mn = fminf(mn, v[k]);
+                        mx = fmaxf(mx, v[k]);
+                    }
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));   // the block's other half
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    float scale, off;
+                    q4k_raw(mn, mx, scale, off);
+                    smax = fmaxf(smax, scale);
+                    omax = fmaxf(omax, off);
+                }
+#pragma unroll
+                for (int o = 2; o < QTPR; o <<= 1) {
+                    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+                    omax = fmaxf(omax, __shfl_xor_sync(0xffffffffu, omax, o));
+                }
+                qd[h] = __fdiv_rn(smax, 63.f);
+                qdm[h] = __fdiv_rn(omax, 63.f);
+                if (valid[h] && part == 0) {
+                    a.dsup[static_cast<int64_t>(r[h]) * ns + sidx] = qd[h];
+                    a.dmin[static_cast<int64_t>(r[h]) * ns + sidx] = qdm[h];
+                }
+            }
+        } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                if (valid[h]) {
+                    qd[h] = a.dsup[static_cast<int64_t>(r[h]) * ns + sidx];
+                    qdm[h] = a.dmin[static_cast<int64_t>(r[h]) * ns + sidx];
+                }
+        }
+    }
     float rs[2] = {1.f / s[0], 1.f / s[1]};
     const int gs_in = (a.gs > 0 && a.gs <= a.block) ? a.gs : 0;
     int next_group = gs_in ? 0 : 1 << 30;
@@ -291,12 +398,23 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
         if (!kGroupsInStep && cbase == next_group) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                group_grid(w[h], part, cbase, gs_in, bw, maxq, s[h], z[h]);
+                float qsc = 0.f, qm = 0.f;
+                if (kQ4K) {   // z holds the block's offset o
+                    float mn, mx;
+                    group_range(w[h], part, cbase, gs_in, bw, mn, mx);
+                    q4k_block_grid(mn, mx, qd[h], qdm[h], s[h], z[h], qsc, qm);
+                } else {
+                    group_grid(w[h], part, cbase, gs_in, bw, maxq, s[h], z[h]);
+                }
                 rs[h] = 1.f / s[h];
                 if (valid[h] && part == 0) {
                     const int g = (j0 + cbase) / gs_in;
                     a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g] = s[h];
                     a.zeros[static_cast<int64_t>(r[h]) * a.n_groups + g] = z[h];
+                    if (kQ4K) {
+                        a.sc6[static_cast<int64_t>(r[h]) * a.n_groups + g] = static_cast<uint8_t>(qsc);
+                        a.m6[static_cast<int64_t>(r[h]) * a.n_groups + g] = static_cast<uint8_t>(qm);
+                    }
                 }
             }
             next_group += gs_in;
@@ -340,9 +458,15 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                 const float wc = nxt[h];
                 // q = clamp(rint(w / s) + z, 0, maxq) and w^ = s (q - z); with
                 // integer-valued floats, q - z = clamp(rint(w / s), -z, maxq - z)
-                const float qz = fminf(fmaxf(rintf(div_rn(wc, s[h], rs[h])), -z[h]), maxq - z[h]);
-                const float q = qz + z[h];
-                const float what = s[h] * qz;
+                float q, what;
+                if (kQ4K) {   // q = clamp(rint((w + o) / s), 0, 15), w^ = s q - o
+                    q = fminf(fmaxf(rintf(div_rn(wc + z[h], s[h], rs[h])), 0.f), 15.f);
+                    what = fmaf(s[h], q, -z[h]);
+                } else {
+                    const float qz = fminf(fmaxf(rintf(div_rn(wc, s[h], rs[h])), -z[h]), maxq - z[h]);
+                    q = qz + z[h];
+                    what = s[h] * qz;
+                }
                 const float e = (wc - what) * rn.x;
                 nxt[h] = fmaf(-e, rn.y, pre[h]);
                 errsum[h] = fmaf(e, e, errsum[h]);
@@ -362,8 +486,13 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
             for (int h = 0; h < 2; ++h) {
                 if (!valid[h]) continue;
                 if (!kGroupsInStep) {
-                    kw[h][0] = s[h] * (kq[h][0] - z[h]);
-                    kw[h][1] = s[h] * (kq[h][1] - z[h]);
+                    if (kQ4K) {
+                        kw[h][0] = fmaf(s[h], kq[h][0], -z[h]);
+                        kw[h][1] = fmaf(s[h], kq[h][1], -z[h]);
+                    } else {
+                        kw[h][0] = s[h] * (kq[h][0] - z[h]);
+                        kw[h][1] = s[h] * (kq[h][1] - z[h]);
+                    }
                 }
                 const int64_t eo = static_cast<int64_t>(r[h]) * kOuterMax + a.e_off + col;
                 *reinterpret_cast<float2*>(a.E + eo) = make_float2(ke[h][0], ke[h][1]);
@@ -591,7 +720,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                             int64_t d_in64, int bits, int gs, int block, uint8_t* codes,
                             float* scales, float* zeros, uint8_t* packed, int32_t* g_idx,
                             float* err_sq, void* workspace, bool with_low_parts, cudaStream_t stream,
-                            QuantizeMarks* marks = nullptr)
+                            QuantizeMarks* marks = nullptr, const Q4KOut* q4k = nullptr)
 {
     auto mark = [&](int c) { return marks ? marks->mark(stream, c) : GPTQ_OK; };
     if (int rc = mark(0)) return rc;
@@ -619,10 +748,13 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     int dev = 0;
     GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
     if (dev < 64 && !attr_set[dev]) {
-        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<false>,
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<false, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kBlockSmem)));
-        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<true>,
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<true, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kBlockSmem)));
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<false, true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kBlockSmem)));
         attr_set[dev] = true;
@@ -674,12 +806,16 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         for (int j0 = J0; j0 < J1; j0 += block) {
             const int bw = (J1 - j0 < block) ? J1 - j0 : block;
             QArgs a{work, Ul, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
-                    codes_p, E, E_lo, j0 - J0, err_sq, status};
+                    codes_p, E, E_lo, j0 - J0, err_sq, status,
+                    q4k ? q4k->sc6 : nullptr, q4k ? q4k->m6 : nullptr,
+                    q4k ? q4k->dsup : nullptr, q4k ? q4k->dmin : nullptr};
             if (int rc = mark(0)) return rc;
-            if (groups_in_step)
-                gptq_block_kernel<true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+            if (q4k)
+                gptq_block_kernel<false, true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+            else if (groups_in_step)
+                gptq_block_kernel<true, false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
             else
-                gptq_block_kernel<false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+                gptq_block_kernel<false, false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
             GPTQ_LAUNCH_CHECK();
             if (int rc = mark(1)) return rc;
             const int rest_in = J1 - j0 - bw;
@@ -717,12 +853,12 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in, int bits,
                  int gs, int block, uint8_t* codes, float* scales, float* zeros, uint8_t* packed,
                  int32_t* g_idx, float* err_sq, void* workspace, size_t ws_bytes, cudaStream_t stream,
-                 bool graphed)
+                 bool graphed, const Q4KOut* q4k)
 {
     const bool low = ws_bytes >= quantize_workspace_bytes(d_out, d_in);
     auto enq = [&](cudaStream_t s, int*) {
         return enqueue_quantize(W, U, perm, d_out, d_in, bits, gs, block, codes, scales, zeros,
-                                packed, g_idx, err_sq, workspace, low, s);
+                                packed, g_idx, err_sq, workspace, low, s, nullptr, q4k);
     };
     if (!graphed) return enq(stream, nullptr);
     auto P = [](const void* p) { return static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p)); };
@@ -731,7 +867,9 @@ int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, i
                                        static_cast<uint64_t>(static_cast<int64_t>(gs)),
                                        static_cast<uint64_t>(block), P(codes), P(scales), P(zeros),
                                        P(packed), P(g_idx), P(err_sq), P(workspace),
-                                       static_cast<uint64_t>(low)};
+                                       static_cast<uint64_t>(low), P(q4k ? q4k->sc6 : nullptr),
+                                       P(q4k ? q4k->m6 : nullptr), P(q4k ? q4k->dsup : nullptr),
+                                       P(q4k ? q4k->dmin : nullptr)};
     return run_graphed(key, false, enq, stream, nullptr);
 }
 

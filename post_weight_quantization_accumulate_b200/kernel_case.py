@@ -85,7 +85,8 @@ def w4a16_case(a):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--call", default="hessian",
-                    choices=["hessian", "prepare", "quantize", "layer", "tf32_peak", "w4a16"])
+                    choices=["hessian", "prepare", "quantize", "quantize_q4k", "layer", "tf32_peak",
+                             "w4a16"])
     ap.add_argument("--workload", default="q_proj_4096")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
@@ -112,6 +113,14 @@ def main():
     q.reset()
     q.add_batch(X)
     q.prepare()
+    Wq = torch.empty_like(W)
+    nb, ns = spec.d_in // 32, max(1, spec.d_in // 256)
+    q4k_out = {"sc6": torch.empty(spec.d_out, nb, dtype=torch.uint8, device=dev),
+               "m6": torch.empty(spec.d_out, nb, dtype=torch.uint8, device=dev),
+               "dsup": torch.empty(spec.d_out, ns, dtype=torch.float32, device=dev),
+               "dmin": torch.empty(spec.d_out, ns, dtype=torch.float32, device=dev),
+               "scales": torch.empty(spec.d_out, nb, dtype=torch.float32, device=dev),
+               "offsets": torch.empty(spec.d_out, nb, dtype=torch.float32, device=dev)}
 
     def once():
         if a.call == "hessian":
@@ -121,6 +130,9 @@ def main():
             q.prepare()
         elif a.call == "quantize":
             q.quantize(W)
+        elif a.call == "quantize_q4k":
+            Wq.copy_(W)
+            B.gptq_quantize_q4k(Wq, q.U, None, q4k_out, q.ws, codes=q.codes)
         else:
             q.reset()
             q.add_batch(X)

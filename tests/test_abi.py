@@ -143,3 +143,16 @@ def test_hessian_f32_arguments_rejected_on_host(lib):
     assert f(ws=P((1 << 20) + 16)) == 6   # workspace not 256-byte aligned
     assert f(ws_bytes=100) == 6
     assert f(n=0) == 0                    # nothing to do, device untouched
+
+
+def test_q4k_arguments_rejected_on_host(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+
+    def q(d_in=512, sc6=fake, ws=fake, ws_bytes=1 << 40):
+        return lib.gptq_quantize_q4k(fake, fake, None, 64, d_in, None, sc6, fake, fake, fake, fake,
+                                     fake, None, None, None, ws, ws_bytes, None)
+    assert q(d_in=384) == 1          # not a multiple of 256
+    assert q(sc6=None) == 1
+    assert q(ws=None) == 6
+    assert q(ws_bytes=100) == 6

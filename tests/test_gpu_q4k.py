@@ -1,0 +1,79 @@
+"""GPTQ onto the two-level Q4_K grid on the device against the float64
+checker, given the device's own factor and order (the staged parity of the
+one-level grid): codes and 6-bit levels agree except at rounding ties (at
+least 99.9%), super-block scales to 1e-5, the layer-output MSE to 1%; the
+device's outputs obey w^ = d sc q - dmin m exactly."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_accumulate_b200 import binding as B
+from post_weight_quantization_accumulate_b200 import synth
+
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(d_out, d_in, n, act_order, seed):
+    W, xb = synth.random_layer(seed, d_out, d_in, n, correlated=True)
+    dev = torch.device("cuda")
+    X = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    H = torch.zeros(d_in, d_in, dtype=torch.float32, device=dev)
+    B.gptq_hessian_accumulate(H, X)
+    perm = torch.empty(d_in, dtype=torch.int32, device=dev)
+    U = torch.empty(d_in, d_in, dtype=torch.float32, device=dev)
+    ws = B.workspace(d_out, d_in, 128, device=dev)
+    B.gptq_prepare(H, 0.01, act_order, perm, U, ws)
+    Wt = torch.from_numpy(W.astype(np.float32)).to(dev)
+    nb, ns = d_in // 32, d_in // 256
+    out = {"sc6": torch.empty(d_out, nb, dtype=torch.uint8, device=dev),
+           "m6": torch.empty(d_out, nb, dtype=torch.uint8, device=dev),
+           "dsup": torch.empty(d_out, ns, dtype=torch.float32, device=dev),
+           "dmin": torch.empty(d_out, ns, dtype=torch.float32, device=dev),
+           "scales": torch.empty(d_out, nb, dtype=torch.float32, device=dev),
+           "offsets": torch.empty(d_out, nb, dtype=torch.float32, device=dev)}
+    codes = torch.empty(d_out, d_in, dtype=torch.uint8, device=dev)
+    packed = torch.empty(d_out, d_in // 2, dtype=torch.uint8, device=dev)
+    g_idx = torch.empty(d_in, dtype=torch.int32, device=dev)
+    B.gptq_quantize_q4k(Wt, U, perm if act_order else None, out, ws, codes=codes,
+                        packed_int4=packed, g_idx=g_idx)
+    torch.cuda.synchronize()
+    assert B.gptq_device_status() == 0
+    g = {k: v.cpu().numpy() for k, v in out.items()}
+    g.update(codes=codes.cpu().numpy(), packed=packed.cpu().numpy(), g_idx=g_idx.cpu().numpy(),
+             W_hat=Wt.cpu().numpy(), H=H.cpu().numpy().astype(np.float64),
+             U=U.cpu().numpy().astype(np.float64), perm=perm.cpu().numpy())
+    return W, g
+
+
+@pytest.mark.parametrize("d_out,d_in,act_order", [(256, 1024, False), (200, 2048, True), (64, 256, False)])
+def test_q4k_matches_checker(d_out, d_in, act_order):
+    W, g = _run(d_out, d_in, 4096, act_order, d_in + d_out)
+    perm = g["perm"] if act_order else None
+    ref = oracle.quantize_q4k(W, g["U"], perm)
+    assert (g["codes"] == ref["codes"]).mean() >= P.CODE_MATCH
+    assert (g["sc6"] == ref["sc6"]).mean() >= P.CODE_MATCH
+    assert (g["m6"] == ref["m6"]).mean() >= P.CODE_MATCH
+    close = np.abs(g["dsup"] - ref["d"]) <= 1e-5 * ref["d"]
+    assert close.mean() >= P.CODE_MATCH
+    close = np.abs(g["dmin"] - ref["dmin"]) <= 1e-5 * np.maximum(ref["dmin"], 1e-30)
+    assert close.mean() >= P.CODE_MATCH
+    n = 4096
+    mse_g = oracle.output_mse(W, g["W_hat"].astype(np.float64), g["H"], n)
+    mse_r = oracle.output_mse(W, ref["W_hat"], g["H"], n)
+    assert abs(mse_g - mse_r) <= 0.01 * mse_r, (mse_g, mse_r)
+    # the device's own outputs: levels in range and w^ = scales q - offsets
+    assert g["codes"].max() <= 15 and g["sc6"].min() >= 1 and g["sc6"].max() <= 63 and g["m6"].max() <= 63
+    blk = np.arange(d_in) // 32
+    sup = np.arange(d_in) // 256
+    np.testing.assert_array_equal(g["scales"], (g["dsup"][:, sup[::32]] * g["sc6"].astype(np.float32)))
+    np.testing.assert_array_equal(g["offsets"], (g["dmin"][:, sup[::32]] * g["m6"].astype(np.float32)))
+    pk = perm if perm is not None else np.arange(d_in)
+    codes_p = g["codes"][:, pk]
+    what_p = (g["scales"][:, blk].astype(np.float64) * codes_p - g["offsets"][:, blk]).astype(np.float32)
+    # one rounding of s q - o (fused on the device): within one ulp of the float64 form
+    assert (np.abs(g["W_hat"][:, pk] - what_p) <= np.spacing(np.abs(what_p))).all()
+    np.testing.assert_array_equal(oracle.unpack_int4(g["packed"]), g["codes"])
+    np.testing.assert_array_equal(g["g_idx"], oracle.g_idx(pk, 32))
