@@ -243,7 +243,7 @@ int gptq_quantize_q4k(float *W, const float *Hinv_chol, const int32_t *perm, int
  * device memory: a plugin inside another engine that is handed only input and
  * output pointers and has no allocator to ask; a serving loop that must not
  * pay cudaMalloc's implicit device-wide synchronisation; a process that has
- * reserved the GPU's memory up front for its own pool.  The paper has no
+ * reserved the GPU's memory up front for its own pool.  The method has no
  * counterpart to this call; it exists only for such callers.
  *
  * Arguments, outputs and results are those of gptq_quantize.  The scratch is

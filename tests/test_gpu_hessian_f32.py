@@ -1,6 +1,6 @@
 """H = 2 X^T X for float32 activations (the tiny workload's fp32 draw and
 ragged shapes) on the device against the float64 checker.  Tolerance: the
-the benchmark spec's Hessian bound, 1e-5 relative in the Frobenius norm (the split
+Hessian bound of the bf16 path, 1e-5 relative in the Frobenius norm (the split
 leaves at most 2^-17 relative per product, the sums are fp32)."""
 import numpy as np
 import pytest
