@@ -58,25 +58,28 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Argument and result types of the checker's C entry points on `lib`."""
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    lib.orc_hessian_accumulate.argtypes = [P, P, I64, I64]
+    lib.orc_hessian_block.argtypes = [P, P, I64, I64, P, I64, P, I64]
+    lib.orc_inverse_gauss_jordan.argtypes = [P, I64]
+    lib.orc_obs_upper.argtypes = [P, I64, P]
+    lib.orc_gptq_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64, I64, P, P, P, P, P, P]
+    lib.orc_gptq_rows_q4k.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, P]
+    for f in (lib.orc_hessian_accumulate, lib.orc_hessian_block, lib.orc_inverse_gauss_jordan,
+              lib.orc_obs_upper, lib.orc_gptq_rows, lib.orc_gptq_rows_q4k):
+        f.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
             build()
-            lib = ctypes.CDLL(_LIB)
-            P = ctypes.c_void_p
-            I64 = ctypes.c_int64
-            lib.orc_hessian_accumulate.argtypes = [P, P, I64, I64]
-            lib.orc_hessian_block.argtypes = [P, P, I64, I64, P, I64, P, I64]
-            lib.orc_inverse_gauss_jordan.argtypes = [P, I64]
-            lib.orc_obs_upper.argtypes = [P, I64, P]
-            lib.orc_gptq_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64, I64, P, P, P, P, P, P]
-            lib.orc_gptq_rows_q4k.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, P]
-            for f in (lib.orc_hessian_accumulate, lib.orc_hessian_block,
-                      lib.orc_inverse_gauss_jordan, lib.orc_obs_upper, lib.orc_gptq_rows,
-                      lib.orc_gptq_rows_q4k):
-                f.restype = ctypes.c_int
-            _lib = lib
+            _lib = configure(ctypes.CDLL(_LIB))
     return _lib
 
 
