@@ -4,6 +4,8 @@
         --call hessian|prepare|quantize|layer --workload q_proj_4096 [--tokens N] [--reps R]
     python -m post_weight_quantization_accumulate_b200.kernel_case \
         --call w4a16 [--m M] [--n N] [--k K] [--group-size G] [--path 0|1|2] [--reps R]
+    python -m post_weight_quantization_accumulate_b200.kernel_case \
+        --call hessian_f32 --workload q_proj_4096 --tokens N [--reps R]
 
 The inputs follow the workload's recipe (see synth.py) with `--tokens`
 overriding the calibration size, so a profiler can capture a launch on a case
@@ -82,11 +84,35 @@ def w4a16_case(a):
           f"{min(ms[1:]) * 1e3:.1f} us/call (cold L2, single launch), status {B.gptq_device_status()}")
 
 
+def hessian_f32_case(a):
+    """gptq_hessian_accumulate_f32 on the workload's fp32 activation draw
+    (`--tokens` of them), 8192-token chunks."""
+    spec = synth.WORKLOADS[a.workload]
+    if a.tokens:
+        spec = synth.scaled(spec, n_tokens=a.tokens)
+    dev = torch.device("cuda", 0)
+    X = torch.from_numpy(synth.x_f32_unrounded(spec)).to(dev)
+    H = torch.zeros(spec.d_in, spec.d_in, dtype=torch.float32, device=dev)
+    chunk = 8192
+    ws = torch.empty(B.gptq_hessian_f32_workspace_bytes(spec.d_in, chunk), dtype=torch.uint8, device=dev)
+    B.gptq_hessian_accumulate_f32(H, X, ws, chunk)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        H.zero_()
+        B.gptq_hessian_accumulate_f32(H, X, ws, chunk)
+    e1.record()
+    torch.cuda.synchronize()
+    print(f"hessian_f32 {spec.name} tokens={spec.n_tokens}: {e0.elapsed_time(e1) / a.reps:.3f} ms/call "
+          f"on the device, status {B.gptq_device_status()}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--call", default="hessian",
-                    choices=["hessian", "prepare", "quantize", "quantize_q4k", "layer", "tf32_peak",
-                             "w4a16"])
+                    choices=["hessian", "hessian_f32", "prepare", "quantize", "quantize_q4k", "layer",
+                             "tf32_peak", "w4a16"])
     ap.add_argument("--workload", default="q_proj_4096")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
@@ -101,6 +127,9 @@ def main():
         return
     if a.call == "w4a16":
         w4a16_case(a)
+        return
+    if a.call == "hessian_f32":
+        hessian_f32_case(a)
         return
     spec = synth.WORKLOADS[a.workload]
     if a.tokens:
