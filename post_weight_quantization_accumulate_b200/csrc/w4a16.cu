@@ -29,6 +29,10 @@
 //     permute each 16-byte chunk of the X tile the same way.
 //   * One thread issues kind::f16 MMAs, A from TMEM, B = X from shared memory,
 //     D = the group's accumulator slot (NP columns; 128 / NP slots in a ring).
+//     The group bookkeeping is done once per group; per 16-column step only
+//     the MMA is issued (eight straight-line MMAs when a whole stage lies in
+//     one group), because the issuing thread's own instruction count sets the
+//     pace at these small MMA shapes.
 //   * The converters read finished group accumulators one stage behind and
 //     accumulate s * acc into registers.
 //   * K is split over a cluster of up to 8 CTAs; the partial sums meet in
