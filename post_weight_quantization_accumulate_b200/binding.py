@@ -235,6 +235,10 @@ def gptq_quantize_q4k(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tens
     (uint8 [d_out, d_in/32]), dsup, dmin (float32 [d_out, d_in/256]) and
     scales, offsets (float32 [d_out, d_in/32])."""
     _need(W, torch.float32, "W")
+    for k in ("sc6", "m6"):
+        _need(out.get(k), torch.uint8, k)
+    for k in ("dsup", "dmin", "scales", "offsets"):
+        _need(out.get(k), torch.float32, k)
     d_out, d_in = W.shape
     _check("gptq_quantize_q4k",
            lib().gptq_quantize_q4k(_ptr(W), _ptr(Hinv_chol), _ptr(perm), d_out, d_in, _ptr(codes),

@@ -71,6 +71,17 @@ class LayerQuantizer:
         B.gptq_hessian_accumulate_host(self.H, X_host, self.staging, chunk_tokens)
         self.n_tokens += X_host.shape[0]
 
+    def add_batch_f32(self, X: torch.Tensor, chunk_tokens: int = 8192):
+        """X float32 [n, d_in] on the device (bf16 hi/lo split through the
+        tensor-core Hessian; see gptq_hessian_accumulate_f32)."""
+        need = B.gptq_hessian_f32_workspace_bytes(self.d_in, chunk_tokens)
+        if need == 0:
+            raise ValueError("d_in or chunk_tokens out of range for the fp32 Hessian")
+        if getattr(self, "ws_f32", None) is None or self.ws_f32.numel() < need:
+            self.ws_f32 = torch.empty(need, dtype=torch.uint8, device=self.device)
+        B.gptq_hessian_accumulate_f32(self.H, X, self.ws_f32, chunk_tokens)
+        self.n_tokens += X.shape[0]
+
     # -- steps 2-5 ----------------------------------------------------------------
     def prepare(self):
         B.gptq_prepare(self.H, self.damp, self.act_order, self.perm, self.U, self.ws)
@@ -87,6 +98,34 @@ class LayerQuantizer:
                         err_sq=self.err_sq)
         return QuantizedLayer(self.packed, self.codes, self.scales, self.zeros, self.g_idx,
                               self.perm, self.W, self.err_sq)
+
+    def quantize_q4k(self, W: torch.Tensor) -> dict:
+        """GPTQ onto the two-level Q4_K grid (d_in a multiple of 256; the
+        layer's bits / group_size / block_size do not apply).  Returns device
+        tensors: codes, packed, g_idx, sc6, m6 (per 32-column block), dsup, dmin
+        (per 256-column super-block), scales, offsets (the blocks' d sc and
+        dmin m) and W_hat; blocks in processing order."""
+        if self.d_in % 256 != 0:
+            raise ValueError("the Q4_K grid needs d_in to be a multiple of 256")
+        if W.dtype == torch.bfloat16:
+            B.gptq_bf16_to_f32(self.W, W)
+        else:
+            self.W.copy_(W)
+        nb, ns = self.d_in // 32, self.d_in // 256
+        dev = self.device
+        out = {"sc6": torch.empty(self.d_out, nb, dtype=torch.uint8, device=dev),
+               "m6": torch.empty(self.d_out, nb, dtype=torch.uint8, device=dev),
+               "dsup": torch.empty(self.d_out, ns, dtype=torch.float32, device=dev),
+               "dmin": torch.empty(self.d_out, ns, dtype=torch.float32, device=dev),
+               "scales": torch.empty(self.d_out, nb, dtype=torch.float32, device=dev),
+               "offsets": torch.empty(self.d_out, nb, dtype=torch.float32, device=dev)}
+        codes = torch.empty(self.d_out, self.d_in, dtype=torch.uint8, device=dev)
+        packed = torch.empty(self.d_out, self.d_in // 2, dtype=torch.uint8, device=dev)
+        g_idx = torch.empty(self.d_in, dtype=torch.int32, device=dev)
+        B.gptq_quantize_q4k(self.W, self.U, self.perm if self.act_order else None, out, self.ws,
+                            codes=codes, packed_int4=packed, g_idx=g_idx)
+        out.update(codes=codes, packed=packed, g_idx=g_idx, W_hat=self.W)
+        return out
 
     def quantize_timed(self, W: torch.Tensor):
         """As quantize, enqueued directly with CUDA events between launches;

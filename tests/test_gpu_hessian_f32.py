@@ -58,3 +58,15 @@ def test_hessian_f32_accumulates_across_calls():
     H = _gpu_h(x[:1500], 512)
     H = _gpu_h(x[1500:], 512, H).cpu().numpy()
     assert P.rel_fro(H, oracle.hessian_f32(x)) <= P.H_RTOL
+
+
+def test_hessian_f32_through_the_layer_wrapper():
+    from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
+    x = _x(9, 3000, 256)
+    q = LayerQuantizer(64, 256)
+    q.reset()
+    q.add_batch_f32(torch.from_numpy(x).cuda(), chunk_tokens=1024)
+    torch.cuda.synchronize()
+    assert B.gptq_device_status() == 0
+    assert q.n_tokens == 3000
+    assert P.rel_fro(q.H.cpu().numpy(), oracle.hessian_f32(x)) <= P.H_RTOL

@@ -77,3 +77,22 @@ def test_q4k_matches_checker(d_out, d_in, act_order):
     assert (np.abs(g["W_hat"][:, pk] - what_p) <= np.spacing(np.abs(what_p))).all()
     np.testing.assert_array_equal(oracle.unpack_int4(g["packed"]), g["codes"])
     np.testing.assert_array_equal(g["g_idx"], oracle.g_idx(pk, 32))
+
+
+def test_q4k_through_the_layer_wrapper():
+    """LayerQuantizer.quantize_q4k (act_order) against the checker with the
+    wrapper's own factor and order."""
+    from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
+    d_out, d_in = 96, 512
+    W, xb = synth.random_layer(77, d_out, d_in, 2048, correlated=True)
+    q = LayerQuantizer(d_out, d_in, act_order=True)
+    q.add_batch(torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16))
+    q.prepare()
+    r = q.quantize_q4k(torch.from_numpy(W.astype(np.float32)).cuda())
+    torch.cuda.synchronize()
+    assert B.gptq_device_status() == 0
+    perm = q.perm.cpu().numpy()
+    ref = oracle.quantize_q4k(W, q.U.cpu().numpy().astype(np.float64), perm)
+    assert (r["codes"].cpu().numpy() == ref["codes"]).mean() >= P.CODE_MATCH
+    assert (r["sc6"].cpu().numpy() == ref["sc6"]).mean() >= P.CODE_MATCH
+    np.testing.assert_array_equal(oracle.unpack_int4(r["packed"].cpu().numpy()), r["codes"].cpu().numpy())
