@@ -33,9 +33,10 @@ MUTATIONS = [
      [("test_obs_upper_equals_lapack_cholesky_of_inverse", (8, 10.0))]),
     ("Q4_K offset with the wrong sign", "float q = rintf(((float)w[c] + o) / s);",
      "float q = rintf(((float)w[c] - o) / s);",
-     [("test_q4k_without_compensation_picks_the_nearest_grid_point", ())]),
+     [("test_q4k_without_compensation_picks_the_nearest_grid_point", ()),
+      ("test_q4k_golden_worked_example", ())]),
     ("Q4_K super-block scale over 15 levels", "d = smax / 63.0f;", "d = smax / 15.0f;",
-     [("test_q4k_super_block_scale_is_attained", ())]),
+     [("test_q4k_super_block_scale_is_attained", ()), ("test_q4k_golden_worked_example", ())]),
     ("Q4_K without error feedback",
      "for (int64_t k = c + 1; k < b1; k++) w[k] -= e * U[c * d_in + k];\n                if (c == b1 - 1) {\n                    for (int64_t k = b1; k < d_in; k++) {\n                        double acc = 0.0;\n                        for (int64_t i = b0; i < b1; i++) acc += e_row[i] * U[i * d_in + k];\n                        w[k] -= acc;\n                    }\n                }\n            }\n        }\n        if (E) memcpy(E + r * d_in, e_row, (size_t)d_in * sizeof(double));\n        free(e_row);\n    }\n    return status;\n}\n",
      None,

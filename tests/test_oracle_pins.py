@@ -494,3 +494,17 @@ def test_q4k_gptq_lowers_the_output_error_of_round_to_nearest():
     gq = oracle.quantize_q4k(W, U, None)
     rt = oracle.quantize_q4k(W, np.eye(W.shape[1]), None)
     assert oracle.output_mse(W, gq["W_hat"], H, 4096) < 0.8 * oracle.output_mse(W, rt["W_hat"], H, 4096)
+
+
+def test_q4k_golden_worked_example():
+    """A hand-derived super-block (tests/golden/q4k_case.json): every binary32
+    step is exact, one value sits on a rounding tie, one block sets both
+    super-block scales and the others quantize against them."""
+    case = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "q4k_case.json")))
+    v = np.array([case["values"]], np.float64)
+    r = oracle.quantize_q4k(v, np.eye(256), None)
+    assert r["d"][0, 0] == np.float32(case["d"]) and r["dmin"][0, 0] == np.float32(case["dmin"])
+    np.testing.assert_array_equal(r["sc6"][0], case["sc6"])
+    np.testing.assert_array_equal(r["m6"][0], case["m6"])
+    np.testing.assert_array_equal(r["codes"][0], case["codes"])
+    np.testing.assert_array_equal(r["W_hat"][0], case["w_hat"])
