@@ -67,7 +67,7 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.orc_inverse_gauss_jordan.argtypes = [P, I64]
     lib.orc_obs_upper.argtypes = [P, I64, P]
     lib.orc_gptq_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64, I64, P, P, P, P, P, P]
-    lib.orc_gptq_rows_q4k.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, P]
+    lib.orc_gptq_rows_q4k.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, P, P, P, P]
     for f in (lib.orc_hessian_accumulate, lib.orc_hessian_block, lib.orc_inverse_gauss_jordan,
               lib.orc_obs_upper, lib.orc_gptq_rows, lib.orc_gptq_rows_q4k):
         f.restype = ctypes.c_int
@@ -331,8 +331,9 @@ def gptq_rows_q4k(Wp: np.ndarray, U: np.ndarray, block: int = 0) -> dict:
     quantization": w = q * block_scale + block_min, 6-bit block scales and
     mins, a super-block scale above them) for W in processing order; see
     orc_gptq_rows_q4k for the parameter choice.  Returns W^ (float64), codes,
-    sc6 and m6 [d_out, d_in/32], d and dmin [d_out, d_in/256], E, all in
-    processing order."""
+    sc6 and m6 [d_out, d_in/32], d and dmin [d_out, d_in/256], E, and the
+    decision values before rounding (qraw = (w + o) / s per column, scraw =
+    scale / d and mraw = offset / dmin per block), all in processing order."""
     W = np.array(Wp, dtype=np.float64, copy=True, order="C")
     d_out, d_in = W.shape
     U = np.ascontiguousarray(U, dtype=np.float64)
@@ -343,10 +344,15 @@ def gptq_rows_q4k(Wp: np.ndarray, U: np.ndarray, block: int = 0) -> dict:
     d = np.empty((d_out, d_in // Q4K_SUPER), dtype=np.float32)
     dmin = np.empty((d_out, d_in // Q4K_SUPER), dtype=np.float32)
     E = np.empty((d_out, d_in), dtype=np.float64)
+    qraw = np.empty((d_out, d_in), dtype=np.float32)
+    scraw = np.empty((d_out, d_in // Q4K_BLOCK), dtype=np.float32)
+    mraw = np.empty((d_out, d_in // Q4K_BLOCK), dtype=np.float32)
     _check(_load().orc_gptq_rows_q4k(_ptr(W), _ptr(U), d_out, d_in, block, _ptr(codes),
-                                     _ptr(sc6), _ptr(m6), _ptr(d), _ptr(dmin), _ptr(E)),
+                                     _ptr(sc6), _ptr(m6), _ptr(d), _ptr(dmin), _ptr(E),
+                                     _ptr(qraw), _ptr(scraw), _ptr(mraw)),
            "gptq_rows_q4k")
-    return dict(W_hat=W, codes=codes, sc6=sc6, m6=m6, d=d, dmin=dmin, E=E)
+    return dict(W_hat=W, codes=codes, sc6=sc6, m6=m6, d=d, dmin=dmin, E=E, qraw=qraw,
+                scraw=scraw, mraw=mraw)
 
 
 def dequant_q4k(codes: np.ndarray, sc6: np.ndarray, m6: np.ndarray, d: np.ndarray,

@@ -295,7 +295,11 @@ int orc_gptq_rows(double *W, const double *U, int64_t d_out, int64_t d_in, int b
  *     q = clamp(rint((w + dmin m) / (d sc)), 0, 15), w^ = d sc q - dmin m,
  *     e = (w - w^) / U[c][c], compensation as in orc_gptq_rows.
  * d_in must be a multiple of 256.  Outputs: codes [d_out][d_in]; sc6, m6
- * [d_out][d_in / 32]; dsup, dmin [d_out][d_in / 256]; E (optional). */
+ * [d_out][d_in / 32]; dsup, dmin [d_out][d_in / 256]; E (optional).
+ * Optional diagnostics (NULL to skip), the decision values before rounding:
+ * qraw [d_out][d_in] = (w + o) / s, scraw and mraw [d_out][d_in / 32] =
+ * scale / d and offset / dmin (0 when dmin = 0); they tell how close each
+ * integer decision was to a rounding tie. */
 static void q4k_block_range(const double *v, int64_t n, float *scale, float *offset)
 {
     float xmin = 0.0f, xmax = 0.0f;
@@ -311,7 +315,7 @@ static void q4k_block_range(const double *v, int64_t n, float *scale, float *off
 
 int orc_gptq_rows_q4k(double *W, const double *U, int64_t d_out, int64_t d_in, int64_t block,
                       uint8_t *codes, uint8_t *sc6, uint8_t *m6, float *dsup, float *dmin,
-                      double *E)
+                      double *E, float *qraw, float *scraw, float *mraw)
 {
     if (!W || !U || !codes || !sc6 || !m6 || !dsup || !dmin || d_out < 0 || d_in <= 0 ||
         d_in % 256 != 0)
@@ -341,10 +345,14 @@ int orc_gptq_rows_q4k(double *W, const double *U, int64_t d_out, int64_t d_in, i
             if (c % 32 == 0) {
                 float sc, of;
                 q4k_block_range(w + c, 32, &sc, &of);
-                float qs = rintf(sc / d);
+                float scr = sc / d;
+                float mr = dm > 0.0f ? of / dm : 0.0f;
+                if (scraw) scraw[r * nb + c / 32] = scr;
+                if (mraw) mraw[r * nb + c / 32] = mr;
+                float qs = rintf(scr);
                 if (qs < 1.0f) qs = 1.0f;
                 if (qs > 63.0f) qs = 63.0f;
-                float qm = dm > 0.0f ? rintf(of / dm) : 0.0f;
+                float qm = rintf(mr);
                 if (qm < 0.0f) qm = 0.0f;
                 if (qm > 63.0f) qm = 63.0f;
                 sc6[r * nb + c / 32] = (uint8_t)qs;
@@ -352,7 +360,9 @@ int orc_gptq_rows_q4k(double *W, const double *U, int64_t d_out, int64_t d_in, i
                 s = d * qs;
                 o = dm * qm;
             }
-            float q = rintf(((float)w[c] + o) / s);
+            float qr = ((float)w[c] + o) / s;
+            if (qraw) qraw[r * d_in + c] = qr;
+            float q = rintf(qr);
             if (q < 0.0f) q = 0.0f;
             if (q > 15.0f) q = 15.0f;
             double what = (double)s * (double)q - (double)o;

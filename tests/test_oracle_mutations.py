@@ -31,8 +31,8 @@ MUTATIONS = [
      "for (int64_t j = c; j < d; j++) U[c * d + j] = M[c * d + j] / r;",
      "for (int64_t j = c; j < d; j++) U[c * d + j] = M[c * d + j] / p;",
      [("test_obs_upper_equals_lapack_cholesky_of_inverse", (8, 10.0))]),
-    ("Q4_K offset with the wrong sign", "float q = rintf(((float)w[c] + o) / s);",
-     "float q = rintf(((float)w[c] - o) / s);",
+    ("Q4_K offset with the wrong sign", "float qr = ((float)w[c] + o) / s;",
+     "float qr = ((float)w[c] - o) / s;",
      [("test_q4k_without_compensation_picks_the_nearest_grid_point", ()),
       ("test_q4k_golden_worked_example", ())]),
     ("Q4_K super-block scale over 15 levels", "d = smax / 63.0f;", "d = smax / 15.0f;",

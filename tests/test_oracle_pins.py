@@ -496,6 +496,36 @@ def test_q4k_gptq_lowers_the_output_error_of_round_to_nearest():
     assert oracle.output_mse(W, gq["W_hat"], H, 4096) < 0.8 * oracle.output_mse(W, rt["W_hat"], H, 4096)
 
 
+def test_q4k_act_order_relabeling_equivariance():
+    """P-h on the Q4_K grid: relabeling the input channels (W's columns and
+    H's rows and columns by one permutation) relabels the original-order
+    outputs the same way and leaves every processing-order output unchanged;
+    and a diagonal already in descending order gives the identity order, the
+    same result as no activation order.  This pins the un-permutation of the
+    act_order path."""
+    W, H, _ = _q4k_layer(34, d_out=12, d_in=512, n=4096)
+    P = np.random.default_rng(8).permutation(512)
+    p1, U1, _, _ = oracle.prepare(H, 0.01, True)
+    p2, U2, _, _ = oracle.prepare(H[np.ix_(P, P)], 0.01, True)
+    np.testing.assert_array_equal(P[p2], p1)
+    r1 = oracle.quantize_q4k(W, U1, p1)
+    r2 = oracle.quantize_q4k(W[:, P], U2, p2)
+    np.testing.assert_array_equal(r2["codes"], r1["codes"][:, P])
+    np.testing.assert_array_equal(r2["W_hat"], r1["W_hat"][:, P])
+    np.testing.assert_array_equal(r2["block_of"], r1["block_of"][P])
+    for k in ("codes_perm", "sc6", "m6", "d", "dmin"):
+        np.testing.assert_array_equal(r2[k], r1[k])
+    order = np.argsort(-np.diag(H), kind="stable")
+    Hs, Ws = H[np.ix_(order, order)], W[:, order]
+    pa, Ua, _, _ = oracle.prepare(Hs, 0.01, True)
+    np.testing.assert_array_equal(pa, np.arange(512))
+    ra, rb = oracle.quantize_q4k(Ws, Ua, pa), oracle.quantize_q4k(Ws, Ua, None)
+    for k in ("codes", "sc6", "m6", "d", "dmin", "W_hat"):
+        np.testing.assert_array_equal(ra[k], rb[k])
+    # the un-permuted codes are the processing-order codes put back in place
+    np.testing.assert_array_equal(r1["codes"][:, p1], r1["codes_perm"])
+
+
 def test_q4k_golden_worked_example():
     """A hand-derived super-block (tests/golden/q4k_case.json): every binary32
     step is exact, one value sits on a rounding tie, one block sets both
