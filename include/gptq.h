@@ -18,7 +18,15 @@
  *
  * Conventions shared by every call:
  *   - Pointers are DEVICE pointers unless a parameter says "host".  The caller
- *     owns every buffer; the library allocates no device memory in any call.
+ *     owns every buffer.  No call allocates device memory for its data (the
+ *     workspace is the caller's).  The only allocations are made by the CUDA
+ *     runtime on the library's behalf: the module's static data (the device
+ *     status word; the static scratch of gptq_quantize_static_scratch) when its
+ *     device code is first loaded on a device, the instantiation of a cached
+ *     CUDA graph the first time gptq_prepare / gptq_quantize /
+ *     gptq_quantize_q4k meet a new set of arguments (at most 16 are kept),
+ *     and one pinned host word (cudaMallocHost) per cached graph and per
+ *     calling thread for the status gptq_prepare reads back.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are stream-ordered and asynchronous unless stated.
  *   - Matrices are row-major.  W is [d_out, d_in] (PyTorch Linear layout; a
@@ -47,7 +55,9 @@ typedef enum {
     GPTQ_ERR_CUDA = 4,        /* a CUDA runtime call failed                    */
     GPTQ_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up            */
     GPTQ_ERR_WORKSPACE = 6,   /* workspace pointer NULL/misaligned or too small */
-    GPTQ_ERR_UNSUPPORTED = 7  /* device is not sm_100                          */
+    GPTQ_ERR_UNSUPPORTED = 7, /* device is not sm_100                          */
+    GPTQ_ERR_NO_MEMORY = 8    /* the static scratch could not be created (only
+                                 gptq_quantize_static_scratch)                 */
 } gptq_status;
 
 /* Static English text for a status code.  Never NULL. */
@@ -89,6 +99,10 @@ size_t gptq_workspace_min_bytes(int64_t d_out, int64_t d_in, int block_size);
  *   H         float32 [d_in, d_in], IN/OUT, full symmetric matrix.  The caller
  *             zero-initialises it before the first chunk.  On return both
  *             triangles hold the sum (bitwise symmetric).  16-byte aligned.
+ *             While the call runs, the strictly lower triangle is scratch
+ *             (ordering counters); it is rewritten from the upper triangle
+ *             before the call's work on `stream` ends.  The sums are added in
+ *             a fixed order, so the same H and X give the same bits every run.
  *   X         bfloat16 bit patterns [n_tokens, d_in], row-major, 16-byte
  *             aligned.  Products of bf16 values are exact; sums are float32
  *             (tensor cores, tcgen05 kind::f16, accumulating in TMEM).
@@ -162,7 +176,10 @@ int gptq_hessian_accumulate_f32(float *H, const float *X, int64_t n_tokens, int6
  *   workspace  >= gptq_workspace_bytes(0, d_in, 1) bytes.
  * Synchronises `stream` once to read the factorisation status.  Returns
  * GPTQ_ERR_NOT_PD if mean(diag H) <= 0 or a pivot is not positive,
- * GPTQ_ERR_NONFINITE if H holds NaN/Inf on its diagonal.
+ * GPTQ_ERR_NONFINITE if H holds NaN/Inf on its diagonal.  Deterministic: the
+ * same H gives the same bits.  One call runs at a time per device: calls of a
+ * device share its internal side streams, so a concurrent call (another host
+ * thread, another stream) waits inside the library until the first returns.
  */
 int gptq_prepare(const float *H, int64_t d_in, float damp, int act_order, int32_t *perm,
                  float *Hinv_chol, void *workspace, size_t ws_bytes, void *stream);
@@ -182,7 +199,11 @@ int gptq_prepare(const float *H, int64_t d_in, float damp, int act_order, int32_
  *   W           float32 [d_out, d_in] IN/OUT, original column order.  On
  *               return it holds the dequantized weights W^ (original order).
  *   Hinv_chol   U from gptq_prepare (processing order).
- *   perm        int32 [d_in] from gptq_prepare, or NULL for identity.
+ *   perm        int32 [d_in] from gptq_prepare, or NULL for identity.  It must
+ *               be a permutation of 0 .. d_in-1; entries out of range or
+ *               columns named twice are detected on the device (status word
+ *               GPTQ_ERR_INVALID_ARG, see gptq_device_status()); the outputs
+ *               are then unspecified, but every access stays in bounds.
  *   bits        1..8 (2, 3, 4 are the GPTQ widths; codes are one byte each).
  *   group_size  > 0 and dividing d_in, or -1 for one (scale, zero) per row
  *               from the original row.  group_size must divide block_size or
@@ -257,7 +278,11 @@ int gptq_quantize_q4k(float *W, const float *Hinv_chol, const int32_t *perm, int
  *     used.
  *   - The first call on each device looks up the array's device address with
  *     that device current (a one-time set-up); make that first call before any
- *     stream capture begins.
+ *     stream capture begins.  CUDA loads device code lazily, so that first
+ *     lookup is also when the array is created on the device: a caller that
+ *     reserves the GPU's memory up front must make its first call before
+ *     reserving.  If the device has no room for it the call returns
+ *     GPTQ_ERR_NO_MEMORY (and leaves no CUDA error pending).
  *   - All calls share the one array, and it keeps whatever the last call left
  *     in it.  Nothing in it needs to start at zero (each call writes every byte
  *     it later reads), but two calls whose work overlaps on the GPU (different

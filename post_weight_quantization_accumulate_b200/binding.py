@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libgptq.so")
 GPTQ_OK = 0
 STATUS_NAMES = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_NOT_PD",
                 3: "GPTQ_ERR_NONFINITE", 4: "GPTQ_ERR_CUDA", 5: "GPTQ_ERR_TIMEOUT",
-                6: "GPTQ_ERR_WORKSPACE", 7: "GPTQ_ERR_UNSUPPORTED"}
+                6: "GPTQ_ERR_WORKSPACE", 7: "GPTQ_ERR_UNSUPPORTED", 8: "GPTQ_ERR_NO_MEMORY"}
 
 # (name, restype, argtypes) of every exported symbol, in header order
 _P, _I64, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t

@@ -113,7 +113,7 @@ int sm_count()
     return g_sm_count[dev];
 }
 
-static int check_device()
+int check_device()
 {
     int dev = 0;
     GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
@@ -202,6 +202,7 @@ const char* gptq_status_string(int status)
         case GPTQ_ERR_TIMEOUT: return "device-side wait timed out";
         case GPTQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case GPTQ_ERR_UNSUPPORTED: return "device is not sm_100 (B200)";
+        case GPTQ_ERR_NO_MEMORY: return "device memory for the library's static scratch could not be created";
         default: return "unknown status";
     }
 }

@@ -32,6 +32,28 @@ int cuda_fail(cudaError_t e);          // stores the message, returns GPTQ_ERR_C
 int cuda_fail_msg(const char* where, cudaError_t e);   // same, naming the failing step
 int* device_status_ptr();              // status word of the current device (device memory)
 int sm_count();                        // SMs of the current device
+int check_device();                    // GPTQ_ERR_UNSUPPORTED unless the current device is sm_100
+
+// Launches kernel `k` on `stream`; with `pdl` as a programmatic dependent
+// launch: the kernel may start while the previous kernel on the stream is
+// still running, once every CTA of that kernel has executed pdl_trigger(), and
+// must call pdl_wait() before it touches anything the previous kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     bool pdl, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
 
 #define GPTQ_LAUNCH_CHECK()                                   \
     do {                                                      \
@@ -158,6 +180,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+
+// Programmatic dependent launch, device side.  pdl_wait: returns once the
+// previous kernel on the stream has completed and its writes are visible (at
+// once for a kernel launched without the attribute).  pdl_trigger: this CTA
+// lets the next kernel start; the next kernel's CTAs may occupy free SMs and
+// run their prologue while this grid still runs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map)
 {

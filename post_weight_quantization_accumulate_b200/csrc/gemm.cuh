@@ -24,10 +24,13 @@ enum GemmFlags : int {
 // A_lo, B_lo (optional, same layout and strides as A and B): the operands'
 // low parts x - trunc_tf32(x), prepared by the caller; with both given the
 // tensor-core path skips its conversion pass and uses 128 x 256 tiles.
+// pdl: launch the tensor-core product as a programmatic dependent launch (its
+// prologue overlaps the previous kernel on the stream; see launch_k).
 int launch_sgemm(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                  int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                  int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream,
-                 int max_ctas = 0, const float* A_lo = nullptr, const float* B_lo = nullptr);
+                 int max_ctas = 0, const float* A_lo = nullptr, const float* B_lo = nullptr,
+                 bool pdl = false);
 
 int launch_sgemm_simt(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                       int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
@@ -35,7 +38,8 @@ int launch_sgemm_simt(bool trans_b, int M, int N, int K, float alpha, const floa
 int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                    int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                    int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream,
-                   int max_ctas = 0, const float* A_lo = nullptr, const float* B_lo = nullptr);
+                   int max_ctas = 0, const float* A_lo = nullptr, const float* B_lo = nullptr,
+                   bool pdl = false);
 bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, int64_t ldb,
                        int64_t sB, int batch);
 

@@ -200,6 +200,11 @@ __global__ void __launch_bounds__(TTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Under a programmatic dependent launch the set-up above overlaps the tail
+    // of the previous kernel; its outputs (the A operand, C) are touched only
+    // after this wait.  The next kernel may then start its own set-up.
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tbase = S.tmem_base;
     volatile int* abort = &S.abort;
     int* status = g.status;
@@ -542,7 +547,7 @@ static int set_smem_attr()
 int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                    int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                    int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream, int max_ctas,
-                   const float* A_lo, const float* B_lo)
+                   const float* A_lo, const float* B_lo, bool pdl)
 {
     if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
     const bool prelo = A_lo && B_lo;
@@ -597,11 +602,11 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;
     const int grid = static_cast<int>(units < cap ? units : cap);
     if (prelo)
-        gemm_tc_kernel<256, true><<<grid, TTHREADS, gemm_smem_bytes<256, true>(), stream>>>(
-            mA, mB, mAlo, mBlo, mC, g);
+        GPTQ_CUDA_CHECK(launch_k(gemm_tc_kernel<256, true>, dim3(grid), dim3(TTHREADS),
+                                 gemm_smem_bytes<256, true>(), stream, pdl, mA, mB, mAlo, mBlo, mC, g));
     else
-        gemm_tc_kernel<128, false><<<grid, TTHREADS, gemm_smem_bytes<128, false>(), stream>>>(
-            mA, mB, mAlo, mBlo, mC, g);
+        GPTQ_CUDA_CHECK(launch_k(gemm_tc_kernel<128, false>, dim3(grid), dim3(TTHREADS),
+                                 gemm_smem_bytes<128, false>(), stream, pdl, mA, mB, mAlo, mBlo, mC, g));
     GPTQ_LAUNCH_CHECK();
     return GPTQ_OK;
 }

@@ -43,9 +43,19 @@
 //    round trip measured faster than more, smaller stages) and two TMEM chain
 //    buffers (2 x 256
 //    columns) let the promotion of one chain overlap the MMAs of the next.
-//  * Every mbarrier wait is bounded; a time-out records GPTQ_ERR_TIMEOUT and
-//    ends the role; both CTAs meet at a cluster barrier before the pair frees
-//    its tensor memory.
+//  * Flush order is fixed, so H is bitwise reproducible: the flush of span s
+//    of a tile waits until the flushes of spans 0 .. s-1 of that tile have
+//    landed (a turn counter per tile and CTA, counting epilogue-warp flushes).
+//    The counters live in H itself, in the strictly lower triangle below the
+//    first tile row (rows 256.., columns 0..255), which no tile flushes into
+//    and which the mirror copy overwrites at the end of the call; each launch
+//    zeroes the ones it uses.  A unit only ever waits on a unit with a smaller
+//    index, and each pair walks its units in increasing order, so with every
+//    pair resident the waits end.  A one-tile H (d <= 256) has no room for
+//    counters and runs its tokens as one unit.
+//  * Every mbarrier and counter wait is bounded; a time-out records
+//    GPTQ_ERR_TIMEOUT (a timed-out turn wait still flushes, unordered); both
+//    CTAs meet at a cluster barrier before the pair frees its tensor memory.
 #include "common.cuh"
 
 #include <algorithm>
@@ -188,6 +198,42 @@ __device__ __forceinline__ void tile_coords(int tile, int n_t, int& ti, int& tj)
     }
     ti = n_t - 1;
     tj = n_t - 1;
+}
+
+// Turn counter of (tile, CTA rank) inside H's strictly lower triangle.
+__device__ __forceinline__ int* turn_counter(float* H, int d, int tile, uint32_t rank)
+{
+    const int c = 2 * tile + static_cast<int>(rank);
+    return reinterpret_cast<int*>(H + static_cast<int64_t>(kTile + c / kTile) * d + c % kTile);
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Waits (lane 0 of the calling warp) until *ctr >= target; bounded like the
+// mbarrier waits.  Returns false on a time-out (recorded in the status word).
+__device__ __forceinline__ bool wait_turn(const int* ctr, int target, int* status)
+{
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(ctr) < target) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            record_status(status, GPTQ_ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(256);
+    }
+    return true;
+}
+
+__global__ void zero_turns_kernel(float* H, int d, int n)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c < n) *reinterpret_cast<int*>(H + static_cast<int64_t>(kTile + c / kTile) * d + c % kTile) = 0;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -338,6 +384,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int ti, tj;
             tile_coords(u % n_tiles, n_t, ti, tj);
             const int row = ti * kTile + row_in_tile;
+            int* turn = n_split > 1 ? turn_counter(H, d, u % n_tiles, rank) : nullptr;
+            if (turn) {
+                // the 8 epilogue warps of this CTA flushed every earlier span
+                if (lane == 0) wait_turn(turn, (u / n_tiles) * kEpiWarps, status);
+                __syncwarp();
+            }
 #pragma unroll
             for (int c = 0; c < kBN / 64; ++c) {
                 const int col0 = tj * kTile + h * (kBN / 2) + c * 32;
@@ -354,6 +406,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int m = 0; m < 32; ++m)
                             if (m < d - col0) atomicAdd(dst + m, 2.f * acc[c * 32 + m]);
                     }
+                }
+            }
+            if (turn) {
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();   // this warp's additions land before its turn is passed on
+                    atomicAdd(turn, 1);
                 }
             }
         }
@@ -450,7 +509,14 @@ int launch_hessian_upper(float* H, const uint16_t* X, int64_t n_rows, int64_t d,
     const int64_t want = 8 * static_cast<int64_t>(sm_count() / 2);
     int span = kSpanMax;
     while (span > kSpanMin && n_tiles * ((n_rows + span - 1) / span) < want) span /= 2;
+    if (n_t == 1) span = static_cast<int>(n_rows);   // no room for turn counters: one unit
     const int n_split = static_cast<int>((n_rows + span - 1) / span);
+    if (n_split > 1) {
+        // turn counters of this launch, inside H's strictly lower triangle
+        const int n = 2 * n_tiles;
+        zero_turns_kernel<<<(n + 255) / 256, 256, 0, stream>>>(H, static_cast<int>(d), n);
+        GPTQ_LAUNCH_CHECK();
+    }
     const int64_t units = static_cast<int64_t>(n_tiles) * n_split;
     // pairs that can be resident at once (a GPC with an odd number of free
     // SMs holds one pair less than half its SMs)

@@ -27,7 +27,11 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name only stands for the variable; its device address has to be
-// looked up once per device, with that device current.
+// looked up once per device, with that device current.  CUDA loads a module's
+// device code lazily, so on each device this lookup is also the moment the
+// array itself is created: it can fail for lack of device memory, which is
+// reported as GPTQ_ERR_NO_MEMORY (and the runtime's error is cleared, so it
+// does not surface in the caller's next CUDA call).
 int scratch_address(void** out)
 {
     int dev = 0;
@@ -38,7 +42,11 @@ int scratch_address(void** out)
     if (!g_scratch_addr[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_quantize_scratch);
-        if (e != cudaSuccess) return gptq::cuda_fail(e);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            const int rc = gptq::cuda_fail_msg("creating the static scratch", e);
+            return e == cudaErrorMemoryAllocation ? GPTQ_ERR_NO_MEMORY : rc;
+        }
         if (!p) return GPTQ_ERR_CUDA;
         g_scratch_addr[dev] = p;
     }
@@ -68,8 +76,12 @@ extern "C" int gptq_quantize_static_scratch(float* W, const float* Hinv_chol,
     // before anything touches the device.
     if (gptq::quantize_workspace_min_bytes(d_out, d_in) > GPTQ_STATIC_SCRATCH_BYTES)
         return GPTQ_ERR_WORKSPACE;
+    // the device check comes before the lookup: on a GPU this library has no
+    // code for, the lookup itself would fail with a less telling error
+    int rc = gptq::check_device();
+    if (rc != GPTQ_OK) return rc;
     void* scratch = nullptr;
-    int rc = scratch_address(&scratch);
+    rc = scratch_address(&scratch);
     if (rc != GPTQ_OK) return rc;
     // Nothing in the scratch has to start at zero: every byte gptq_quantize
     // reads from its workspace is written earlier in the same call.  The

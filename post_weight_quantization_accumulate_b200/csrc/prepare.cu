@@ -658,12 +658,15 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
     GPTQ_LAUNCH_CHECK();
     if (d <= kGatherSmemMax) {
         const size_t sm = static_cast<size_t>(d) * sizeof(float);
-        static bool attr = false;
-        if (!attr) {
+        static bool attr[64] = {};   // per device: the attribute is set per context
+        int dev = 0;
+        GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
+        if (dev < 0 || dev >= 64) return GPTQ_ERR_UNSUPPORTED;
+        if (!attr[dev]) {
             GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gather_rev_kernel,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  kGatherSmemMax * static_cast<int>(sizeof(float))));
-            attr = true;
+            attr[dev] = true;
         }
         gather_rev_kernel<<<std::min(d, nsm * 8), 256, sm, stream>>>(H, d, perm, hdr, A);
     } else {
@@ -746,9 +749,22 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
     return GPTQ_OK;
 }
 
+// One factorisation in flight per device: the calls of a device share its
+// side streams and events (and, when graphs are off or the caller's stream is
+// being captured, enqueue on them directly), so a second call -- another host
+// thread, another stream -- waits here until the first has synchronised.
+static std::mutex& prepare_mutex()
+{
+    static std::mutex mu[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    return mu[dev];
+}
+
 int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* perm, float* U,
                 void* workspace, cudaStream_t stream, int* host_status, bool graphed)
 {
+    std::lock_guard<std::mutex> one_in_flight(prepare_mutex());
     uint32_t damp_bits = 0;
     static_assert(sizeof damp_bits == sizeof damp, "float is 32-bit");
     memcpy(&damp_bits, &damp, sizeof damp);

@@ -153,6 +153,28 @@ __device__ __forceinline__ float div_rn(float w, float s, float rs)
     return fmaf(fmaf(-t, s, w), rs, t);
 }
 
+// Operands of the quotient w / s for one group.  The correction above needs
+// the residual w - t s exactly and a finite RN(1 / s); both hold while s and
+// the residual stay clear of the subnormal range, i.e. for s >= 2^-100 (the
+// residual's lowest bit is at least 2^-47 s when |w / s| >= 1/2, where the
+// rounding is decided).  A group whose range is that tiny (1 / s overflows
+// below 2^-128) has its scale and every quotient numerator lifted by 2^100:
+// multiplying both by a power of two is exact and leaves w / s unchanged.
+struct QuotOp {
+    float f;    // 1 or 2^100
+    float s;    // s * f
+    float rs;   // RN(1 / (s * f))
+};
+
+__device__ __forceinline__ QuotOp quot_op(float s)
+{
+    const float f = s < 0x1p-60f ? 0x1p100f : 1.f;
+    const float sf = s * f;
+    return {f, sf, 1.f / sf};
+}
+
+__device__ __forceinline__ float quot(float w, const QuotOp& o) { return div_rn(w * o.f, o.s, o.rs); }
+
 // Scale and zero of the group starting at in-block column c, from one row's
 // current values: each part reduces its registers whose column lies in
 // [c, c + gs) and below bw, then the QTPR parts of the row pair combine.
@@ -248,6 +270,12 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
             bulk_load(qsm_raw + S * UCH_BYTES, src + S * UCH_FLOATS, UCH_BYTES, &bars[S]);
         }
     }
+    // Under a programmatic dependent launch everything above (the U block is
+    // laid out before the first block's launch) overlaps the previous kernel,
+    // the lazy-batch product that corrects this block's columns; W is read
+    // only after it completes.  The next product may start its set-up now.
+    pdl_wait();
+    pdl_trigger();
 
     const int pair = tid / QTPR, part = tid % QTPR;
     const int lane = tid & 31;
@@ -377,7 +405,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                 }
         }
     }
-    float rs[2] = {1.f / s[0], 1.f / s[1]};
+    QuotOp qo[2] = {quot_op(s[0]), quot_op(s[1])};
     const int gs_in = (a.gs > 0 && a.gs <= a.block) ? a.gs : 0;
     int next_group = gs_in ? 0 : 1 << 30;
 
@@ -406,7 +434,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                 } else {
                     group_grid(w[h], part, cbase, gs_in, bw, maxq, s[h], z[h]);
                 }
-                rs[h] = 1.f / s[h];
+                qo[h] = quot_op(s[h]);
                 if (valid[h] && part == 0) {
                     const int g = (j0 + cbase) / gs_in;
                     a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g] = s[h];
@@ -443,7 +471,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     group_grid(w[h], part, c, gs_in, bw, maxq, s[h], z[h]);
-                    rs[h] = 1.f / s[h];
+                    qo[h] = quot_op(s[h]);
                     if (valid[h] && part == 0) {
                         const int g = (j0 + c) / gs_in;
                         a.scales[static_cast<int64_t>(r[h]) * a.n_groups + g] = s[h];
@@ -460,10 +488,10 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                 // integer-valued floats, q - z = clamp(rint(w / s), -z, maxq - z)
                 float q, what;
                 if (kQ4K) {   // q = clamp(rint((w + o) / s), 0, 15), w^ = s q - o
-                    q = fminf(fmaxf(rintf(div_rn(wc + z[h], s[h], rs[h])), 0.f), 15.f);
+                    q = fminf(fmaxf(rintf(quot(wc + z[h], qo[h])), 0.f), 15.f);
                     what = fmaf(s[h], q, -z[h]);
                 } else {
-                    const float qz = fminf(fmaxf(rintf(div_rn(wc, s[h], rs[h])), -z[h]), maxq - z[h]);
+                    const float qz = fminf(fmaxf(rintf(quot(wc, qo[h])), -z[h]), maxq - z[h]);
                     q = qz + z[h];
                     what = s[h] * qz;
                 }
@@ -534,7 +562,8 @@ __global__ void row_grid_kernel(const float* __restrict__ W, int d_out, int d_in
     }
 }
 
-// inv[perm[k]] = k, with a range check of perm.
+// inv[perm[k]] = k, with a range check of perm (inv starts as all -1, so a
+// column that no entry of perm names stays -1 and finish_kernel reports it).
 __global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int d, int32_t* __restrict__ inv,
                                    int* status)
 {
@@ -564,11 +593,13 @@ __global__ void gather_cols_kernel(const float* __restrict__ W, int d_out, int d
 }
 
 // Original-order outputs: codes, packed nibbles, and (with a permutation) W^.
-// One thread per pair of original columns (2i, 2i+1).
+// One thread per pair of original columns (2i, 2i+1).  A column missing from
+// the permutation (perm not a bijection) records GPTQ_ERR_INVALID_ARG; its
+// outputs are then unspecified, but every access stays in bounds.
 __global__ void finish_kernel(const uint8_t* __restrict__ codes_p, const float* __restrict__ Wp,
                               const int32_t* __restrict__ inv, int d_out, int d_in,
                               float* __restrict__ W, uint8_t* __restrict__ codes,
-                              uint8_t* __restrict__ packed)
+                              uint8_t* __restrict__ packed, int* status)
 {
     const int half = d_in / 2;
     const int64_t n = static_cast<int64_t>(d_out) * half;
@@ -579,8 +610,11 @@ __global__ void finish_kernel(const uint8_t* __restrict__ codes_p, const float* 
         const int c0 = 2 * i, c1 = 2 * i + 1;
         int k0 = inv ? inv[c0] : c0;
         int k1 = inv ? inv[c1] : c1;
-        k0 = (k0 < 0 || k0 >= d_in) ? 0 : k0;   // a malformed permutation stays in bounds
-        k1 = (k1 < 0 || k1 >= d_in) ? 0 : k1;
+        if (k0 < 0 || k0 >= d_in || k1 < 0 || k1 >= d_in) {   // a malformed permutation
+            if (r == 0) record_status(status, GPTQ_ERR_INVALID_ARG);
+            k0 = (k0 < 0 || k0 >= d_in) ? 0 : k0;
+            k1 = (k1 < 0 || k1 >= d_in) ? 0 : k1;
+        }
         const int64_t ro = r * d_in;
         const uint8_t q0 = codes_p[ro + k0], q1 = codes_p[ro + k1];
         if (codes) {
@@ -633,16 +667,18 @@ __device__ __forceinline__ float st_unif(uint64_t k) { return (st_mix(k) >> 8) *
 
 __device__ unsigned long long g_quotient_bad;   // mismatch count of the self-test
 
-// div_rn against IEEE division on three operand families: s log-uniform in
-// [2^-40, 2^20] with |w / s| < 2^12, s with an all-ones significand, and w
-// within 4 ulps of (n + 1/2) s (quotients next to a rounding tie of rint).
+// The column loop's quotient (quot after quot_op) against IEEE division on
+// four operand families: s log-uniform in [2^-40, 2^20] with |w / s| < 2^12,
+// s with an all-ones significand, w within 4 ulps of (n + 1/2) s (quotients
+// next to a rounding tie of rint), and tiny scales, s log-uniform in
+// [2^-149, 2^-60] (subnormals included) with w within 4 ulps of (n + 1/2) s.
 __global__ void quotient_selftest_kernel(uint64_t seed, int64_t n, unsigned long long* bad)
 {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     unsigned long long local = 0;
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
         const uint64_t k = (seed << 40) ^ (4 * static_cast<uint64_t>(i));
-        const int mode = static_cast<int>(i % 3);
+        const int mode = static_cast<int>(i % 4);
         float s, w;
         if (mode == 0) {
             s = exp2f(-40.f + 60.f * st_unif(k));
@@ -653,13 +689,15 @@ __global__ void quotient_selftest_kernel(uint64_t seed, int64_t n, unsigned long
             s = __uint_as_float((static_cast<uint32_t>(e + 127) << 23) | m);
             w = s * (st_unif(k + 1) * 600.f - 300.f);
         } else {
-            s = exp2f(-20.f + 24.f * st_unif(k));
+            s = mode == 2 ? exp2f(-20.f + 24.f * st_unif(k)) : exp2f(-149.f + 89.f * st_unif(k));
             const float m = floorf(st_unif(k + 1) * 600.f - 300.f);
             const float w0 = (m + 0.5f) * s;
             w = __uint_as_float(__float_as_uint(w0) + static_cast<int>(st_mix(k + 3) % 9) - 4);
         }
-        const float rs = 1.f / s;
-        if (div_rn(w, s, rs) != __fdiv_rn(w, s)) ++local;
+        // skip an ulp step below a zero numerator's bit pattern, and a scale
+        // that came out as zero
+        if (!isfinite(w) || !(s > 0.f)) continue;
+        if (quot(w, quot_op(s)) != __fdiv_rn(w, s)) ++local;
     }
     if (local) atomicAdd(bad, local);
 }
@@ -724,6 +762,10 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
 {
     auto mark = [&](int c) { return marks ? marks->mark(stream, c) : GPTQ_OK; };
     if (int rc = mark(0)) return rc;
+    // The column-loop kernels and the lazy-batch products alternate on the
+    // stream as programmatic dependent launches, each one's set-up overlapping
+    // the previous one's tail -- except when events are recorded between them.
+    const bool pdl = false && marks == nullptr;
     const int d_out = static_cast<int>(d_out64), d_in = static_cast<int>(d_in64);
     const size_t n = static_cast<size_t>(d_out) * d_in;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -774,6 +816,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
 
     float* work = W;
     if (perm) {
+        GPTQ_CUDA_CHECK(cudaMemsetAsync(inv, 0xFF, static_cast<size_t>(d_in) * sizeof(int32_t), stream));
         invert_perm_kernel<<<(d_in + 255) / 256, 256, 0, stream>>>(perm, d_in, inv, status);
         GPTQ_LAUNCH_CHECK();
         gather_cols_kernel<<<nsm * 8, 256, 0, stream>>>(W, d_out, d_in, perm, Wp);
@@ -810,12 +853,9 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                     q4k ? q4k->sc6 : nullptr, q4k ? q4k->m6 : nullptr,
                     q4k ? q4k->dsup : nullptr, q4k ? q4k->dmin : nullptr};
             if (int rc = mark(0)) return rc;
-            if (q4k)
-                gptq_block_kernel<false, true><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
-            else if (groups_in_step)
-                gptq_block_kernel<true, false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
-            else
-                gptq_block_kernel<false, false><<<grid, QTHREADS, kBlockSmem, stream>>>(a);
+            auto kern = q4k ? gptq_block_kernel<false, true>
+                            : (groups_in_step ? gptq_block_kernel<true, false> : gptq_block_kernel<false, false>);
+            GPTQ_CUDA_CHECK(launch_k(kern, dim3(grid), dim3(QTHREADS), kBlockSmem, stream, pdl, a));
             GPTQ_LAUNCH_CHECK();
             if (int rc = mark(1)) return rc;
             const int rest_in = J1 - j0 - bw;
@@ -823,7 +863,8 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                 const int64_t uo = static_cast<int64_t>(j0) * d_in + j0 + bw;
                 int rc = launch_sgemm(false, d_out, rest_in, bw, -1.f, E + (j0 - J0), kOuterMax, 0,
                                       U + uo, d_in, 0, 1.f, work + j0 + bw, d_in, 0, 1, 0, stream, 0,
-                                      E_lo ? E_lo + (j0 - J0) : nullptr, U_lo ? U_lo + uo : nullptr);
+                                      E_lo ? E_lo + (j0 - J0) : nullptr, U_lo ? U_lo + uo : nullptr,
+                                      pdl);
                 if (rc) return rc;
                 if ((rc = mark(2))) return rc;
             }
@@ -833,14 +874,14 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
             const int64_t uo = static_cast<int64_t>(J0) * d_in + J1;
             int rc = launch_sgemm(false, d_out, rest, J1 - J0, -1.f, E, kOuterMax, 0, U + uo, d_in, 0,
                                   1.f, work + J1, d_in, 0, 1, 0, stream, 0, E_lo,
-                                  U_lo ? U_lo + uo : nullptr);
+                                  U_lo ? U_lo + uo : nullptr, pdl);
             if (rc) return rc;
             if ((rc = mark(2))) return rc;
         }
     }
     if (codes || packed || perm) {
         finish_kernel<<<nsm * 8, 256, 0, stream>>>(codes_p, Wp, perm ? inv : nullptr, d_out, d_in,
-                                                   W, codes, packed);
+                                                   W, codes, packed, status);
         GPTQ_LAUNCH_CHECK();
     }
     if (g_idx) {

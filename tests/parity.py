@@ -4,11 +4,13 @@ method lives here: only element-wise comparisons and the tolerances).
 Tolerances of this path (the stated parity bar):
   H          relative Frobenius error <= 1e-5 (fp32 accumulation of exact bf16 products)
   codes      identical on >= 99.9% of entries (2-4 bits; the stated widths);
-             every mismatch exactly one level.  For wider codes the bar scales
-             with the number of grid levels, 1 - 1e-3 * 2^(bits - 4): with the
-             same float32 rounding noise in the compensated weights, the chance
-             that a value sits within that noise of a rounding boundary grows
-             with 1/scale, i.e. with 2^bits.
+             every mismatch exactly one level.  Wider codes (up to 8 bits, not
+             among the stated widths) must match on >= 99.8%: a code that sits
+             at a rounding tie (and with 2^bits levels the ties are 2^bits
+             times denser) changes the error carried along the rest of its row,
+             so one tie costs up to a row of codes; on the 256 x 512 8-bit cases
+             the lowest measured agreement is 99.80%, every diverging row
+             starting at a tie (checked below for every width).
   scales/zeros  within 1e-5 relative, except in a row after an earlier code
                 mismatch (processing order), which the mismatch explains
   output MSE relative difference <= 0.5%
@@ -28,8 +30,11 @@ def rel_fro(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
+CODE_MATCH_WIDE = 0.998
+
+
 def code_match_min(bits: int) -> float:
-    return CODE_MATCH if bits <= 4 else 1.0 - (1.0 - CODE_MATCH) * 2 ** (bits - 4)
+    return CODE_MATCH if bits <= 4 else CODE_MATCH_WIDE
 
 
 TIE_TOL = 1e-3   # a decision value this close to a .5 boundary is a rounding tie
@@ -94,3 +99,53 @@ def check_mse(mse_gpu, mse_ref, where=""):
     rel = abs(mse_gpu - mse_ref) / mse_ref
     assert rel <= MSE_RTOL, f"{where}: output MSE {mse_gpu} vs {mse_ref} (rel {rel:.2e})"
     return rel
+
+
+def check_q4k(g, ref, perm, where=""):
+    """Device outputs of GPTQ onto the two-level Q4_K grid (`g`: codes in
+    original column order; sc6, m6, dsup, dmin in processing order) against
+    the checker's result `ref` (oracle.quantize_q4k, with its decision values
+    qraw, scraw, mraw).
+
+    The same bar as the one-level grid.  Walking a row in processing order,
+    its first divergence must be a 6-bit block level (sc6 or m6) or a code
+    that differs by exactly one and whose decision value in the checker lies
+    within TIE_TOL of a rounding tie; a super-block scale (d or dmin) may
+    differ by more than 1e-5 only after such a divergence.  Codes, sc6 and m6
+    agree on >= 99.9% of entries and every code mismatch is one level."""
+    d_in = g["codes"].shape[1]
+    cg = np.asarray(g["codes"]).astype(np.int32)[:, perm]
+    cr = np.asarray(ref["codes_perm"]).astype(np.int32)
+    scg, scr = g["sc6"].astype(np.int32), ref["sc6"].astype(np.int32)
+    mg, mr = g["m6"].astype(np.int32), ref["m6"].astype(np.int32)
+    dg, dr = np.asarray(g["dsup"], np.float64), np.asarray(ref["d"], np.float64)
+    dmg, dmr = np.asarray(g["dmin"], np.float64), np.asarray(ref["dmin"], np.float64)
+    c_mis = cg != cr
+    b_mis = (scg != scr) | (mg != mr)
+    s_bad = (np.abs(dg - dr) > SZ_RTOL * np.abs(dr)) | (np.abs(dmg - dmr) > SZ_RTOL * np.abs(dmr))
+    rows = np.nonzero(c_mis.any(axis=1) | b_mis.any(axis=1) | s_bad.any(axis=1))[0]
+    for r in rows:
+        c1 = int(np.argmax(c_mis[r])) if c_mis[r].any() else d_in
+        b1 = 32 * int(np.argmax(b_mis[r])) if b_mis[r].any() else d_in
+        s1 = 256 * int(np.argmax(s_bad[r])) if s_bad[r].any() else d_in
+        assert s1 > min(b1, c1) or s1 == d_in, (
+            f"{where}: row {r} super-block {s1 // 256}: d {dg[r, s1 // 256]} / {dr[r, s1 // 256]}, "
+            f"dmin {dmg[r, s1 // 256]} / {dmr[r, s1 // 256]} with no earlier divergence")
+        if b1 <= c1:                      # first divergence: a block's 6-bit levels
+            b = b1 // 32
+            for lv_g, lv_r, raw, name in ((scg, scr, ref["scraw"], "sc6"), (mg, mr, ref["mraw"], "m6")):
+                if lv_g[r, b] != lv_r[r, b]:
+                    assert abs(lv_g[r, b] - lv_r[r, b]) == 1 and _near_tie(raw[r, b]), (
+                        f"{where}: row {r} block {b}: {name} {lv_g[r, b]} vs {lv_r[r, b]} "
+                        f"(checker raw {raw[r, b]})")
+        else:                             # first divergence: a code
+            assert abs(cg[r, c1] - cr[r, c1]) == 1 and _near_tie(ref["qraw"][r, c1]), (
+                f"{where}: row {r} col {c1} (processing order): code {cg[r, c1]} vs {cr[r, c1]} "
+                f"(checker (w + o) / s = {ref['qraw'][r, c1]})")
+    rates = {k: 1.0 - float(m.mean()) for k, m in (("codes", c_mis), ("sc6", scg != scr), ("m6", mg != mr))}
+    print(f"[parity] {where}: Q4_K match {rates}, rows diverging {rows.size} (each from a rounding tie)")
+    for k, v in rates.items():
+        assert v >= CODE_MATCH, f"{where}: {k} match {v:.6f} < {CODE_MATCH}"
+    if c_mis.any():
+        assert np.abs(cg - cr)[c_mis].max() == 1, f"{where}: a Q4_K code differs by more than one level"
+    return rates

@@ -1,8 +1,12 @@
 """GPTQ onto the two-level Q4_K grid on the device against the float64
 checker, given the device's own factor and order (the staged parity of the
-one-level grid): codes and 6-bit levels agree except at rounding ties (at
-least 99.9%), super-block scales to 1e-5, the layer-output MSE to 1%; the
-device's outputs obey w^ = d sc q - dmin m exactly."""
+one-level grid, with the same bar): walking each row in processing order,
+its first divergence is a code or a 6-bit level one step off at a rounding
+tie; codes, sc6 and m6 agree on >= 99.9% of entries, every code mismatch is
+one level, super-block scales agree to 1e-5 before a row's first divergence,
+and the layer-output MSE agrees to 0.5%.  The device's outputs obey
+w^ = d sc q - dmin m.  A full-size 4096 x 4096 layer is checked on sampled
+rows."""
 import numpy as np
 import pytest
 import torch
@@ -53,17 +57,11 @@ def test_q4k_matches_checker(d_out, d_in, act_order):
     W, g = _run(d_out, d_in, 4096, act_order, d_in + d_out)
     perm = g["perm"] if act_order else None
     ref = oracle.quantize_q4k(W, g["U"], perm)
-    assert (g["codes"] == ref["codes"]).mean() >= P.CODE_MATCH
-    assert (g["sc6"] == ref["sc6"]).mean() >= P.CODE_MATCH
-    assert (g["m6"] == ref["m6"]).mean() >= P.CODE_MATCH
-    close = np.abs(g["dsup"] - ref["d"]) <= 1e-5 * ref["d"]
-    assert close.mean() >= P.CODE_MATCH
-    close = np.abs(g["dmin"] - ref["dmin"]) <= 1e-5 * np.maximum(ref["dmin"], 1e-30)
-    assert close.mean() >= P.CODE_MATCH
+    P.check_q4k(g, ref, g["perm"] if act_order else np.arange(d_in), f"q4k {d_out}x{d_in} ao{act_order}")
     n = 4096
     mse_g = oracle.output_mse(W, g["W_hat"].astype(np.float64), g["H"], n)
     mse_r = oracle.output_mse(W, ref["W_hat"], g["H"], n)
-    assert abs(mse_g - mse_r) <= 0.01 * mse_r, (mse_g, mse_r)
+    P.check_mse(mse_g, mse_r, f"q4k {d_out}x{d_in}")
     # the device's own outputs: levels in range and w^ = scales q - offsets
     assert g["codes"].max() <= 15 and g["sc6"].min() >= 1 and g["sc6"].max() <= 63 and g["m6"].max() <= 63
     blk = np.arange(d_in) // 32
@@ -93,6 +91,35 @@ def test_q4k_through_the_layer_wrapper():
     assert B.gptq_device_status() == 0
     perm = q.perm.cpu().numpy()
     ref = oracle.quantize_q4k(W, q.U.cpu().numpy().astype(np.float64), perm)
-    assert (r["codes"].cpu().numpy() == ref["codes"]).mean() >= P.CODE_MATCH
-    assert (r["sc6"].cpu().numpy() == ref["sc6"]).mean() >= P.CODE_MATCH
+    g = {k: r[k].cpu().numpy() for k in ("codes", "sc6", "m6", "dsup", "dmin")}
+    P.check_q4k(g, ref, perm, "q4k layer wrapper")
     np.testing.assert_array_equal(oracle.unpack_int4(r["packed"].cpu().numpy()), r["codes"].cpu().numpy())
+
+
+@pytest.mark.slow
+def test_q4k_full_size_q_proj_sampled_rows():
+    """The q_proj workload (4096 x 4096, 262144 tokens) onto the Q4_K grid in
+    the launch configuration of the benchmark's layer: sampled rows rerun by
+    the checker with the device's factor, under the same bar."""
+    from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
+    spec = synth.WORKLOADS["q_proj_4096"]
+    xb = synth.x_bf16(spec)
+    W = synth.weight_f32(spec)
+    q = LayerQuantizer(spec.d_out, spec.d_in, 4, 32, 128, spec.damp, spec.act_order)
+    q.reset()
+    q.add_batch(torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16))
+    del xb
+    q.prepare()
+    r = q.quantize_q4k(torch.from_numpy(W).cuda())
+    torch.cuda.synchronize()
+    assert B.gptq_device_status() == 0
+    rows = np.sort(np.random.default_rng(3).choice(spec.d_out, 24, replace=False))
+    perm = q.perm.cpu().numpy()
+    U = q.U.cpu().numpy().astype(np.float64)
+    ref = oracle.quantize_q4k(W[rows].astype(np.float64), U, perm, block=128)
+    g = {k: r[k].cpu().numpy()[rows] for k in ("codes", "sc6", "m6", "dsup", "dmin")}
+    P.check_q4k(g, ref, perm, "q4k q_proj_4096")
+    H64 = q.H.cpu().numpy().astype(np.float64)
+    mse_g = oracle.output_mse(W[rows], r["W_hat"].cpu().numpy()[rows].astype(np.float64), H64, spec.n_tokens)
+    mse_r = oracle.output_mse(W[rows], ref["W_hat"], H64, spec.n_tokens)
+    P.check_mse(mse_g, mse_r, "q4k q_proj_4096")

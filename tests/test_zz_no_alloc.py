@@ -75,14 +75,33 @@ def test_static_scratch_matches_workspace_entry_point_twice_in_a_row():
         for call in range(2):
             W = W0.clone()
             out = _outputs(d_out, d_in, bits, gs)
+            torch.cuda.synchronize()
+            free0, torch0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
             B.gptq_quantize_static_scratch(W, U, perm, bits, gs, 128, out["scales"], out["zeros"],
                                            codes=out["codes"], packed_int4=out["packed_int4"],
                                            g_idx=out["g_idx"], err_sq=out["err_sq"])
+            torch.cuda.synchronize()
+            if call == 1:
+                # once the first call has created the array, a call takes no
+                # device memory: neither from the device nor from torch's pool
+                assert torch.cuda.mem_get_info()[0] == free0
+                assert torch.cuda.memory_allocated() == torch0
             _compare(W_ref, ref, W, out, bits, gs, perm, f"static scratch {d_out}x{d_in} call {call}")
 
 
 def test_static_scratch_refuses_layers_larger_than_the_array():
-    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the size check comes first
-    st = B.lib().gptq_quantize_static_scratch(fake, fake, None, 4096, 11008, 4, 128, 128, None,
-                                               fake, fake, None, None, None, None)
+    """A layer whose working set exceeds the fixed array (4096 x 11008) is
+    refused with GPTQ_ERR_WORKSPACE.  The buffers handed over are real device
+    tensors of the declared shapes, so even a refusal that came too late
+    could not touch memory outside them."""
+    d_out, d_in = 4096, 11008
+    W = torch.zeros(d_out, d_in, device=DEV)
+    U = torch.zeros(d_in, d_in, device=DEV)
+    out = _outputs(d_out, d_in, 4, 128)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = B.lib().gptq_quantize_static_scratch(ptr(W), ptr(U), None, d_out, d_in, 4, 128, 128,
+                                               ptr(out["codes"]), ptr(out["scales"]),
+                                               ptr(out["zeros"]), None, None, None, None)
     assert st == 6  # GPTQ_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert B.gptq_device_status() == 0
