@@ -15,6 +15,15 @@ are resident in HBM before the timed region.  With N > 1 (torchrun), every
 rank quantizes its own independent layer (layers are independent, GPTQ
 overview page "Równoległość"): weak scaling, no collective in the data path.
 
+With --split tokens_rows (torchrun, N ranks) the ranks instead share ONE
+layer: each accumulates the Hessian over its own slice of the tokens, one NCCL
+all-reduce sums H, every rank factorises the same H, and each quantizes its
+own block of rows (GPTQ overview page, "Równoległość"; strong scaling).
+
+The default run also times the other single-GPU workloads of the layer recipe
+once each (down_proj 11008, 70B up_proj, a full Llama-2-7B decoder layer, the
+fp32-activation Hessian) under "by_config" of the same line.
+
 Prints one JSON line (rank 0).  value = quantized weights/s over all ranks.
 """
 from __future__ import annotations
@@ -47,6 +56,13 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="decoder_layer: bits {2,3,4} x group_size {64,128,per-channel}")
+    ap.add_argument("--split", default="layers", choices=["layers", "tokens_rows"],
+                    help="N > 1: an independent layer per rank, or one layer split over the ranks")
+    ap.add_argument("--no-by-config", action="store_true",
+                    help="skip the other workloads in the default run")
+    ap.add_argument("--validate-cost-laws", action="store_true",
+                    help="reference arm: also run the checker's factorisation at full d_in and "
+                         "256 full rows of the column loop, against the sample's extrapolation")
     return ap.parse_args()
 
 
@@ -119,16 +135,36 @@ def measured_peaks():
 PROFILE_TF32 = os.path.join(ROOT, "profiles", "tf32_peak_cublas.md")
 
 
-def tf32_peak():
-    """Measured dense tf32 throughput of the vendor GEMM (sustained), from the
-    committed measurement; None if it is missing."""
+def tf32_peaks():
+    """Measured dense tf32 throughput of the vendor GEMM, burst and
+    sustained, from the committed measurement; None where missing."""
+    out = {"burst": None, "sustained": None}
     try:
         for line in open(PROFILE_TF32):
+            if line.startswith("tf32_tflops:"):
+                out["burst"] = float(line.split(":", 1)[1].split()[0])
             if line.startswith("tf32_tflops_sustained:"):
-                return float(line.split(":", 1)[1].split()[0])
+                out["sustained"] = float(line.split(":", 1)[1].split()[0])
     except OSError:
         pass
-    return None
+    return out
+
+
+def regime(clocks) -> str:
+    """Which measured peak applies to this run: "burst" when the clock record
+    of the timed region never showed the power cap and the median SM clock sat
+    at its maximum, else "sustained" (the figure taken under the power cap)."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if mhz is None or mx is None:
+        return "sustained"
+    if "sw_power_cap" in clocks.get("reasons", []) or mhz < 0.97 * mx:
+        return "sustained"
+    return "burst"
+
+
+def bf16_peaks(peaks):
+    return {"burst": float(peaks.get("bf16_tflops")),
+            "sustained": float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))}
 
 
 def lazy_flops(spec) -> float:
@@ -139,32 +175,81 @@ def lazy_flops(spec) -> float:
 
 
 def lazy_batch_line(spec, stage):
+    """All lazy-batch products of the column loop (events between launches,
+    gptq_quantize_timed) against the measured tf32 peak: `frac` against the
+    burst figure (the products run as short bursts inside the column loop),
+    `frac_sustained` against the power-capped one."""
     if not stage or not stage.get("lazy_batch_ms"):
         return None
     fl = lazy_flops(spec)
     rate = fl / (stage["lazy_batch_ms"] / 1e3) / 1e12
-    peak = tf32_peak()
+    pk = tf32_peaks()
     return {"flops_fp32": fl, "ms": stage["lazy_batch_ms"], "achieved_fp32_tflops": rate,
-            "tf32_rate_tflops": 3 * rate, "peak": peak, "unit": "TFLOP/s",
-            "frac": (3 * rate / peak) if peak else None,
-            "note": "3xTF32: three tf32 MMAs per fp32-accurate product; peak = measured cuBLAS tf32, sustained"}
+            "tf32_rate_tflops": 3 * rate, "peak": pk["burst"], "peak_sustained": pk["sustained"],
+            "unit": "TFLOP/s", "frac": (3 * rate / pk["burst"]) if pk["burst"] else None,
+            "frac_sustained": (3 * rate / pk["sustained"]) if pk["sustained"] else None,
+            "note": "3xTF32: three tf32 MMAs per fp32-accurate product; peaks = measured cuBLAS tf32 "
+                    "(profiles/tf32_peak_cublas.md)"}
 
 
-def layer_roofline(spec, ms, bf16_peak, stage):
-    """Ideal time of the layer's tensor work at the measured peaks (Hessian on
-    bf16, factorisation and lazy batch as 3xTF32) against the measured step;
-    the column loop's chain of dependent column steps has no flop roofline and
-    is not in the ideal."""
-    peak = tf32_peak()
-    if not peak:
+def layer_roofline(spec, ms, reg, peaks):
+    """Ideal time of the layer's tensor work at the measured peaks of this
+    run's clock regime (Hessian on bf16, factorisation and lazy batch as
+    3xTF32) against the measured step; the column loop's chain of dependent
+    column steps has no flop roofline and is not in the ideal."""
+    tf = tf32_peaks()[reg]
+    if not tf:
         return None
     d = spec.d_in
-    t_h = spec.n_tokens * d * (d + 1) / (bf16_peak * 1e12) * 1e3
-    t_f = 3 * (2.0 / 3.0) * d ** 3 / (peak * 1e12) * 1e3
-    t_l = 3 * lazy_flops(spec) / (peak * 1e12) * 1e3
+    t_h = spec.n_tokens * d * (d + 1) / (bf16_peaks(peaks)[reg] * 1e12) * 1e3
+    t_f = 3 * (2.0 / 3.0) * d ** 3 / (tf * 1e12) * 1e3
+    t_l = 3 * lazy_flops(spec) / (tf * 1e12) * 1e3
     ideal = t_h + t_f + t_l
-    return {"ideal_ms": ideal, "measured_ms": ms, "frac": ideal / ms,
+    return {"ideal_ms": ideal, "measured_ms": ms, "frac": ideal / ms, "peaks": reg,
             "terms_ms": {"hessian": t_h, "factorisation": t_f, "lazy_batch": t_l}}
+
+
+def hessian_split(spec, sms: int = 148) -> int:
+    """Token spans per tile of one Hessian launch (the launcher's rule): the
+    longest power-of-two span in 4096 .. 32768 that still gives every pair of
+    SMs about eight work units; a single unit when H is one 256-column tile."""
+    n_t = (spec.d_in + 255) // 256
+    if n_t == 1:
+        return 1
+    tiles = n_t * (n_t + 1) // 2
+    span = 32768
+    while span > 4096 and tiles * -(-spec.n_tokens // span) < 8 * (sms // 2):
+        span //= 2
+    return -(-spec.n_tokens // span)
+
+
+def hessian_alg_bytes(spec) -> float:
+    """Algorithmic DRAM bytes of one Hessian launch: X read once, and every
+    token span's partial sum added into the upper triangle of H (one read and
+    one write of each element per span)."""
+    d = spec.d_in
+    return 2.0 * spec.n_tokens * d + hessian_split(spec) * (d * (d + 1) / 2) * 8.0
+
+
+def hessian_roofline(spec, h_ms, clocks, peaks, peak_kind):
+    """Roofline object of the Hessian kernel (the dominant kernel): achieved =
+    N d (d + 1) flops (upper triangle incl. the diagonal) / launch time, peak
+    = the measured bf16 figure of the run's clock regime; both fractions."""
+    reg = regime(clocks)
+    pk = bf16_peaks(peaks)
+    alg_flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)
+    achieved = alg_flops / (h_ms / 1e3) / 1e12
+    traffic = profiled_traffic(os.path.join(ROOT, "post_weight_quantization_accumulate_b200",
+                                            "csrc", "hessian.cu"))
+    if traffic is not None and spec.name != "q_proj_4096":
+        traffic = None
+    alg_bytes = hessian_alg_bytes(spec)
+    return {"kernel": "hessian_tc_kernel (+ mirror copy)", "bound": "tensor",
+            "achieved": achieved, "peak": pk[reg], "unit": "TFLOP/s", "frac": achieved / pk[reg],
+            "traffic": traffic, "peak_source": f"{peak_kind} bf16_tflops ({reg}; clocks of this run)",
+            "frac_burst": achieved / pk["burst"], "frac_sustained": achieved / pk["sustained"],
+            "flops_per_launch": alg_flops, "launch_ms": h_ms, "alg_bytes": alg_bytes,
+            "traffic_over_alg_bytes": (traffic / alg_bytes) if traffic else None}
 
 
 def profiled_traffic(kernel_src: str):
@@ -191,7 +276,8 @@ def cpu_baseline(spec, threads: int):
       Hessian      2048 of n_tokens tokens, full d_in     (x n_tokens/2048, O(N d^2))
       factor       leading 1024 x 1024 block of that H    (x (d_in/1024)^3, O(d^3))
       column loop  32 rows at d_in = 1024                 (x d_out/32 x (d_in/1024)^2)
-    """
+    `measured_s` is the time the sample took; `extrapolated_layer_s` the full
+    layer's time by those laws (an extrapolation, not a measurement)."""
     import numpy as np
     import oracle
     from post_weight_quantization_accumulate_b200 import synth
@@ -209,40 +295,89 @@ def cpu_baseline(spec, threads: int):
     oracle.quantize(W, U, perm, spec.bits, spec.group_size if spec.group_size <= d_s else -1,
                     spec.block_size)
     t_q = time.perf_counter() - t0
-    full = (t_h * spec.n_tokens / n_s + t_p * (spec.d_in / d_s) ** 3 +
-            t_q * (spec.d_out / r_s) * (spec.d_in / d_s) ** 2)
-    sample = (f"Hessian on {n_s}/{spec.n_tokens} tokens (x{spec.n_tokens / n_s:g}); factor at d={d_s} "
-              f"(x{(spec.d_in / d_s) ** 3:g}); column loop {r_s} rows at d_in={d_s} "
-              f"(x{(spec.d_out / r_s) * (spec.d_in / d_s) ** 2:g}); float64, OpenMP")
+    laws = {"hessian": spec.n_tokens / n_s, "factor": (spec.d_in / d_s) ** 3,
+            "column_loop": (spec.d_out / r_s) * (spec.d_in / d_s) ** 2}
+    stages = {"hessian": t_h, "factor": t_p, "column_loop": t_q}
+    full = sum(stages[k] * laws[k] for k in stages)
+    sample = (f"Hessian on {n_s}/{spec.n_tokens} tokens (x{laws['hessian']:g}); factor at d={d_s} "
+              f"(x{laws['factor']:g}); column loop {r_s} rows at d_in={d_s} "
+              f"(x{laws['column_loop']:g}); float64, OpenMP; value extrapolated by these cost laws")
     return {"value": spec.d_out * spec.d_in / full, "unit": UNIT, "cores": threads,
             "kind": "oracle", "sample": sample, "measured_s": t_h + t_p + t_q,
-            "extrapolated_layer_s": full}
+            "stages_measured_s": stages, "extrapolated_layer_s": full,
+            "value_basis": "extrapolated: full-layer time from the measured sample by the cost laws"}
+
+
+def validate_cost_laws(spec, threads: int):
+    """Checks the extrapolation once against full-size runs of the checker:
+    the factorisation at the workload's own d_in (from the Hessian of 2048
+    tokens), and 256 full rows of the column loop (with that factor); each
+    against the sample's time scaled by its cost law."""
+    import numpy as np
+    import oracle
+    from post_weight_quantization_accumulate_b200 import synth
+    d_s, r_s, rows = min(1024, spec.d_in), 32, 256
+    xb = synth.x_bf16(spec, tokens=slice(0, 2048))
+    H = oracle.hessian(xb)
+    t0 = time.perf_counter()
+    oracle.prepare(np.ascontiguousarray(H[:d_s, :d_s]), spec.damp, spec.act_order)
+    t_small = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    perm, U, _, _ = oracle.prepare(H, spec.damp, spec.act_order)
+    t_full = time.perf_counter() - t0
+    gs = spec.group_size
+    Ws = synth.weight_f32(spec, rows=slice(0, r_s))[:, :d_s].astype(np.float64)
+    perm_s, U_s, _, _ = oracle.prepare(np.ascontiguousarray(H[:d_s, :d_s]), spec.damp, spec.act_order)
+    t0 = time.perf_counter()
+    oracle.quantize(Ws, U_s, perm_s, spec.bits, gs if gs <= d_s else -1, spec.block_size)
+    q_small = time.perf_counter() - t0
+    Wf = synth.weight_f32(spec, rows=slice(0, rows)).astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.quantize(Wf, U, perm, spec.bits, gs, spec.block_size)
+    q_full = time.perf_counter() - t0
+    f_pred = t_small * (spec.d_in / d_s) ** 3
+    q_pred = q_small * (rows / r_s) * (spec.d_in / d_s) ** 2
+    return {"factor": {"d": spec.d_in, "measured_s": t_full, "extrapolated_s": f_pred,
+                       "extrapolated_over_measured": f_pred / t_full},
+            "column_loop": {"rows": rows, "d_in": spec.d_in, "measured_s": q_full,
+                            "extrapolated_s": q_pred, "extrapolated_over_measured": q_pred / q_full},
+            "cores": threads}
 
 
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank, world):
+    """The float64 checker (the reference of this path) on the host cores.
+    One step = one bounded sample of the workload (see cpu_baseline); the
+    line's ms_per_step is the time a sample took, and `value` the full
+    layer's rate extrapolated from it by the stages' cost laws."""
     if rank != 0:
         return 0
     threads = len(os.sched_getaffinity(0))
     os.environ.setdefault("OMP_NUM_THREADS", str(threads))
     from post_weight_quantization_accumulate_b200 import synth
-    spec = synth.WORKLOADS[args.workload]
+    spec = synth.WORKLOADS[args.workload if args.workload in synth.WORKLOADS else "q_proj_4096"]
     vals = []
     for i in range(args.warmup + args.steps):
         cb = cpu_baseline(spec, threads)
         if i >= args.warmup:
             vals.append(cb)
     value = statistics.median(v["value"] for v in vals)
+    step_ms = statistics.median(v["measured_s"] for v in vals) * 1e3
     layer_s = spec.d_out * spec.d_in / value
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": config_of(spec, args.gpus),
+            "step": "one bounded sample of the layer (ms_per_step is its measured time)",
+            "extrapolated_layer_ms": layer_s * 1e3,
+            "value_basis": vals[0]["value_basis"],
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": vals[0]["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if args.validate_cost_laws:
+        line["cost_law_check"] = validate_cost_laws(spec, threads)
     print(json.dumps(line), flush=True)
     return 0
 
@@ -273,8 +408,9 @@ def run_decoder_layer(args, rank) -> int:
     shape = D.LLAMA2_7B
     W, X = D.synthetic_layer(shape)
     combos = [(b, g) for b in (2, 3, 4) for g in (64, 128, -1)] if args.sweep else [(4, 128)]
+    cache = {}
     for _ in range(max(1, min(args.warmup, 1))):
-        D.calibrate(X, W, shape, bits=4, group_size=128)
+        D.calibrate(X, W, shape, bits=4, group_size=128, cache=cache)
     torch.cuda.synchronize()
     rows = []
     for bits, gs in combos:
@@ -282,7 +418,7 @@ def run_decoder_layer(args, rank) -> int:
         for _ in range(max(1, min(args.steps, 3))):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            r = D.calibrate(X, W, shape, bits=bits, group_size=gs)
+            r = D.calibrate(X, W, shape, bits=bits, group_size=gs, cache=cache)
             b.record()
             torch.cuda.synchronize()
             ms.append(a.elapsed_time(b))
@@ -378,6 +514,248 @@ def run_w4a16(args, rank) -> int:
     return 0
 
 
+def _timed_layer(q, X, Wd, stream, steps, warmup, barrier, clock_gpu):
+    """`steps` timed per-layer steps (H zeroed, Hessian over X, factorisation,
+    column loop) after `warmup` untimed ones; returns (ms per step, mean
+    Hessian-call ms, launches, clocks)."""
+    import torch
+    from post_weight_quantization_accumulate_b200 import binding as B
+    ev_h = []
+
+    def step(record=False):
+        q.reset()
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        q.add_batch(X)
+        if record:
+            e1.record(stream)
+            ev_h.append((e0, e1))
+        q.run(Wd)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = B.gptq_launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(clock_gpu) as clk:
+        t_start.record(stream)
+        for _ in range(steps):
+            step(record=True)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = B.gptq_launch_count() - launches0
+    ms = t_start.elapsed_time(t_end) / steps
+    h_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_h)
+    return ms, h_ms, launches, clk.summary()
+
+
+def _stages(q, X, Wd, stream):
+    """One step broken down by stage (after the timed region), and the column
+    loop split into its kernel classes (events between launches)."""
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    evs[0].record(stream)
+    q.reset()
+    q.add_batch(X)
+    evs[1].record(stream)
+    q.prepare()
+    evs[2].record(stream)
+    q.quantize(Wd)
+    evs[3].record(stream)
+    torch.cuda.synchronize()
+    stage = {"hessian_ms": evs[0].elapsed_time(evs[1]), "prepare_ms": evs[1].elapsed_time(evs[2]),
+             "quantize_ms": evs[2].elapsed_time(evs[3])}
+    qt = q.quantize_timed(Wd)
+    stage.update({"column_loop_ms": qt[0], "lazy_batch_ms": qt[1], "quantize_other_ms": qt[2]})
+    return stage
+
+
+def _host_inputs(spec):
+    """Seeded synthetic X (bf16) and W of the workload in pinned host memory."""
+    import numpy as np
+    import torch
+    from post_weight_quantization_accumulate_b200 import synth
+    X_host = torch.empty(spec.n_tokens, spec.d_in, dtype=torch.int16).pin_memory()
+    synth.x_bf16(spec, out=X_host.numpy().view(np.uint16))
+    X_host = X_host.view(torch.bfloat16)
+    wbits = synth.weight_bf16_bits(spec) if spec.w_bf16 else None
+    W_host = (torch.from_numpy(wbits.view(np.int16)).view(torch.bfloat16) if spec.w_bf16
+              else torch.from_numpy(synth.weight_f32(spec))).pin_memory()
+    return X_host, W_host
+
+
+def by_config_line(name, dev, peaks, peak_kind, steps=2, warmup=1):
+    """One other single-GPU workload of the recipe: its step time, stages and
+    rooflines (no e2e, no CPU baseline)."""
+    import torch
+    from post_weight_quantization_accumulate_b200 import binding as B
+    from post_weight_quantization_accumulate_b200 import synth
+    from post_weight_quantization_accumulate_b200.layer import LayerQuantizer
+    spec = synth.WORKLOADS[name]
+    X_host, W_host = _host_inputs(spec)
+    X, Wd = X_host.to(dev), W_host.to(dev)
+    del X_host, W_host
+    q = LayerQuantizer(spec.d_out, spec.d_in, spec.bits, spec.group_size, spec.block_size,
+                       spec.damp, spec.act_order, device=dev, keep_codes=False)
+    stream = torch.cuda.current_stream(dev)
+    ms, h_ms, launches, clocks = _timed_layer(q, X, Wd, stream, steps, warmup, lambda: None, dev.index)
+    stage = _stages(q, X, Wd, stream)
+    status = B.gptq_device_status()
+    reg = regime(clocks)
+    out = {"workload": name, "config": config_of(spec, 1), "value": spec.d_out * spec.d_in / (ms / 1e3),
+           "unit": UNIT, "ms_per_step": ms, "steps": steps, "warmup": warmup,
+           "roofline": hessian_roofline(spec, h_ms, clocks, peaks, peak_kind),
+           "lazy_batch": lazy_batch_line(spec, stage),
+           "layer_roofline": layer_roofline(spec, ms, reg, peaks), "stages_ms": stage,
+           "clocks": clocks, "gpu_launches": int(launches), "device_status": status}
+    del q, X, Wd
+    torch.cuda.empty_cache()
+    return out
+
+
+def decoder_layer_result(bits=4, group_size=128, steps=1, warmup=1):
+    """One Llama-2-7B-shaped decoder layer, layer-sequential, on cuda:0."""
+    import torch
+    from post_weight_quantization_accumulate_b200 import decoder as D
+    shape = D.LLAMA2_7B
+    W, X = D.synthetic_layer(shape)
+    cache = {}   # the layer quantizers of one decoder layer, reused as a model's layers would
+    for _ in range(warmup):
+        D.calibrate(X, W, shape, bits=bits, group_size=group_size, cache=cache)
+    torch.cuda.synchronize()
+    ms, r = [], None
+    for _ in range(max(1, steps)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        r = D.calibrate(X, W, shape, bits=bits, group_size=group_size, cache=cache)
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    n_w = D.quantized_weights(shape)
+    out = {"bits": bits, "group_size": group_size, "ms": min(ms), "groups_ms": r.ms,
+           "weights": n_w, "value": n_w / (min(ms) / 1e3), "unit": UNIT}
+    del r, W, X, cache
+    torch.cuda.empty_cache()
+    return out
+
+
+def hessian_f32_line(dev, peaks, reps=3):
+    """gptq_hessian_accumulate_f32 at the q_proj size (262144 x 4096 fp32
+    activations, N(0, 1) drawn on the device by a seeded generator) in
+    16384-token chunks; its tensor work is four bf16 Hessians of the
+    [hi | lo] split, so the roofline counts 4 N d (d + 1) flops."""
+    import torch
+    from post_weight_quantization_accumulate_b200 import binding as B
+    n, d, chunk = 262144, 4096, 16384
+    g = torch.Generator(device=dev)
+    g.manual_seed(4096)
+    X = torch.randn(n, d, generator=g, device=dev, dtype=torch.float32)
+    H = torch.zeros(d, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(B.gptq_hessian_f32_workspace_bytes(d, chunk), dtype=torch.uint8, device=dev)
+    B.gptq_hessian_accumulate_f32(H, X, ws, chunk)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        H.zero_()
+        B.gptq_hessian_accumulate_f32(H, X, ws, chunk)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    status = B.gptq_device_status()
+    tensor_flops = float(n) * (2 * d) * (2 * d + 1)   # upper triangle of the 2d x 2d block Hessian
+    pk = bf16_peaks(peaks)
+    del X, H, ws
+    torch.cuda.empty_cache()
+    return {"workload": "hessian_f32_262144x4096", "ms": ms, "tokens": n, "d_in": d,
+            "chunk_tokens": chunk, "tensor_tflops": tensor_flops / (ms / 1e3) / 1e12,
+            "frac_of_bf16_burst": tensor_flops / (ms / 1e3) / 1e12 / pk["burst"],
+            "note": "tensor work = upper triangle of 2 Z^T Z for Z = [hi | lo] (n x 2d), plus "
+                    "the split and fold passes", "device_status": status}
+
+
+def run_split(args, rank, world, local):
+    """One layer over all ranks (--split tokens_rows): token-sharded Hessian,
+    one NCCL all-reduce of H, the factorisation on every rank, each rank's
+    block of rows.  value = one layer's weights per step time (strong
+    scaling); at N = 1 this is the default line's work."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from post_weight_quantization_accumulate_b200 import binding as B
+    from post_weight_quantization_accumulate_b200 import build as build_mod
+    from post_weight_quantization_accumulate_b200 import ranks, synth
+    from post_weight_quantization_accumulate_b200.sharded import ShardedLayer, token_range
+
+    if rank == 0:
+        build_mod.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=600))
+        dist.barrier()
+        if rank != 0:
+            build_mod.build()
+    B.lib()
+    spec = synth.WORKLOADS[args.workload]
+    t0, t1 = token_range(spec.n_tokens, rank, world)
+    xb = synth.x_bf16(spec, tokens=slice(t0, t1))
+    X = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    del xb
+    W = torch.from_numpy(synth.weight_f32(spec)).to(dev)
+    sl = ShardedLayer(spec.d_out, spec.d_in, spec.bits, spec.group_size, spec.block_size, spec.damp,
+                      spec.act_order, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sl.reset()
+        sl.add_batch(X)
+        sl.prepare()
+        sl.quantize(W)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = B.gptq_launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = B.gptq_launch_count() - launches0
+    ms = ranks.max_over_ranks([a.elapsed_time(b) / args.steps], device=dev)[0]
+    status = B.gptq_device_status()
+    if rank == 0:
+        cfg = config_of(spec, world)
+        cfg["parallelism"] = f"one layer over {world} ranks: tokens sharded, H all-reduced, rows sharded"
+        print(json.dumps({
+            "metric": METRIC, "value": spec.d_out * spec.d_in / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": cfg, "clocks": clk.summary(), "gpu_launches": int(launches),
+            "device_status": status, "split": "tokens_rows"}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -389,8 +767,9 @@ def main():
         return run_decoder_layer(args, rank)
     if args.workload == "w4a16":
         return run_w4a16(args, rank)
+    if args.split == "tokens_rows":
+        return run_split(args, rank, world, local)
 
-    import numpy as np
     import torch
     import torch.distributed as dist
     from post_weight_quantization_accumulate_b200 import binding as B
@@ -415,76 +794,21 @@ def main():
     threads = len(os.sched_getaffinity(0))
 
     # inputs: generated on the host, pinned, copied to HBM once
-    xb = synth.x_bf16(spec)
-    X_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
-    del xb
-    wbits = synth.weight_bf16_bits(spec) if spec.w_bf16 else None
-    W_host = (torch.from_numpy(wbits.view(np.int16)).view(torch.bfloat16) if spec.w_bf16
-              else torch.from_numpy(synth.weight_f32(spec))).pin_memory()
+    X_host, W_host = _host_inputs(spec)
     X = X_host.to(dev, non_blocking=False)
     Wd = W_host.to(dev)
     q = LayerQuantizer(spec.d_out, spec.d_in, spec.bits, spec.group_size, spec.block_size,
                        spec.damp, spec.act_order, device=dev, keep_codes=False)
     stream = torch.cuda.current_stream(dev)
 
-    ev_h = []   # (start, end) of the Hessian call per timed step
-
-    def step(record=False):
-        q.reset()
-        if record:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        q.add_batch(X)
-        if record:
-            e1.record(stream)
-            ev_h.append((e0, e1))
-        q.run(Wd)
-
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    launches0 = B.gptq_launch_count()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for _ in range(args.steps):
-            step(record=True)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    launches = B.gptq_launch_count() - launches0
-    ms = t_start.elapsed_time(t_end) / args.steps
-    h_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_h)
+    ms, h_ms, launches, clocks = _timed_layer(q, X, Wd, stream, args.steps, args.warmup, barrier, local)
     status = B.gptq_device_status()
     ms, h_ms = ranks.max_over_ranks([ms, h_ms], device=dev)
-    clocks = clk.summary()
-
-    # one step broken down by stage (after the timed region)
-    stage = {}
-    if rank == 0:
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        evs[0].record(stream)
-        q.reset()
-        q.add_batch(X)
-        evs[1].record(stream)
-        q.prepare()
-        evs[2].record(stream)
-        q.quantize(Wd)
-        evs[3].record(stream)
-        torch.cuda.synchronize()
-        stage = {"hessian_ms": evs[0].elapsed_time(evs[1]), "prepare_ms": evs[1].elapsed_time(evs[2]),
-                 "quantize_ms": evs[2].elapsed_time(evs[3])}
-        # the column-loop stage split into its kernel classes (events between launches)
-        qt = q.quantize_timed(Wd)
-        stage.update({"column_loop_ms": qt[0], "lazy_batch_ms": qt[1], "quantize_other_ms": qt[2]})
+    stage = _stages(q, X, Wd, stream) if rank == 0 else {}
 
     # end to end through the public API with host buffers: X and W copied in
     # (overlapped chunked copy of X), packed codes + scales + zeros + g_idx out
@@ -522,6 +846,18 @@ def main():
         d2h = (packed_h.numel() + scales_h.numel() * 4 + zeros_h.numel() * 4 + gidx_h.numel() * 4)
         e2e = {"value": ranks.job_rate(world, spec.d_out, spec.d_in, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        del Wd2
+
+    peaks, peak_kind = measured_peaks()
+    by_config = None
+    if rank == 0 and world == 1 and not args.no_by_config and args.workload == "q_proj_4096":
+        del q, X, Wd
+        torch.cuda.empty_cache()
+        by_config = {}
+        for name in ("down_proj_11008", "up_proj_70b"):
+            by_config[name] = by_config_line(name, dev, peaks, peak_kind)
+        by_config["llama2_7b_decoder_layer_4bit_g128"] = decoder_layer_result()
+        by_config["hessian_f32_262144x4096"] = hessian_f32_line(dev, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -529,28 +865,19 @@ def main():
         cpu = cpu_baseline(spec, threads)
 
     if rank == 0:
-        peaks, peak_kind = measured_peaks()
-        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-        alg_flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)   # upper triangle incl. diagonal
-        achieved = alg_flops / (h_ms / 1e3) / 1e12
-        traffic = profiled_traffic(os.path.join(ROOT, "post_weight_quantization_accumulate_b200",
-                                                "csrc", "hessian.cu"))
+        reg = regime(clocks)
         line = {
             "metric": METRIC, "value": ranks.job_rate(world, spec.d_out, spec.d_in, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": config_of(spec, world),
-            "roofline": {"kernel": "hessian_tc_kernel (+ mirror copy)", "bound": "tensor",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_kind} bf16_tflops_sustained",
-                         "flops_per_launch": alg_flops, "launch_ms": h_ms},
+            "roofline": hessian_roofline(spec, h_ms, clocks, peaks, peak_kind),
             "hessian_tflops_dense_equiv": 2 * spec.n_tokens * spec.d_in ** 2 / (h_ms / 1e3) / 1e12,
             "lazy_batch": lazy_batch_line(spec, stage),
-            "layer_roofline": layer_roofline(spec, ms, peak, stage),
+            "layer_roofline": layer_roofline(spec, ms, reg, peaks),
             "stages_ms": stage,
             "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
-            "e2e": e2e, "cpu_baseline": cpu,
+            "e2e": e2e, "cpu_baseline": cpu, "by_config": by_config,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -1,10 +1,10 @@
 """Runs one library call on a synthetic layer, a few times, for profiling.
 
-    python -m post_weight_quantization_accumulate_b200.kernel_case \
+    python kernel_case.py \
         --call hessian|prepare|quantize|layer --workload q_proj_4096 [--tokens N] [--reps R]
-    python -m post_weight_quantization_accumulate_b200.kernel_case \
+    python kernel_case.py \
         --call w4a16 [--m M] [--n N] [--k K] [--group-size G] [--path 0|1|2] [--reps R]
-    python -m post_weight_quantization_accumulate_b200.kernel_case \
+    python kernel_case.py \
         --call hessian_f32 --workload q_proj_4096 --tokens N [--reps R]
 
 The inputs follow the workload's recipe (see synth.py) with `--tokens`
@@ -22,7 +22,7 @@ import time
 import numpy as np
 import torch
 
-sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 from post_weight_quantization_accumulate_b200 import binding as B  # noqa: E402
 from post_weight_quantization_accumulate_b200 import synth  # noqa: E402

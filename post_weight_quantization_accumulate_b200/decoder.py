@@ -115,16 +115,26 @@ def _copy(ql: QuantizedLayer) -> QuantizedLayer:
 
 def calibrate(X_attn: torch.Tensor, W: dict, shape: DecoderShape, bits: int = 4, group_size: int = 128,
               block_size: int = 128, damp: float = 0.01, act_order: bool = False,
-              keep_state: bool = False) -> DecoderResult:
+              keep_state: bool = False, cache: dict | None = None) -> DecoderResult:
     """Quantizes the seven linears group by group; each group's Hessian comes
-    from the input the earlier (already quantized) groups produce."""
+    from the input the earlier (already quantized) groups produce.
+
+    `cache` (a dict the caller keeps between calls) holds the per-shape
+    LayerQuantizer buffers, so that repeated calibrations of layers of the
+    same shape reuse them -- and the library's CUDA graphs, which are keyed
+    by the buffers' addresses -- instead of allocating and capturing anew."""
     res = DecoderResult()
     inputs = {"qkv": X_attn}
     for group, names in GROUPS:
         X = inputs[group]
         d_out, d_in = shape.linear_shape(names[0])
-        q = LayerQuantizer(d_out, d_in, bits, group_size, block_size, damp, act_order,
-                           device=X.device)
+        key = (d_out, d_in, bits, group_size, block_size, damp, act_order, str(X.device))
+        q = cache.get(key) if cache is not None else None
+        if q is None:
+            q = LayerQuantizer(d_out, d_in, bits, group_size, block_size, damp, act_order,
+                               device=X.device)
+            if cache is not None:
+                cache[key] = q
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record()
         q.reset()
