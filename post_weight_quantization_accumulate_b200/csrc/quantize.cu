@@ -47,6 +47,14 @@ constexpr int UT_LD = QTPR * UT_PART;
 constexpr int UCH_FLOATS = QSUB * UT_LD + 2 * QSUB;
 constexpr int UCH_BYTES = UCH_FLOATS * 4;          // 10368, a multiple of 16
 constexpr size_t kBlockSmem = static_cast<size_t>(QNSUB) * UCH_BYTES + 128;
+// Shared memory a column-loop launch asks for when its grid fits on the SMs
+// at once: more than half of an SM's, so that one CTA holds an SM by itself.
+// Two CTAs on one SM would each take longer, and every launch lasts as long as
+// its slowest CTA; with programmatic dependent launches the early CTAs of a
+// launch would otherwise double up on the few SMs the previous kernel leaves
+// free.
+constexpr size_t kBlockSmemLaunch = 116 * 1024;
+static_assert(kBlockSmemLaunch >= kBlockSmem, "the launch covers the kernel's shared memory");
 static_assert(UCH_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 struct QArgs {
@@ -592,6 +600,70 @@ __global__ void gather_cols_kernel(const float* __restrict__ W, int d_out, int d
     }
 }
 
+// Row-staged forms of the two column gathers of the act_order path, for rows
+// of at most kRowStageMax columns: a CTA reads a whole row with coalesced
+// 16-byte loads into shared memory, then writes the permuted row in order, so
+// the scattered reads hit shared memory instead of pulling a 32-byte sector
+// from L2 for every 4 useful bytes.
+constexpr int kRowStageMax = 16384;
+constexpr int kRowThreads = 512;
+
+// Wp[r][k] = W[r][perm[k]]
+__global__ void __launch_bounds__(kRowThreads)
+    gather_cols_rows_kernel(const float* __restrict__ W, int d_out, int d_in,
+                            const int32_t* __restrict__ perm, float* __restrict__ Wp)
+{
+    extern __shared__ __align__(16) float row[];
+    for (int r = blockIdx.x; r < d_out; r += gridDim.x) {
+        const float4* src = reinterpret_cast<const float4*>(W + static_cast<int64_t>(r) * d_in);
+        __syncthreads();   // the previous row has been written out
+        for (int i = threadIdx.x; i < d_in / 4; i += blockDim.x) reinterpret_cast<float4*>(row)[i] = src[i];
+        __syncthreads();
+        float* dst = Wp + static_cast<int64_t>(r) * d_in;
+        for (int k = threadIdx.x; k < d_in; k += blockDim.x) {
+            int p = perm[k];
+            p = (p < 0 || p >= d_in) ? 0 : p;
+            dst[k] = row[p];
+        }
+    }
+}
+
+// finish_kernel's work for a permuted layer, one staged row (W^ and codes in
+// processing order) at a time: W^, codes and packed nibbles in original order.
+__global__ void __launch_bounds__(kRowThreads)
+    finish_rows_kernel(const uint8_t* __restrict__ codes_p, const float* __restrict__ Wp,
+                       const int32_t* __restrict__ inv, int d_out, int d_in, float* __restrict__ W,
+                       uint8_t* __restrict__ codes, uint8_t* __restrict__ packed, int* status)
+{
+    extern __shared__ __align__(16) float wrow[];
+    uint8_t* crow = reinterpret_cast<uint8_t*>(wrow + d_in);
+    const int half = d_in / 2;
+    for (int r = blockIdx.x; r < d_out; r += gridDim.x) {
+        const int64_t ro = static_cast<int64_t>(r) * d_in;
+        __syncthreads();   // the previous row has been written out
+        for (int i = threadIdx.x; i < d_in / 4; i += blockDim.x)
+            reinterpret_cast<float4*>(wrow)[i] = reinterpret_cast<const float4*>(Wp + ro)[i];
+        for (int i = threadIdx.x; i < d_in / 8; i += blockDim.x)
+            reinterpret_cast<uint2*>(crow)[i] = reinterpret_cast<const uint2*>(codes_p + ro)[i];
+        __syncthreads();
+        for (int i = threadIdx.x; i < half; i += blockDim.x) {
+            int k0 = inv[2 * i], k1 = inv[2 * i + 1];
+            if (k0 < 0 || k0 >= d_in || k1 < 0 || k1 >= d_in) {   // a malformed permutation
+                if (r == 0) record_status(status, GPTQ_ERR_INVALID_ARG);
+                k0 = (k0 < 0 || k0 >= d_in) ? 0 : k0;
+                k1 = (k1 < 0 || k1 >= d_in) ? 0 : k1;
+            }
+            const uint8_t q0 = crow[k0], q1 = crow[k1];
+            if (codes) {   // byte stores: the caller's codes buffer has no alignment rule
+                codes[ro + 2 * i] = q0;
+                codes[ro + 2 * i + 1] = q1;
+            }
+            if (packed) packed[static_cast<int64_t>(r) * half + i] = static_cast<uint8_t>((q0 & 15) | ((q1 & 15) << 4));
+            *reinterpret_cast<float2*>(W + ro + 2 * i) = make_float2(wrow[k0], wrow[k1]);
+        }
+    }
+}
+
 // Original-order outputs: codes, packed nibbles, and (with a permutation) W^.
 // One thread per pair of original columns (2i, 2i+1).  A column missing from
 // the permutation (perm not a bijection) records GPTQ_ERR_INVALID_ARG; its
@@ -765,7 +837,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     // The column-loop kernels and the lazy-batch products alternate on the
     // stream as programmatic dependent launches, each one's set-up overlapping
     // the previous one's tail -- except when events are recorded between them.
-    const bool pdl = false && marks == nullptr;
+    const bool pdl = marks == nullptr;
     const int d_out = static_cast<int>(d_out64), d_in = static_cast<int>(d_in64);
     const size_t n = static_cast<size_t>(d_out) * d_in;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -792,13 +864,19 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     if (dev < 64 && !attr_set[dev]) {
         GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<false, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kBlockSmem)));
+                                             static_cast<int>(kBlockSmemLaunch)));
         GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<true, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kBlockSmem)));
+                                             static_cast<int>(kBlockSmemLaunch)));
         GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gptq_block_kernel<false, true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kBlockSmem)));
+                                             static_cast<int>(kBlockSmemLaunch)));
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gather_cols_rows_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kRowStageMax * static_cast<int>(sizeof(float))));
+        GPTQ_CUDA_CHECK(cudaFuncSetAttribute(finish_rows_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kRowStageMax * static_cast<int>(sizeof(float) + 1)));
         attr_set[dev] = true;
     }
     // groups start only at 16-column sub-block starts when group_size is a
@@ -819,7 +897,12 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         GPTQ_CUDA_CHECK(cudaMemsetAsync(inv, 0xFF, static_cast<size_t>(d_in) * sizeof(int32_t), stream));
         invert_perm_kernel<<<(d_in + 255) / 256, 256, 0, stream>>>(perm, d_in, inv, status);
         GPTQ_LAUNCH_CHECK();
-        gather_cols_kernel<<<nsm * 8, 256, 0, stream>>>(W, d_out, d_in, perm, Wp);
+        if (d_in <= kRowStageMax)
+            gather_cols_rows_kernel<<<std::min(d_out, 2 * nsm), kRowThreads,
+                                      static_cast<size_t>(d_in) * sizeof(float), stream>>>(W, d_out, d_in,
+                                                                                          perm, Wp);
+        else
+            gather_cols_kernel<<<nsm * 8, 256, 0, stream>>>(W, d_out, d_in, perm, Wp);
         GPTQ_LAUNCH_CHECK();
         work = Wp;
     }
@@ -844,6 +927,9 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
     else
         outer = (kOuterMax / block) * block;
     const int grid = (d_out + QROWS - 1) / QROWS;
+    // one CTA per SM while the grid fits on the SMs at once; beyond that two
+    // per SM (more warps to hide each other's step latency in every wave)
+    const size_t block_smem = grid <= nsm ? kBlockSmemLaunch : kBlockSmem;
     for (int J0 = 0; J0 < d_in; J0 += outer) {
         const int J1 = (d_in - J0 < outer) ? d_in : J0 + outer;
         for (int j0 = J0; j0 < J1; j0 += block) {
@@ -855,7 +941,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
             if (int rc = mark(0)) return rc;
             auto kern = q4k ? gptq_block_kernel<false, true>
                             : (groups_in_step ? gptq_block_kernel<true, false> : gptq_block_kernel<false, false>);
-            GPTQ_CUDA_CHECK(launch_k(kern, dim3(grid), dim3(QTHREADS), kBlockSmem, stream, pdl, a));
+            GPTQ_CUDA_CHECK(launch_k(kern, dim3(grid), dim3(QTHREADS), block_smem, stream, pdl, a));
             GPTQ_LAUNCH_CHECK();
             if (int rc = mark(1)) return rc;
             const int rest_in = J1 - j0 - bw;
@@ -880,8 +966,13 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         }
     }
     if (codes || packed || perm) {
-        finish_kernel<<<nsm * 8, 256, 0, stream>>>(codes_p, Wp, perm ? inv : nullptr, d_out, d_in,
-                                                   W, codes, packed, status);
+        if (perm && d_in <= kRowStageMax)
+            finish_rows_kernel<<<std::min(d_out, 2 * nsm), kRowThreads,
+                                 static_cast<size_t>(d_in) * (sizeof(float) + 1), stream>>>(
+                codes_p, Wp, inv, d_out, d_in, W, codes, packed, status);
+        else
+            finish_kernel<<<nsm * 8, 256, 0, stream>>>(codes_p, Wp, perm ? inv : nullptr, d_out, d_in,
+                                                       W, codes, packed, status);
         GPTQ_LAUNCH_CHECK();
     }
     if (g_idx) {

@@ -6,9 +6,10 @@ but the Hessian is a sum over calibration tokens and the rows of W are
 independent given the factor.  So:
   1. each rank accumulates H over its own contiguous slice of the tokens;
   2. one all-reduce (sum) of the d x d fp32 H, the only exchange;
-  3. every rank runs the damping, ordering and factorisation on the same H,
-     so they all hold the same perm, and U equal up to the rounding of the
-     factorisation's unordered reduce-add epilogues, without a broadcast;
+  3. every rank runs the damping, ordering and factorisation on the same H
+     (the all-reduce hands every rank the same bits), and the factorisation
+     has no unordered reduction, so all ranks hold the same perm and the same
+     U bit for bit, without a broadcast;
   4. each rank quantizes its own contiguous block of rows of W;
   5. optionally one all-gather of the per-row outputs.
 
