@@ -151,10 +151,21 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
 // columns: warp 0 factors the strip with shuffles (lane l holds rows 4P+l and
 // 4P+l+32), then all warps subtract its rank-4 product from the trailing
 // lower triangle (thread (ty, tx) owns the 4 x 4 tile rows 4ty.., cols 4tx..).
-// Inverse Z = L^{-1} by recursive doubling: the 16 diagonal 4 x 4 inverses,
-// then Z21 = -Z22 (L21 Z11) for block sizes 8, 16, 32, 64.
+// The factor is then used through triangular solves, never inverted as a
+// whole: the panel rows P solve P L^T = T and the row block of M^{-1} solves
+// L X = T, by substitution -- one thread per row (or column) of the 64 x 64
+// right-hand side, holding it in registers; at step s it divides entry s by
+// L[s][s] and subtracts the multiple of L's column s (read from a transposed
+// copy with 16-byte loads) from the later entries.  The diagonal block of
+// M^{-1} is the solve with T = I.
+// The previous panel's rows enter every product of the kernel as its k index
+// (the 64 columns of that panel), so they are kept k-major: KTile[k][r] with
+// 16-byte aligned rows, read four rows (or columns) of the product at a time.
 typedef float Tile64[kNB + 1];
-constexpr size_t kPanelSmem = (5 * kNB * (kNB + 1) + 32 * 33) * sizeof(float) + 16;
+constexpr int kLTld = kNB + 4;   // row pitch of k-major tiles: 16-byte aligned rows
+typedef float KTile[kLTld];
+constexpr size_t kPanelSmem = (2 * kNB * (kNB + 1) + 3 * kNB * kLTld + kNB) * sizeof(float) + 16;
+static_assert((2 * kNB * (kNB + 1) * sizeof(float)) % 16 == 0, "the k-major tiles start 16-byte aligned");
 
 // 4-byte asynchronous copy global -> shared; `valid` false writes a zero.
 __device__ __forceinline__ void cp_async4(void* dst, const float* src, bool valid)
@@ -180,24 +191,84 @@ __device__ __forceinline__ void load_tile_async(Tile64* dst, const float* A, int
     }
 }
 
+// 64 x 64 tile of A into a k-major tile, asynchronously: transposed
+// (dst[j][i] = A[r_begin + i][c_begin + j]) or as it is (dst[i][j]).
+__device__ __forceinline__ void load_ktile_async(KTile* dst, const float* A, int d, int r_begin, int nrows,
+                                                 int c_begin, int ncols, bool transpose)
+{
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        const bool valid = i < nrows && j < ncols;
+        float* slot = transpose ? &dst[j][i] : &dst[i][j];
+        cp_async4(slot, valid ? A + static_cast<int64_t>(r_begin + i) * d + c_begin + j : A, valid);
+    }
+}
+
+__device__ __forceinline__ void load_ktile(KTile* dst, const float* A, int d, int r_begin, int nrows,
+                                           int c_begin, int ncols, bool transpose)
+{
+    const int tid = threadIdx.x;
+    float tv[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        tv[t] = (i < nrows && j < ncols) ? A[static_cast<int64_t>(r_begin + i) * d + c_begin + j] : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        if (transpose)
+            dst[j][i] = tv[t];
+        else
+            dst[i][j] = tv[t];
+    }
+}
+
+// acc[i][j] (tile rows r0.., cols c0..) -= sum_k X[k][r0 + i] Y[k][c0 + j], X
+// and Y k-major: per k one 16-byte load of each, 16 fmas as 8 paired fmas
+// (two independent IEEE fmas each, the bits of 16 fmaf).
+__device__ __forceinline__ void tile_minus_kmajor(float (&acc)[4][4], const KTile* X, const KTile* Y,
+                                                  int r0, int c0)
+{
+#pragma unroll 4
+    for (int k = 0; k < kNB; ++k) {
+        const float4 xv = *reinterpret_cast<const float4*>(&X[k][r0]);
+        const float4 yv = *reinterpret_cast<const float4*>(&Y[k][c0]);
+        const float xs[4] = {-xv.x, -xv.y, -xv.z, -xv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 nx = make_float2(xs[i], xs[i]);
+            float2 a = make_float2(acc[i][0], acc[i][1]);
+            float2 b = make_float2(acc[i][2], acc[i][3]);
+            a = __ffma2_rn(nx, make_float2(yv.x, yv.y), a);
+            b = __ffma2_rn(nx, make_float2(yv.z, yv.w), b);
+            acc[i][0] = a.x;
+            acc[i][1] = a.y;
+            acc[i][2] = b.x;
+            acc[i][3] = b.y;
+        }
+    }
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// acc[i][j] (tile rows 4ty.., cols 4tx..) -= X[rows] . Y[cols] over 64 columns:
-// the rank-64 correction of the previous panel applied on the fly.
-__device__ __forceinline__ void tile_minus_xyT(float (&acc)[4][4], const Tile64* X, const Tile64* Y,
-                                               int r0, int c0)
+// The first nrows x ncols entries of a tile back to A (rows r_begin..,
+// columns c_begin..), coalesced.
+__device__ __forceinline__ void store_tile(const Tile64* src, float* A, int d, int r_begin, int nrows,
+                                           int c_begin, int ncols)
 {
-    for (int k = 0; k < kNB; ++k) {
-        float xv[4], yv[4];
+    const int tid = threadIdx.x;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xv[i] = X[r0 + i][k];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) yv[j] = Y[c0 + j][k];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(-xv[i], yv[j], acc[i][j]);
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        if (i < nrows && j < ncols) A[static_cast<int64_t>(r_begin + i) * d + c_begin + j] = src[i][j];
     }
 }
 
@@ -225,18 +296,55 @@ __device__ __forceinline__ void load_tile(Tile64* dst, const float* A, int d, in
     }
 }
 
+// One step-by-step substitution on a 64-vector held whole in one thread's
+// registers: for s = 0 .. 63, v[s] = v[s] / L[s][s], then v[e] -= v[s] L[e][s]
+// for e > s.  LT is L transposed (LT[s][e] = L[e][s], kLTld floats per row,
+// the same address in every thread: broadcast 16-byte loads), rl[s] =
+// 1 / L[s][s].  The dependent chain is one multiply and one fma per step; the
+// updates of the later entries go two at a time (__ffma2_rn: two IEEE fmas).
+__device__ __forceinline__ void substitute64(float (&t)[kNB], const float* __restrict__ LT,
+                                             const float* __restrict__ rl)
+{
+#pragma unroll
+    for (int s = 0; s < kNB; ++s) {
+        const float v = t[s] * rl[s];
+        t[s] = v;
+        const float2 nv = make_float2(-v, -v);
+        const float4* lt = reinterpret_cast<const float4*>(LT + s * kLTld);
+#pragma unroll
+        for (int n = (s + 1) / 4; n < kNB / 4; ++n) {
+            const float4 l4 = lt[n];
+            if (4 * n > s) {
+                float2 a = make_float2(t[4 * n], t[4 * n + 1]);
+                float2 b = make_float2(t[4 * n + 2], t[4 * n + 3]);
+                a = __ffma2_rn(nv, make_float2(l4.x, l4.y), a);
+                b = __ffma2_rn(nv, make_float2(l4.z, l4.w), b);
+                t[4 * n] = a.x;
+                t[4 * n + 1] = a.y;
+                t[4 * n + 2] = b.x;
+                t[4 * n + 3] = b.y;
+            } else {   // the 16-byte group holding entry s: only the entries after it
+                const float l[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (4 * n + e > s) t[4 * n + e] = fmaf(-v, l[e], t[4 * n + e]);
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256)
     chol_panel_kernel(float* __restrict__ A, int d, int k0, int kb, int pk0,
                       float* __restrict__ Minv, PrepHeader* hdr)
 {
     extern __shared__ __align__(16) float psm[];
     Tile64* As = reinterpret_cast<Tile64*>(psm);
-    Tile64* Zs = As + kNB;
-    Tile64* Pd = Zs + kNB;       // previous panel, rows of this diagonal block
-    Tile64* Pr = Pd + kNB;       // previous panel, rows of this CTA's panel block
-    Tile64* Ts = Pr + kNB;       // this CTA's operand tile (panel rows, or a block of M^{-1})
-    float* Ys = reinterpret_cast<float*>(Ts + kNB);
-    int& bad_any = *reinterpret_cast<int*>(Ys + 32 * 33);
+    Tile64* Ts = As + kNB;       // this CTA's operand tile (panel rows, or a block of M^{-1})
+    KTile* Pd = reinterpret_cast<KTile*>(Ts + kNB);   // previous panel, rows of this diagonal block, k-major
+    KTile* Pr = Pd + kNB;        // previous panel's rows of this CTA's panel block (k-major), or Y_{k-1}
+    float* LT = reinterpret_cast<float*>(Pr + kNB);   // the factor transposed, [kNB][kLTld]
+    float* rls = LT + kNB * kLTld;                     // 1 / L[i][i]
+    int& bad_any = *reinterpret_cast<int*>(rls + kNB);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
@@ -250,21 +358,21 @@ __global__ void __launch_bounds__(256)
         if (it >= n_trsm) {
             const int cb = (it - n_trsm) * kNB;
             if (async) {
-                load_tile_async(Ts, Minv, d, k0, kb, cb, kNB);   // Y~_k
-                load_tile_async(Pr, Minv, d, pk0, kNB, cb, kNB); // Y_{k-1}
+                load_tile_async(Ts, Minv, d, k0, kb, cb, kNB);              // Y~_k
+                load_ktile_async(Pr, Minv, d, pk0, kNB, cb, kNB, false);    // Y_{k-1}, [k][c]
             } else {
                 load_tile(Ts, Minv, d, k0, kb, cb, kNB, false, false);
-                load_tile(Pr, Minv, d, pk0, kNB, cb, kNB, false, false);
+                load_ktile(Pr, Minv, d, pk0, kNB, cb, kNB, false);
             }
         } else {
             const int pr0 = k0 + kb + it * kNB;
             const int prn = min(kNB, d - pr0);
             if (async) {
                 load_tile_async(Ts, A, d, pr0, prn, k0, kb);
-                if (pk0 >= 0) load_tile_async(Pr, A, d, pr0, prn, pk0, kNB);
+                if (pk0 >= 0) load_ktile_async(Pr, A, d, pr0, prn, pk0, kNB, true);
             } else {
                 load_tile(Ts, A, d, pr0, prn, k0, kb, false, false);
-                if (pk0 >= 0) load_tile(Pr, A, d, pr0, prn, pk0, kNB, false, false);
+                if (pk0 >= 0) load_ktile(Pr, A, d, pr0, prn, pk0, kNB, true);
             }
         }
     };
@@ -276,8 +384,7 @@ __global__ void __launch_bounds__(256)
 
     // diagonal block (lower part); padding beyond kb is the identity
     load_tile(As, A, d, k0, kb, k0, kb, true, true);
-    for (int idx = tid; idx < kNB * kNB; idx += 256) Zs[idx / kNB][idx % kNB] = 0.f;
-    if (pk0 >= 0) load_tile(Pd, A, d, k0, kb, pk0, kNB, false, false);
+    if (pk0 >= 0) load_ktile(Pd, A, d, k0, kb, pk0, kNB, true);
     if (tid == 0) bad_any = 0;
     __syncthreads();
     if (pk0 >= 0) {
@@ -288,7 +395,7 @@ __global__ void __launch_bounds__(256)
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[i][j] = As[r0 + i][c0 + j];
-        if (ty >= tx) tile_minus_xyT(acc, Pd, Pd, r0, c0);
+        if (ty >= tx) tile_minus_kmajor(acc, Pd, Pd, r0, c0);
         __syncthreads();
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -393,94 +500,35 @@ __global__ void __launch_bounds__(256)
         __syncthreads();
     }
 
-    // Z = L^{-1}: diagonal 4 x 4 inverses
-    if (tid < kNB / 4) {
-        const int o = 4 * tid;
-        float l[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) l[i][j] = (j <= i) ? As[o + i][o + j] : 0.f;
-        float z[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float acc = (i == j) ? 1.f : 0.f;
-#pragma unroll
-                for (int k = 0; k < i; ++k) acc = fmaf(-l[i][k], (k >= j) ? z[k][j] : 0.f, acc);
-                z[i][j] = (i >= j) ? acc / l[i][i] : 0.f;
-            }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) Zs[o + i][o + j] = z[i][j];
+    // the factor transposed for the solves, and the reciprocals of its diagonal
+    for (int idx = tid; idx < kNB * kNB; idx += 256) {
+        const int sj = idx / kNB, e = idx % kNB;
+        LT[sj * kLTld + e] = (e >= sj) ? As[e][sj] : 0.f;
     }
-    __syncthreads();
-    // doubling: pairs of h-blocks at offsets o = p * 2h; every thread owns
-    // 2 x 2 output tiles (four independent accumulators)
-    for (int h = 4; h < kNB; h *= 2) {
-        const int hh = h / 2;
-        const int n_tiles = (kNB / (2 * h)) * hh * hh;
-        // Y = L21 Z11: Y[i][j] = sum_{k >= j} L[o+h+i][o+k] Z[o+k][o+j]
-        for (int t = tid; t < n_tiles; t += 256) {
-            const int p = t / (hh * hh), rem = t % (hh * hh);
-            const int i = 2 * (rem / hh), j = 2 * (rem % hh);
-            const int o = p * 2 * h;
-            float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-            for (int k = j; k < h; ++k) {
-                const float a0 = As[o + h + i][o + k], a1 = As[o + h + i + 1][o + k];
-                const float b0 = Zs[o + k][o + j], b1 = Zs[o + k][o + j + 1];
-                y00 = fmaf(a0, b0, y00);
-                y01 = fmaf(a0, b1, y01);
-                y10 = fmaf(a1, b0, y10);
-                y11 = fmaf(a1, b1, y11);
-            }
-            float* yp = Ys + p * h * h;
-            yp[i * h + j] = y00;
-            yp[i * h + j + 1] = y01;
-            yp[(i + 1) * h + j] = y10;
-            yp[(i + 1) * h + j + 1] = y11;
-        }
-        __syncthreads();
-        // Z21[i][j] = -sum_{k <= i} Z[o+h+i][o+h+k] Y[k][j]
-        for (int t = tid; t < n_tiles; t += 256) {
-            const int p = t / (hh * hh), rem = t % (hh * hh);
-            const int i = 2 * (rem / hh), j = 2 * (rem % hh);
-            const int o = p * 2 * h;
-            const float* yp = Ys + p * h * h;
-            float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
-            for (int k = 0; k <= i + 1; ++k) {
-                const float a0 = Zs[o + h + i][o + h + k], a1 = Zs[o + h + i + 1][o + h + k];
-                const float b0 = yp[k * h + j], b1 = yp[k * h + j + 1];
-                z00 = fmaf(a0, b0, z00);
-                z01 = fmaf(a0, b1, z01);
-                z10 = fmaf(a1, b0, z10);
-                z11 = fmaf(a1, b1, z11);
-            }
-            Zs[o + h + i][o + j] = -z00;
-            Zs[o + h + i][o + j + 1] = -z01;
-            Zs[o + h + i + 1][o + j] = -z10;
-            Zs[o + h + i + 1][o + j + 1] = -z11;
-        }
-        __syncthreads();
-    }
+    if (tid < kNB) rls[tid] = 1.f / As[tid][tid];
     if (bad) bad_any = 1;
     __syncthreads();
     if (bad_any && tid == 0 && blockIdx.x == 0) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
 
+    // the solves: one thread per row (TRSM) or column (M^{-1}) of the 64 x 64
+    // right-hand side, threads 0 .. 63
+    const int sv = tid;
+
     if (blockIdx.x == 0) {
-        // L_kk itself is not needed later (the trailing updates use the
-        // off-diagonal panels, the inverse L_kk^{-1}), and the other CTAs of
-        // this launch may still be reading the diagonal block of A, so only
-        // the diagonal block of M^{-1} is written.
+        // diagonal block of M^{-1}: L^{-1}, the solve L X = I column by column
+        // (L_kk itself is not needed later -- the trailing updates use the
+        // off-diagonal panels -- and the other CTAs of this launch may still be
+        // reading the diagonal block of A, so only M^{-1} is written)
+        if (sv < kNB) {
+            float t[kNB];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int e = 0; e < kNB; ++e) t[e] = (e == sv) ? 1.f : 0.f;
+            substitute64(t, LT, rls);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int gi = r0 + i, gj = c0 + j;
-                if (gi < kb && gj < kb) Minv[static_cast<int64_t>(k0 + gi) * d + k0 + gj] = Zs[gi][gj];
-            }
+            for (int e = 0; e < kNB; ++e) Ts[e][sv] = t[e];
+        }
+        __syncthreads();
+        store_tile(Ts, Minv, d, k0, kb, k0, kb);
         return;
     }
     cp_async_wait_all();
@@ -491,51 +539,34 @@ __global__ void __launch_bounds__(256)
         }
         __syncthreads();
         if (it >= n_trsm) {
-            // column block cb of row block k of M^{-1} (pk0 >= 0 here)
+            // column block cb of row block k of M^{-1} (pk0 >= 0 here):
+            // T = Y~_k - L_k,k-1 Y_{k-1}, then X = L_kk^{-1} T
             const int cb = (it - n_trsm) * kNB;
             float t4[4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
-            for (int k = 0; k < kNB; ++k) {
-                float a4[4], b4[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) a4[i] = Pd[r0 + i][k];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) b4[j] = Pr[k][c0 + j];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) t4[i][j] = fmaf(-a4[i], b4[j], t4[i][j]);
-            }
-            __syncthreads();
+            tile_minus_kmajor(t4, Pd, Pr, r0, c0);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = t4[i][j];
+                for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = t4[i][j];
             __syncthreads();
-            float y4[4][4] = {};
-            for (int k = 0; k < kNB; ++k) {
-                float a4[4], b4[4];
+            if (sv < kNB) {
+                float t[kNB];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) a4[i] = Zs[r0 + i][k];
+                for (int e = 0; e < kNB; ++e) t[e] = Ts[e][sv];
+                substitute64(t, LT, rls);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) b4[j] = As[k][c0 + j];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) y4[i][j] = fmaf(a4[i], b4[j], y4[i][j]);
+                for (int e = 0; e < kNB; ++e) Ts[e][sv] = t[e];
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (r0 + i < kb) Minv[static_cast<int64_t>(k0 + r0 + i) * d + cb + c0 + j] = y4[i][j];
+            __syncthreads();
+            store_tile(Ts, Minv, d, k0, kb, cb, kNB);
             continue;
         }
-        // panel rows: P[i][j] = sum_{k <= j} T[i][k] Z[j][k], with
-        // T = A[rows][block] - P_prev[rows] P_prev,kk^T
+        // panel rows: T = A[rows][block] - P_prev[rows] P_prev,kk^T, then
+        // P solves P L^T = T
         const int pr0 = k0 + kb + it * kNB;
         if (pk0 >= 0) {
             float t4[4][4];
@@ -543,33 +574,24 @@ __global__ void __launch_bounds__(256)
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
-            tile_minus_xyT(t4, Pr, Pd, r0, c0);
+            tile_minus_kmajor(t4, Pr, Pd, r0, c0);
             __syncthreads();
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = (c0 + j < kb) ? t4[i][j] : 0.f;
+                for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = t4[i][j];
             __syncthreads();
         }
-        float acc[4][4] = {};
-        for (int k = 0; k < kNB; ++k) {
-            float t[4], xv[4];
+        if (sv < kNB) {
+            float t[kNB];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) t[i] = Ts[r0 + i][k];
+            for (int e = 0; e < kNB; ++e) t[e] = (e < kb) ? Ts[sv][e] : 0.f;
+            substitute64(t, LT, rls);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) xv[j] = Zs[c0 + j][k];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(t[i], xv[j], acc[i][j]);
+            for (int e = 0; e < kNB; ++e) Ts[sv][e] = t[e];
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = pr0 + r0 + i, cj = c0 + j;
-                if (r < d && cj < kb) A[static_cast<int64_t>(r) * d + k0 + cj] = acc[i][j];
-            }
+        __syncthreads();
+        store_tile(Ts, A, d, pr0, min(kNB, d - pr0), k0, kb);
     }
 }
 

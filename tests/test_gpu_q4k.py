@@ -2,9 +2,10 @@
 checker, given the device's own factor and order (the staged parity of the
 one-level grid, with the same bar): walking each row in processing order,
 its first divergence is a code or a 6-bit level one step off at a rounding
-tie; codes, sc6 and m6 agree on >= 99.9% of entries, every code mismatch is
-one level, super-block scales agree to 1e-5 before a row's first divergence,
-and the layer-output MSE agrees to 0.5%.  The device's outputs obey
+tie; the 4-bit codes agree on >= 99.9% of entries and every code mismatch is
+one level; at most 3% of the rows diverge (the 6-bit levels carry a tie
+through the rest of a row); super-block scales agree to 1e-5 before a row's
+first divergence; and the layer-output MSE agrees to 0.5%.  The device's outputs obey
 w^ = d sc q - dmin m.  A full-size 4096 x 4096 layer is checked on sampled
 rows."""
 import numpy as np
