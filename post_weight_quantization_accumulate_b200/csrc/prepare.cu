@@ -164,7 +164,7 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
 typedef float Tile64[kNB + 1];
 constexpr int kLTld = kNB + 4;   // row pitch of k-major tiles: 16-byte aligned rows
 typedef float KTile[kLTld];
-constexpr size_t kPanelSmem = (2 * kNB * (kNB + 1) + 3 * kNB * kLTld + kNB) * sizeof(float) + 16;
+constexpr size_t kPanelSmem = (2 * kNB * (kNB + 1) + 3 * kNB * kLTld + kNB + 2 * 4 * kLTld) * sizeof(float) + 16;
 static_assert((2 * kNB * (kNB + 1) * sizeof(float)) % 16 == 0, "the k-major tiles start 16-byte aligned");
 
 // 4-byte asynchronous copy global -> shared; `valid` false writes a zero.
@@ -272,6 +272,20 @@ __device__ __forceinline__ void store_tile(const Tile64* src, float* A, int d, i
     }
 }
 
+// The same for a tile that holds the block transposed: A[r_begin + i][c_begin
+// + j] = src[j][i].
+__device__ __forceinline__ void store_tile_t(const Tile64* src, float* A, int d, int r_begin, int nrows,
+                                             int c_begin, int ncols)
+{
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        if (i < nrows && j < ncols) A[static_cast<int64_t>(r_begin + i) * d + c_begin + j] = src[j][i];
+    }
+}
+
 // 64 x 64 tile of A (rows r_begin.., columns c_begin..c_begin+ncols) into smem;
 // rows >= d or columns >= ncols read as `pad` on the diagonal, 0 elsewhere
 // (lower_only: entries above the diagonal read as 0 too).
@@ -296,40 +310,64 @@ __device__ __forceinline__ void load_tile(Tile64* dst, const float* A, int d, in
     }
 }
 
-// One step-by-step substitution on a 64-vector held whole in one thread's
-// registers: for s = 0 .. 63, v[s] = v[s] / L[s][s], then v[e] -= v[s] L[e][s]
-// for e > s.  LT is L transposed (LT[s][e] = L[e][s], kLTld floats per row,
-// the same address in every thread: broadcast 16-byte loads), rl[s] =
-// 1 / L[s][s].  The dependent chain is one multiply and one fma per step; the
-// updates of the later entries go two at a time (__ffma2_rn: two IEEE fmas).
-__device__ __forceinline__ void substitute64(float (&t)[kNB], const float* __restrict__ LT,
-                                             const float* __restrict__ rl)
+// The 64 rows of S (a 64 x 64 right-hand side in shared memory) solved in
+// place against the panel's factor: row r becomes p with p L^T = S[r], i.e.
+// for s = 0 .. 63, p[s] = S[r][s] / L[s][s] and S[r][e] -= p[s] L[e][s] for
+// e > s.  LT is L transposed (LT[s][e] = L[e][s], kLTld floats per row),
+// rls[s] = 1 / L[s][s].  Blocked by 16 columns: one thread per row solves a
+// block's 16 columns step by step (its entries in registers, L's entries by
+// broadcast loads), then all 256 threads subtract the block's product from
+// the columns to its right, 4 x 4 entries each.  Called by every thread.
+__device__ __forceinline__ void solve_rows(Tile64* S, const float* __restrict__ LT,
+                                           const float* __restrict__ rls)
 {
+    const int tid = threadIdx.x;
+    const int ty = tid >> 4, tx = tid & 15;
+#pragma unroll 1
+    for (int b = 0; b < kNB / 16; ++b) {
+        const int b0 = 16 * b;
+        if (tid < kNB) {
+            float t[16];
 #pragma unroll
-    for (int s = 0; s < kNB; ++s) {
-        const float v = t[s] * rl[s];
-        t[s] = v;
-        const float2 nv = make_float2(-v, -v);
-        const float4* lt = reinterpret_cast<const float4*>(LT + s * kLTld);
+            for (int e = 0; e < 16; ++e) t[e] = S[tid][b0 + e];
 #pragma unroll
-        for (int n = (s + 1) / 4; n < kNB / 4; ++n) {
-            const float4 l4 = lt[n];
-            if (4 * n > s) {
-                float2 a = make_float2(t[4 * n], t[4 * n + 1]);
-                float2 b = make_float2(t[4 * n + 2], t[4 * n + 3]);
-                a = __ffma2_rn(nv, make_float2(l4.x, l4.y), a);
-                b = __ffma2_rn(nv, make_float2(l4.z, l4.w), b);
-                t[4 * n] = a.x;
-                t[4 * n + 1] = a.y;
-                t[4 * n + 2] = b.x;
-                t[4 * n + 3] = b.y;
-            } else {   // the 16-byte group holding entry s: only the entries after it
-                const float l[4] = {l4.x, l4.y, l4.z, l4.w};
+            for (int s = 0; s < 16; ++s) {
+                const float v = t[s] * rls[b0 + s];
+                t[s] = v;
+                const float* lt = LT + (b0 + s) * kLTld + b0;
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (4 * n + e > s) t[4 * n + e] = fmaf(-v, l[e], t[4 * n + e]);
+                for (int e = s + 1; e < 16; ++e) t[e] = fmaf(-v, lt[e], t[e]);
             }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) S[tid][b0 + e] = t[e];
         }
+        __syncthreads();
+        const int c0 = b0 + 16 + 4 * tx;   // 4 x 4 entries: rows 4 ty .., columns c0 ..
+        if (c0 < kNB) {
+            const int r0 = 4 * ty;
+            float acc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = S[r0 + i][c0 + j];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float4 l4 = *reinterpret_cast<const float4*>(LT + (b0 + k) * kLTld + c0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float p = S[r0 + i][b0 + k];
+                    acc[i][0] = fmaf(-p, l4.x, acc[i][0]);
+                    acc[i][1] = fmaf(-p, l4.y, acc[i][1]);
+                    acc[i][2] = fmaf(-p, l4.z, acc[i][2]);
+                    acc[i][3] = fmaf(-p, l4.w, acc[i][3]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) S[r0 + i][c0 + j] = acc[i][j];
+        }
+        __syncthreads();
     }
 }
 
@@ -344,7 +382,8 @@ __global__ void __launch_bounds__(256)
     KTile* Pr = Pd + kNB;        // previous panel's rows of this CTA's panel block (k-major), or Y_{k-1}
     float* LT = reinterpret_cast<float*>(Pr + kNB);   // the factor transposed, [kNB][kLTld]
     float* rls = LT + kNB * kLTld;                     // 1 / L[i][i]
-    int& bad_any = *reinterpret_cast<int*>(rls + kNB);
+    float* LsT = rls + kNB;      // a strip's 4 columns of L, k-major, two buffers of [4][kLTld]
+    int& bad_any = *reinterpret_cast<int*>(LsT + 2 * 4 * kLTld);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
@@ -377,64 +416,109 @@ __global__ void __launch_bounds__(256)
         }
     };
 
-    // The operand tiles of the first item do not depend on the diagonal
-    // block: they are fetched asynchronously while it is factored.
+    // The diagonal block (lower part; padding beyond kb is the identity) and
+    // the previous panel's rows of it are read first, in one round trip; the
+    // operand tiles of the first item do not depend on the diagonal block, so
+    // they are fetched asynchronously afterwards, while it is factored.
+    float ta[16], tp[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        float v = (i == j) ? 1.f : 0.f;
+        if (i < kb && j <= i) v = A[static_cast<int64_t>(k0 + i) * d + k0 + j];
+        ta[t] = v;
+        tp[t] = (pk0 >= 0 && i < kb) ? A[static_cast<int64_t>(k0 + i) * d + pk0 + j] : 0.f;
+    }
     if (blockIdx.x > 0 && static_cast<int>(blockIdx.x) - 1 < n_items) fetch_item(blockIdx.x - 1, true);
     cp_async_commit();
-
-    // diagonal block (lower part); padding beyond kb is the identity
-    load_tile(As, A, d, k0, kb, k0, kb, true, true);
-    if (pk0 >= 0) load_ktile(Pd, A, d, k0, kb, pk0, kNB, true);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const int idx = tid + t * 256;
+        const int i = idx / kNB, j = idx % kNB;
+        As[i][j] = ta[t];
+        Pd[j][i] = tp[t];   // k-major
+    }
     if (tid == 0) bad_any = 0;
     __syncthreads();
-    if (pk0 >= 0) {
-        // A_kk -= P_prev,kk P_prev,kk^T (the previous panel's correction of
-        // this block column is applied here rather than in memory)
-        float acc[4][4];
+    // This thread's 4 x 4 tile of the diagonal block (tiles on and below the
+    // diagonal) stays in registers through the previous panel's correction
+    // and every strip's update; it is written back to shared memory once, at
+    // the strip before the one that needs its columns, and not re-read in
+    // between.
+    const bool own = ty >= tx;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = As[r0 + i][c0 + j];
+    // A_kk -= P_prev,kk P_prev,kk^T: the previous panel's correction of this
+    // block column, applied here rather than in memory
+    if (pk0 >= 0 && own) tile_minus_kmajor(acc, Pd, Pd, r0, c0);
+    auto flush = [&]() {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = As[r0 + i][c0 + j];
-        if (ty >= tx) tile_minus_kmajor(acc, Pd, Pd, r0, c0);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (c0 + j <= r0 + i) As[r0 + i][c0 + j] = acc[i][j];
-        __syncthreads();
-    }
+            for (int j = 0; j < 4; ++j) As[r0 + i][c0 + j] = acc[i][j];
+    };
+    if (own && tx <= 1) flush();   // the columns of strips 0 and 1
+    __syncthreads();
     bool bad = false;
 
     // Strips of 4 columns with look-ahead: while warps 1-7 subtract strip P's
-    // rank-4 product from the columns right of strip P+1, warp 0 applies it to
+    // rank-4 product from their tiles right of strip P+1, warp 0 applies it to
     // strip P+1 itself and factors that strip, so each strip costs one barrier
     // and the long update is off the chain.  Warp 0 keeps rows 4P+l and
-    // 4P+l+32 of a strip in registers (lane l).
-    auto factor_strip = [&](int cb, float (&x)[4], float (&y)[4]) {
+    // 4P+l+32 of a strip in registers (lane l), and publishes the strip's L
+    // both in As (for the solves later) and k-major in LsT (for the updates).
+    // Every lane factors the strip's 4 x 4 diagonal block itself, from the
+    // lower entries it gathers with independent shuffles, then its own rows
+    // with the same steps (so lanes 0-3, the block's rows, match it bit for
+    // bit): no shuffle waits on the previous column.
+    auto factor_strip = [&](int cb, float (&x)[4], float (&y)[4], float* ls) {
+        float D[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j <= i; ++j) D[i][j] = __shfl_sync(0xffffffffu, x[j], i);
+        float rs[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            float piv = __shfl_sync(0xffffffffu, x[c], c);
+            float piv = D[c][c];
             if (!(piv > 0.f) || !isfinite(piv)) {
                 bad = true;
                 piv = 1.f;
             }
-            const float rs = rsqrtf(piv);
-            const float lx = x[c] * rs, ly = y[c] * rs;
+            rs[c] = rsqrtf(piv);
+#pragma unroll
+            for (int i = c; i < 4; ++i) D[i][c] = D[i][c] * rs[c];
+#pragma unroll
+            for (int j = c + 1; j < 4; ++j)
+#pragma unroll
+                for (int i = j; i < 4; ++i) D[i][j] = fmaf(-D[i][c], D[j][c], D[i][j]);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float lx = x[c] * rs[c], ly = y[c] * rs[c];
             x[c] = lx;
             y[c] = ly;
 #pragma unroll
             for (int j = c + 1; j < 4; ++j) {
-                const float lj = __shfl_sync(0xffffffffu, lx, j);   // row cb+j, column c
-                x[j] = fmaf(-lx, lj, x[j]);
-                y[j] = fmaf(-ly, lj, y[j]);
+                x[j] = fmaf(-lx, D[j][c], x[j]);
+                y[j] = fmaf(-ly, D[j][c], y[j]);
             }
         }
         const int ra = cb + lane, rb = cb + lane + 32;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-            if (ra < kNB) As[ra][cb + t] = x[t];
-            if (rb < kNB) As[rb][cb + t] = y[t];
+            if (ra < kNB) {
+                As[ra][cb + t] = x[t];
+                ls[t * kLTld + ra] = x[t];
+            }
+            if (rb < kNB) {
+                As[rb][cb + t] = y[t];
+                ls[t * kLTld + rb] = y[t];
+            }
         }
     };
     if (warp == 0) {
@@ -444,11 +528,12 @@ __global__ void __launch_bounds__(256)
             x[t] = As[lane][t];
             y[t] = As[lane + 32][t];
         }
-        factor_strip(0, x, y);
+        factor_strip(0, x, y, LsT);
     }
     __syncthreads();
     for (int P = 0; P < kNB / 4; ++P) {
         const int cb = 4 * P;
+        const float* lcur = LsT + (P & 1) * 4 * kLTld;   // strip P, k-major
         if (warp == 0) {
             if (P + 1 < kNB / 4) {
                 const int nb = cb + 4;
@@ -457,12 +542,12 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
                 for (int t = 0; t < 4; ++t)
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) lstrip[t][u] = As[nb + t][cb + u];
+                    for (int u = 0; u < 4; ++u) lstrip[t][u] = lcur[u * kLTld + nb + t];
                 float x[4], y[4], la[4], lb[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    la[u] = ra < kNB ? As[ra][cb + u] : 0.f;
-                    lb[u] = rb < kNB ? As[rb][cb + u] : 0.f;
+                    la[u] = ra < kNB ? lcur[u * kLTld + ra] : 0.f;
+                    lb[u] = rb < kNB ? lcur[u * kLTld + rb] : 0.f;
                 }
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
@@ -476,26 +561,30 @@ __global__ void __launch_bounds__(256)
                     x[t] = xa;
                     y[t] = ya;
                 }
-                factor_strip(nb, x, y);
+                factor_strip(nb, x, y, LsT + ((P + 1) & 1) * 4 * kLTld);
             }
-        } else if (tx > P + 1 && ty >= tx) {
-            float li[4][4], lj[4][4];
+        } else if (own && tx > P + 1) {
+            float li[4][4], lj[4][4];   // L[r0 + i][cb + t], L[c0 + j][cb + t]
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float4 a4 = *reinterpret_cast<const float4*>(lcur + t * kLTld + r0);
+                const float4 b4 = *reinterpret_cast<const float4*>(lcur + t * kLTld + c0);
+                li[0][t] = a4.x;
+                li[1][t] = a4.y;
+                li[2][t] = a4.z;
+                li[3][t] = a4.w;
+                lj[0][t] = b4.x;
+                lj[1][t] = b4.y;
+                lj[2][t] = b4.z;
+                lj[3][t] = b4.w;
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    li[i][t] = As[r0 + i][cb + t];
-                    lj[i][t] = As[c0 + i][cb + t];
-                }
+                for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float acc = As[r0 + i][c0 + j];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) acc = fmaf(-li[i][t], lj[j][t], acc);
-                    As[r0 + i][c0 + j] = acc;
-                }
+                    for (int t = 0; t < 4; ++t) acc[i][j] = fmaf(-li[i][t], lj[j][t], acc[i][j]);
+            if (tx == P + 2) flush();   // warp 0 reads these columns next strip
         }
         __syncthreads();
     }
@@ -510,25 +599,17 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     if (bad_any && tid == 0 && blockIdx.x == 0) atomicCAS(&hdr->status, 0, GPTQ_ERR_NOT_PD);
 
-    // the solves: one thread per row (TRSM) or column (M^{-1}) of the 64 x 64
-    // right-hand side, threads 0 .. 63
-    const int sv = tid;
 
     if (blockIdx.x == 0) {
         // diagonal block of M^{-1}: L^{-1}, the solve L X = I column by column
         // (L_kk itself is not needed later -- the trailing updates use the
         // off-diagonal panels -- and the other CTAs of this launch may still be
         // reading the diagonal block of A, so only M^{-1} is written)
-        if (sv < kNB) {
-            float t[kNB];
-#pragma unroll
-            for (int e = 0; e < kNB; ++e) t[e] = (e == sv) ? 1.f : 0.f;
-            substitute64(t, LT, rls);
-#pragma unroll
-            for (int e = 0; e < kNB; ++e) Ts[e][sv] = t[e];
-        }
+        // (the transposed problem: rows of X^T solve X^T L^T = I)
+        for (int idx = tid; idx < kNB * kNB; idx += 256) Ts[idx / kNB][idx % kNB] = (idx / kNB == idx % kNB) ? 1.f : 0.f;
         __syncthreads();
-        store_tile(Ts, Minv, d, k0, kb, k0, kb);
+        solve_rows(Ts, LT, rls);
+        store_tile_t(Ts, Minv, d, k0, kb, k0, kb);
         return;
     }
     cp_async_wait_all();
@@ -548,21 +629,15 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) t4[i][j] = Ts[r0 + i][c0 + j];
             tile_minus_kmajor(t4, Pd, Pr, r0, c0);
+            // T transposed into As (the factor lives on in LT): the rows of
+            // X^T solve X^T L^T = T^T
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = t4[i][j];
+                for (int j = 0; j < 4; ++j) As[c0 + j][r0 + i] = t4[i][j];
             __syncthreads();
-            if (sv < kNB) {
-                float t[kNB];
-#pragma unroll
-                for (int e = 0; e < kNB; ++e) t[e] = Ts[e][sv];
-                substitute64(t, LT, rls);
-#pragma unroll
-                for (int e = 0; e < kNB; ++e) Ts[e][sv] = t[e];
-            }
-            __syncthreads();
-            store_tile(Ts, Minv, d, k0, kb, cb, kNB);
+            solve_rows(As, LT, rls);
+            store_tile_t(As, Minv, d, k0, kb, cb, kNB);
             continue;
         }
         // panel rows: T = A[rows][block] - P_prev[rows] P_prev,kk^T, then
@@ -582,15 +657,7 @@ __global__ void __launch_bounds__(256)
                 for (int j = 0; j < 4; ++j) Ts[r0 + i][c0 + j] = t4[i][j];
             __syncthreads();
         }
-        if (sv < kNB) {
-            float t[kNB];
-#pragma unroll
-            for (int e = 0; e < kNB; ++e) t[e] = (e < kb) ? Ts[sv][e] : 0.f;
-            substitute64(t, LT, rls);
-#pragma unroll
-            for (int e = 0; e < kNB; ++e) Ts[sv][e] = t[e];
-        }
-        __syncthreads();
+        solve_rows(Ts, LT, rls);
         store_tile(Ts, A, d, pr0, min(kNB, d - pr0), k0, kb);
     }
 }
