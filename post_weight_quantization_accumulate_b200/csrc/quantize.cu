@@ -701,6 +701,34 @@ __global__ void finish_kernel(const uint8_t* __restrict__ codes_p, const float* 
     }
 }
 
+// finish_kernel's work for a layer without a permutation (W^ is already in
+// place), 8 columns per thread with 8-byte loads of the codes and 8- and
+// 4-byte stores; the caller's codes and packed buffers must be 8- and 4-byte
+// aligned (checked on the host).
+__global__ void finish_noperm_kernel(const uint8_t* __restrict__ codes_p, int d_out, int d_in,
+                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ packed)
+{
+    const int per_row = d_in / 8;
+    const int64_t n = static_cast<int64_t>(d_out) * per_row;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / per_row;
+        const int g = static_cast<int>(idx - r * per_row);
+        const int64_t off = r * d_in + 8 * g;
+        const uint2 q = *reinterpret_cast<const uint2*>(codes_p + off);
+        if (codes) *reinterpret_cast<uint2*>(codes + off) = q;
+        if (packed) {
+            // bytes b0..b7 of q -> nibbles: byte k of the result = b(2k) | b(2k+1) << 4
+            const uint32_t lo = q.x, hi = q.y;
+            const uint32_t p0 = (lo & 0x0F) | ((lo >> 4) & 0xF0);                 // bytes 0, 1
+            const uint32_t p1 = ((lo >> 16) & 0x0F) | ((lo >> 20) & 0xF0);        // bytes 2, 3
+            const uint32_t p2 = (hi & 0x0F) | ((hi >> 4) & 0xF0);
+            const uint32_t p3 = ((hi >> 16) & 0x0F) | ((hi >> 20) & 0xF0);
+            *reinterpret_cast<uint32_t*>(packed + r * (d_in / 2) + 4 * g) = p0 | (p1 << 8) | (p2 << 16) | (p3 << 24);
+        }
+    }
+}
+
 __global__ void g_idx_kernel(const int32_t* __restrict__ perm, int d, int gs, int32_t* __restrict__ g_idx)
 {
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
@@ -966,10 +994,14 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         }
     }
     if (codes || packed || perm) {
+        const bool vec_ok = (reinterpret_cast<uintptr_t>(codes) % 8 == 0) &&
+                            (reinterpret_cast<uintptr_t>(packed) % 4 == 0);
         if (perm && d_in <= kRowStageMax)
             finish_rows_kernel<<<std::min(d_out, 2 * nsm), kRowThreads,
                                  static_cast<size_t>(d_in) * (sizeof(float) + 1), stream>>>(
                 codes_p, Wp, inv, d_out, d_in, W, codes, packed, status);
+        else if (!perm && vec_ok)
+            finish_noperm_kernel<<<nsm * 8, 256, 0, stream>>>(codes_p, d_out, d_in, codes, packed);
         else
             finish_kernel<<<nsm * 8, 256, 0, stream>>>(codes_p, Wp, perm ? inv : nullptr, d_out, d_in,
                                                        W, codes, packed, status);
