@@ -465,8 +465,10 @@ def run_w4a16(args, rank) -> int:
            "config": {"workload": "w4a16_llama2_7b_decode", "layers": L, "group_size": gs,
                       "shapes": [list(x) for x in W4A16_SHAPES], "l2": "weights > L2 (0.46 GB)"}}
     lines = {}
+    paths = {1: ((B.W4A16_AUTO, "auto"), (B.W4A16_TENSOR_CORE, "tensor_core"), (B.W4A16_GENERAL, "general")),
+             16: ((B.W4A16_AUTO, "auto"), (B.W4A16_GENERAL, "general"))}
     for M in (1, 16):
-        for path, pname in ((B.W4A16_TENSOR_CORE, "tensor_core"), (B.W4A16_GENERAL, "general")):
+        for path, pname in paths[M]:
             ops, wbytes = [], 0
             for name, N, K in W4A16_SHAPES:
                 x, p, sc, z, _ = synth.w4a16_operands(11, M, N, K, gs)
@@ -505,7 +507,7 @@ def run_w4a16(args, rank) -> int:
                                       "frac_of_hbm": gbs / peaks["hbm_gbs"], "clocks": clk.summary()}
             del g, ops
             torch.cuda.empty_cache()
-    head = lines["M1_tensor_core"]
+    head = lines["M1_auto"]   # M = 1 takes the decode path, M = 16 the tensor-core path
     out.update({"value": head["gbs"], "ms_per_step": head["ms_per_step"], "gpu_launches": head["launches_per_step"] * max(args.steps, 400),
                 "roofline": {"bound": "hbm", "achieved": head["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": head["frac_of_hbm"], "peak_source": src, "traffic": None},

@@ -323,7 +323,7 @@ int gptq_selftest_bounded_wait(int64_t limit_cycles);
 int gptq_selftest_quotient(int64_t n_pairs, uint64_t seed, int64_t* mismatches);
 
 /* Paths of gptq_w4a16_gemm. */
-enum { GPTQ_W4A16_AUTO = 0, GPTQ_W4A16_TENSOR_CORE = 1, GPTQ_W4A16_GENERAL = 2 };
+enum { GPTQ_W4A16_AUTO = 0, GPTQ_W4A16_TENSOR_CORE = 1, GPTQ_W4A16_GENERAL = 2, GPTQ_W4A16_DECODE = 3 };
 
 /*
  * Y = X W^T with W^ the dequantized 4-bit weights gptq_quantize writes: the
@@ -340,16 +340,21 @@ enum { GPTQ_W4A16_AUTO = 0, GPTQ_W4A16_TENSOR_CORE = 1, GPTQ_W4A16_GENERAL = 2 }
  *               integer values 0..15; n_groups = K / group_size (1 for -1).
  *   g_idx       int32 [K] or NULL (groups contiguous along K).
  *   M >= 0, N >= 0, K > 0 with K % 8 == 0; group_size -1 or dividing K.
- *   path        GPTQ_W4A16_AUTO picks the tensor-core path when it applies:
- *               g_idx NULL, K % 32 == 0, group_size dividing 128 (a multiple
- *               of 16) or a multiple of 128 or -1.  GPTQ_W4A16_TENSOR_CORE
- *               asks for it (GPTQ_ERR_INVALID_ARG when it does not apply);
- *               GPTQ_W4A16_GENERAL takes the SIMT path for any layout.
+ *   path        GPTQ_W4A16_AUTO picks the decode path for M <= 4 when it
+ *               applies (g_idx NULL, K % 32 == 0, group_size a multiple of
+ *               32 or -1), else the tensor-core path when it applies: g_idx
+ *               NULL, K % 32 == 0, group_size dividing 128 (a multiple of 16)
+ *               or a multiple of 128 or -1.  GPTQ_W4A16_TENSOR_CORE and
+ *               GPTQ_W4A16_DECODE ask for their path (GPTQ_ERR_INVALID_ARG
+ *               when it does not apply); GPTQ_W4A16_GENERAL takes the SIMT
+ *               path for any layout.
  * Tensor-core path: Y = sum_g s * (sum over the group's columns of
  * (q - z) x), the inner sums exact bf16 products accumulated in fp32 on
  * tcgen05 (q - z is exact in bf16), the scale applied per group; split-K
  * partial sums are added in a fixed order, so results are deterministic.
- * General path: fp32 W^ = s * (q - z) and fp32 dot products.  Both are
+ * Decode path (M <= 4): the weights streamed once with 16-byte loads, per
+ * 32-column chunk the fp32 sum of (q - z) x (exact q - z), scaled once.
+ * General path: fp32 W^ = s * (q - z) and fp32 dot products.  All are
  * X W^T up to fp32 rounding of the sums.  Stream-ordered; allocates nothing.
  * Y must not overlap the inputs.
  */

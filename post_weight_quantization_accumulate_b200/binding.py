@@ -49,7 +49,7 @@ SIGNATURES = [
     ("gptq_bf16_to_f32", _I, [_P, _P, _I64, _P]),
 ]
 
-W4A16_AUTO, W4A16_TENSOR_CORE, W4A16_GENERAL = 0, 1, 2
+W4A16_AUTO, W4A16_TENSOR_CORE, W4A16_GENERAL, W4A16_DECODE = 0, 1, 2, 3
 
 _lib = None
 _lock = threading.Lock()

@@ -28,6 +28,7 @@ int run_hessian_f32(float* H, const float* X, int64_t n, int64_t d, int64_t chun
                     cudaStream_t s);
 bool w4a16_tc_supported(const uint16_t* X, const uint8_t* packed, const int32_t* g_idx,
                         int64_t K, int gs);
+bool gemv_supported(const int32_t* g_idx, int64_t M, int64_t K, int gs);
 int run_w4a16(float* Y, const uint16_t* X, const uint8_t* packed, const float* scales,
               const float* zeros, const int32_t* g_idx, int64_t M, int64_t N, int64_t K, int gs,
               int path, cudaStream_t stream);
@@ -404,7 +405,7 @@ int gptq_w4a16_gemm(float* Y, const uint16_t* X, const uint8_t* packed, const fl
 {
     if (M < 0 || N < 0 || K <= 0 || K % 8 != 0 || K > (int64_t(1) << 30) ||
         M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || M * N > (int64_t(1) << 40) ||
-        path < GPTQ_W4A16_AUTO || path > GPTQ_W4A16_GENERAL)
+        path < GPTQ_W4A16_AUTO || path > GPTQ_W4A16_DECODE)
         return GPTQ_ERR_INVALID_ARG;
     if (group_size != -1 && (group_size <= 0 || K % group_size != 0)) return GPTQ_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return GPTQ_OK;
@@ -413,6 +414,7 @@ int gptq_w4a16_gemm(float* Y, const uint16_t* X, const uint8_t* packed, const fl
         return GPTQ_ERR_INVALID_ARG;
     if (path == GPTQ_W4A16_TENSOR_CORE && !w4a16_tc_supported(X, packed, g_idx, K, group_size))
         return GPTQ_ERR_INVALID_ARG;
+    if (path == GPTQ_W4A16_DECODE && !gemv_supported(g_idx, M, K, group_size)) return GPTQ_ERR_INVALID_ARG;
     int rc = check_device();
     if (rc) return rc;
     return run_w4a16(Y, X, packed, scales, zeros, g_idx, M, N, K, group_size, path,

@@ -126,6 +126,139 @@ __global__ void __launch_bounds__(kWThreads)
     }
 }
 
+// ------------------------------------------------------------ decode path
+// For at most four rows of activations the product is a matrix-vector
+// product per row: about 2 M flops per half-byte of weights, so the issue
+// rate of the SIMT pipes, not the tensor cores, decides whether the weights
+// stream at HBM speed.  The packed bytes are read once with 16-byte loads
+// and never staged.  Work unit: a block of kGvWarps warps owns kGvRows
+// weight rows; lane l of warp w takes the 32-column chunks
+// c = l + 32 w, l + 32 (w + kGvWarps), ... of all kGvRows rows, so one read of
+// the chunk's activations (64 bytes per activation row, from L1) serves
+// kGvRows weight rows.  Per 8-column word: four bf16 pairs 128 + q from the
+// exponent trick (columns (i, i + 4)), minus the pair 128 + z (exact: q - z
+// is an integer of at most 15 in magnitude), then one mixed-precision FMA per
+// column, bf16 (q - z) times bf16 x accumulated in fp32 (the product is
+// exact in fp32).  The chunk's sum is scaled once: acc += s * dot.  Lanes
+// and then warps are reduced in a fixed order (deterministic).  Needs
+// K % 32 == 0 and groups of a multiple of 32 columns (or one group per row),
+// contiguous along K, zeros integer-valued in 0..15.
+constexpr int kGvRows = 4;
+constexpr int kGvWarps = 4;
+
+__device__ __forceinline__ float fma_f32_bf16(uint32_t a, uint32_t b, float c)
+{
+    // a, b: bf16 in the low 16 bits
+    float d;
+    asm("fma.rn.f32.bf16 %0, %1, %2, %3;"
+        : "=f"(d)
+        : "h"(static_cast<uint16_t>(a)), "h"(static_cast<uint16_t>(b)), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+template <int MM>
+__global__ void __launch_bounds__(kGvWarps * 32)
+    w4a16_gemv_kernel(float* __restrict__ Y, const uint16_t* __restrict__ X,
+                      const uint8_t* __restrict__ packed, const float* __restrict__ scales,
+                      const float* __restrict__ zeros, int N, int K, int gs, int ng)
+{
+    __shared__ float red[kGvWarps][kGvRows * MM];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int chunks = K >> 5;
+    const int64_t row_bytes = K / 2;
+    for (int n0 = blockIdx.x * kGvRows; n0 < N; n0 += gridDim.x * kGvRows) {
+        float acc[kGvRows][MM];
+#pragma unroll
+        for (int r = 0; r < kGvRows; ++r)
+#pragma unroll
+            for (int m = 0; m < MM; ++m) acc[r][m] = 0.f;
+#pragma unroll(MM <= 2 ? 2 : 1)
+        for (int c = lane + 32 * warp; c < chunks; c += 32 * kGvWarps) {
+            const int g = gs > 0 ? (32 * c) / gs : 0;
+            uint4 q4[kGvRows];
+            float s[kGvRows];
+            uint32_t zb[kGvRows];
+#pragma unroll
+            for (int r = 0; r < kGvRows; ++r) {
+                const int n = min(n0 + r, N - 1);   // rows past N repeat row N - 1 and are not stored
+                q4[r] = __ldcs(reinterpret_cast<const uint4*>(packed + n * row_bytes) + c);
+                s[r] = __ldg(scales + static_cast<int64_t>(n) * ng + g);
+                zb[r] = 0x43004300u + static_cast<uint32_t>(__ldg(zeros + static_cast<int64_t>(n) * ng + g)) * 0x00010001u;
+            }
+#pragma unroll
+            for (int m = 0; m < MM; ++m) {
+                const uint4* xp = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K + 32 * c);
+                uint4 xv[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) xv[v] = __ldg(xp + v);   // 8 bf16: columns 32c + 8v .. + 7
+#pragma unroll
+                for (int r = 0; r < kGvRows; ++r) {
+                    const uint32_t qw[4] = {q4[r].x, q4[r].y, q4[r].z, q4[r].w};
+                    float dot = 0.f;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const uint32_t w = qw[v];
+                        const uint32_t xw[4] = {xv[v].x, xv[v].y, xv[v].z, xv[v].w};
+                        // (q - z) pairs for columns (0, 4), (1, 5), (2, 6), (3, 7) of the word
+                        const uint32_t p0 = sub_bf16x2((w & 0x000F000Fu) | 0x43004300u, zb[r]);
+                        const uint32_t p1 = sub_bf16x2(((w >> 4) & 0x000F000Fu) | 0x43004300u, zb[r]);
+                        const uint32_t p2 = sub_bf16x2(((w >> 8) & 0x000F000Fu) | 0x43004300u, zb[r]);
+                        const uint32_t p3 = sub_bf16x2(((w >> 12) & 0x000F000Fu) | 0x43004300u, zb[r]);
+                        dot = fma_f32_bf16(p0, xw[0], dot);
+                        dot = fma_f32_bf16(p1, xw[0] >> 16, dot);
+                        dot = fma_f32_bf16(p2, xw[1], dot);
+                        dot = fma_f32_bf16(p3, xw[1] >> 16, dot);
+                        dot = fma_f32_bf16(p0 >> 16, xw[2], dot);
+                        dot = fma_f32_bf16(p1 >> 16, xw[2] >> 16, dot);
+                        dot = fma_f32_bf16(p2 >> 16, xw[3], dot);
+                        dot = fma_f32_bf16(p3 >> 16, xw[3] >> 16, dot);
+                    }
+                    acc[r][m] = fmaf(s[r], dot, acc[r][m]);
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kGvRows; ++r)
+#pragma unroll
+            for (int m = 0; m < MM; ++m)
+#pragma unroll
+                for (int o = 16; o; o >>= 1) acc[r][m] += __shfl_xor_sync(0xffffffffu, acc[r][m], o);
+        if (lane == 0) {
+#pragma unroll
+            for (int r = 0; r < kGvRows; ++r)
+#pragma unroll
+                for (int m = 0; m < MM; ++m) red[warp][r * MM + m] = acc[r][m];
+        }
+        __syncthreads();
+        if (threadIdx.x < kGvRows * MM) {
+            const int r = threadIdx.x / MM, m = threadIdx.x % MM;
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < kGvWarps; ++w) t += red[w][threadIdx.x];
+            if (n0 + r < N) Y[static_cast<int64_t>(m) * N + n0 + r] = t;
+        }
+        __syncthreads();
+    }
+}
+
+template <int MM>
+int launch_gemv(float* Y, const uint16_t* X, const uint8_t* packed, const float* scales,
+                const float* zeros, int N, int K, int gs, int ng, cudaStream_t stream)
+{
+    const int64_t tiles = (static_cast<int64_t>(N) + kGvRows - 1) / kGvRows;
+    const int blocks = static_cast<int>(std::min<int64_t>(tiles, int64_t(1) << 30));
+    w4a16_gemv_kernel<MM><<<blocks, kGvWarps * 32, 0, stream>>>(Y, X, packed, scales, zeros, N, K, gs, ng);
+    GPTQ_LAUNCH_CHECK();
+    return GPTQ_OK;
+}
+
 // ------------------------------------------------------- tensor-core path
 constexpr int kRows = 128;          // weight rows per tile = MMA M
 constexpr int kStageCols = 128;     // K columns per stage
@@ -696,6 +829,11 @@ int launch_tc(float* Y, const uint16_t* X, const uint8_t* packed, const float* s
 // The tensor-core path takes groups contiguous along K whose length divides
 // the 128-column stage or is a multiple of it (or one group per row), K a
 // multiple of 32 (16-byte rows of packed codes) and 16-byte aligned operands.
+bool gemv_supported(const int32_t* g_idx, int64_t M, int64_t K, int gs)
+{
+    return !g_idx && M >= 1 && M <= 4 && K % 32 == 0 && (gs <= 0 || gs % 32 == 0);
+}
+
 bool w4a16_tc_supported(const uint16_t* X, const uint8_t* packed, const int32_t* g_idx,
                         int64_t K, int gs)
 {
@@ -711,6 +849,15 @@ int run_w4a16(float* Y, const uint16_t* X, const uint8_t* packed, const float* s
               int path, cudaStream_t stream)
 {
     const int ng = gs > 0 ? static_cast<int>(K / gs) : 1;
+    if (path == 3 || (path == 0 && gemv_supported(g_idx, M, K, gs))) {
+        const int Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+        switch (M) {
+            case 1: return launch_gemv<1>(Y, X, packed, scales, zeros, Ni, Ki, gs, ng, stream);
+            case 2: return launch_gemv<2>(Y, X, packed, scales, zeros, Ni, Ki, gs, ng, stream);
+            case 3: return launch_gemv<3>(Y, X, packed, scales, zeros, Ni, Ki, gs, ng, stream);
+            default: return launch_gemv<4>(Y, X, packed, scales, zeros, Ni, Ki, gs, ng, stream);
+        }
+    }
     const bool tc = path == 1 || (path == 0 && w4a16_tc_supported(X, packed, g_idx, K, gs));
     if (tc) {
         const int gs_e = gs > 0 ? gs : static_cast<int>(K);

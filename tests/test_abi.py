@@ -110,7 +110,7 @@ def test_w4a16_arguments_rejected_on_host(lib):
     assert w(M=-1) == 1
     assert w(gs=100) == 1            # does not divide K
     assert w(gs=0) == 1
-    assert w(path=3) == 1
+    assert w(path=4) == 1            # no such path
     assert w(X=None) == 1
     assert w(Y=None) == 1
     assert w(X=P((1 << 20) + 2)) == 1       # X not 16-byte aligned
@@ -119,6 +119,12 @@ def test_w4a16_arguments_rejected_on_host(lib):
     assert w(path=1, g_idx=fake) == 1       # groups given per column
     assert w(path=1, K=264, gs=-1) == 1     # K not a multiple of 32
     assert w(path=1, K=192, gs=48) == 1     # group neither divides nor is a multiple of 128
+    # the decode path refuses more than 4 rows, scattered groups, groups of fewer
+    # than 32 columns and K not a multiple of 32
+    assert w(path=3, M=5) == 1
+    assert w(path=3, g_idx=fake) == 1
+    assert w(path=3, gs=16) == 1
+    assert w(path=3, K=264, gs=-1) == 1
     # empty products are done without a device
     assert w(M=0) == 0
     assert w(N=0) == 0

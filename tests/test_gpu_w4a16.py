@@ -1,7 +1,7 @@
 """The 4-bit linear (Y = X W^T from the packed codes, scales, zeros and group
 map) on the device against the float64 checker, element by element.
 
-Tolerance, from the arithmetic: both paths form sums of K products of bf16
+Tolerance, from the arithmetic: every path forms sums of K products of bf16
 activations with W^ = s (q - z) (exact in fp32 on the general path; exact bf16
 products scaled once per group on the tensor-core path) in fp32, so an output
 differs from the exact sum by at most about 2 K u sum_k |x_k W^_k| with
@@ -73,6 +73,37 @@ def test_w4a16_tensor_core_path(M, N, K, gs):
     ops = synth.w4a16_operands(1, M, N, K, gs)
     Y = _run(*ops, gs, B.W4A16_TENSOR_CORE)
     _check(Y, *ops, gs, f"tc {M}x{N}x{K} g{gs}")
+
+
+# decode path (M <= 4): ragged row counts, groups of 32 .. 256 columns and one
+# group per row, a chunk count that is not a multiple of the 32 lanes
+# (K = 11008: 344 chunks), every M from 1 to 4
+GEMV_CASES = [
+    (1, 384, 1024, 128),
+    (2, 77, 512, 32),
+    (3, 130, 11008, 128),
+    (4, 64, 2048, 256),
+    (1, 1000, 4096, -1),
+    (1, 33, 96, 32),
+]
+
+
+@pytest.mark.parametrize("M,N,K,gs", GEMV_CASES)
+def test_w4a16_decode_path(M, N, K, gs):
+    ops = synth.w4a16_operands(4, M, N, K, gs)
+    Y = _run(*ops, gs, B.W4A16_DECODE)
+    _check(Y, *ops, gs, f"decode {M}x{N}x{K} g{gs}")
+    # the automatic choice takes the same path for these shapes
+    np.testing.assert_array_equal(_run(*ops, gs, B.W4A16_AUTO), Y)
+
+
+def test_w4a16_decode_path_refuses_what_it_cannot_do():
+    ops = synth.w4a16_operands(5, 5, 64, 512, 128)   # M > 4
+    with pytest.raises(B.GptqError):
+        _run(*ops, 128, B.W4A16_DECODE)
+    ops = synth.w4a16_operands(5, 2, 64, 512, 16)    # groups of 16 columns
+    with pytest.raises(B.GptqError):
+        _run(*ops, 16, B.W4A16_DECODE)
 
 
 @pytest.mark.parametrize("M,N,K,gs", [(1, 384, 1024, 128), (9, 77, 520, 8), (3, 64, 96, -1)])
