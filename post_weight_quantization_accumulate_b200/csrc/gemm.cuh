@@ -21,6 +21,9 @@ enum GemmFlags : int {
 // floats (the TMA rules), else on the SIMT kernel (gemm_simt.cu).
 // max_ctas > 0 caps the number of CTAs (and so of SMs) the product occupies,
 // which leaves SMs free for latency-critical work on another stream.
+// max_ctas < 0: one CTA per output tile (tensor-core path) instead of at most
+// one per SM looping over tiles, so the product's CTAs retire tile by tile
+// and work of higher-priority streams gets SMs as they free up.
 // A_lo, B_lo (optional, same layout and strides as A and B): the operands'
 // low parts x - trunc_tf32(x), prepared by the caller; with both given the
 // tensor-core path skips its conversion pass and uses 128 x 256 tiles.

@@ -598,8 +598,9 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     g.n_nt = (N + tn - 1) / tn;
     g.status = device_status_ptr();
     const int64_t units = static_cast<int64_t>(g.n_mt) * g.n_nt * batch;
-    int cap = sm_count();
+    int64_t cap = sm_count();
     if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;
+    if (max_ctas < 0) cap = units;   // one CTA per tile
     const int grid = static_cast<int>(units < cap ? units : cap);
     if (prelo)
         GPTQ_CUDA_CHECK(launch_k(gemm_tc_kernel<256, true>, dim3(grid), dim3(TTHREADS),

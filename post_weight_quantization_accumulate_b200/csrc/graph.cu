@@ -93,7 +93,7 @@ int run_graphed(const std::vector<uint64_t>& key, bool want_status,
         if (e.status_host) cudaFreeHost(e.status_host);
         return rc ? rc : cuda_fail(ce);
     }
-    ce = cudaGraphInstantiate(&e.exec, graph, 0);
+    ce = cudaGraphInstantiate(&e.exec, graph, cudaGraphInstantiateFlagUseNodePriority);
     cudaGraphDestroy(graph);
     if (ce != cudaSuccess) {
         if (e.status_host) cudaFreeHost(e.status_host);

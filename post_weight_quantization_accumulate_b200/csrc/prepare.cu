@@ -675,15 +675,19 @@ __global__ void reverse_upper_kernel(const float* __restrict__ Minv, int d, floa
 
 }  // namespace
 
-// Second stream of the factorisation (one per device, created on first use)
-// with its events; the caller's stream forks to it and joins it again.
+// Side streams of the factorisation (one set per device, created on first
+// use) with their events; the caller's stream forks to them and joins them.
 struct SideStream {
     static constexpr int kRing = 4;
-    cudaStream_t s = nullptr;          // trailing symmetric updates of A
-    cudaStream_t s2 = nullptr;         // updates of the lower rows of M^{-1}
-    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr, done_panel = nullptr;
-    cudaEvent_t cleared = nullptr;
-    cudaEvent_t ev[kRing] = {}, ev2[kRing] = {};
+    cudaStream_t sp = nullptr;         // the chain of panel kernels
+    cudaStream_t s = nullptr;          // narrow and band updates of A
+    cudaStream_t s2 = nullptr;         // narrow and band updates of M^{-1}
+    cudaStream_t s3 = nullptr;         // far updates of A
+    cudaStream_t s4 = nullptr;         // far updates of M^{-1}
+    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr, join3 = nullptr, join4 = nullptr;
+    cudaEvent_t ready = nullptr, join_p = nullptr, done_panel = nullptr, cleared = nullptr;
+    cudaEvent_t ev[kRing] = {}, ev2[kRing] = {};     // narrow/band work of a panel done
+    cudaEvent_t far[kRing] = {}, far2[kRing] = {};   // far update of a batch done
 };
 
 static int side_stream(SideStream** out)
@@ -696,19 +700,24 @@ static int side_stream(SideStream** out)
     std::lock_guard<std::mutex> lk(mu);
     SideStream& st = streams[dev];
     if (!st.s) {
-        // lowest priority: CTAs of the panel chain are placed first on free SMs
+        // the panel chain and the products it waits for at the highest
+        // priority, the far updates at the lowest: when a far product's CTA
+        // retires, a waiting CTA of the chain takes the SM first
         int lo = 0, hi = 0;
         GPTQ_CUDA_CHECK(cudaDeviceGetStreamPriorityRange(&lo, &hi));
-        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s, cudaStreamNonBlocking, lo));
-        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s2, cudaStreamNonBlocking, lo));
-        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming));
-        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming));
-        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.join2, cudaEventDisableTiming));
-        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.done_panel, cudaEventDisableTiming));
-        GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.cleared, cudaEventDisableTiming));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.sp, cudaStreamNonBlocking, hi));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s, cudaStreamNonBlocking, hi));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s2, cudaStreamNonBlocking, hi));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s3, cudaStreamNonBlocking, lo));
+        GPTQ_CUDA_CHECK(cudaStreamCreateWithPriority(&st.s4, cudaStreamNonBlocking, lo));
+        for (cudaEvent_t* e : {&st.fork, &st.join, &st.join2, &st.join3, &st.join4, &st.ready,
+                               &st.join_p, &st.done_panel, &st.cleared})
+            GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
         for (int i = 0; i < SideStream::kRing; ++i) {
             GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.ev[i], cudaEventDisableTiming));
             GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.ev2[i], cudaEventDisableTiming));
+            GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.far[i], cudaEventDisableTiming));
+            GPTQ_CUDA_CHECK(cudaEventCreateWithFlags(&st.far2[i], cudaEventDisableTiming));
         }
     }
     *out = &st;
@@ -737,6 +746,8 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
     GPTQ_CUDA_CHECK(cudaEventRecord(side->fork, stream));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->fork, 0));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->fork, 0));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s3, side->fork, 0));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s4, side->fork, 0));
     GPTQ_CUDA_CHECK(cudaMemsetAsync(Minv, 0, dd, side->s2));
     GPTQ_CUDA_CHECK(cudaEventRecord(side->cleared, side->s2));
 
@@ -763,13 +774,36 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
     }
     GPTQ_LAUNCH_CHECK();
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->cleared, 0));
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->ready, stream));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->sp, side->ready, 0));
 
     // Blocked right-looking Cholesky, A = M M^T (lower), with look-ahead:
     // panel k+1 applies panel k's correction to its own block column (and to
-    // its row block of M^{-1}) on the fly; the corrections of everything
-    // below block k+1 -- the symmetric trailing update of A on one side
-    // stream, the update of M^{-1}'s lower rows on the other -- are waited for
-    // only by panel k+2.  The critical path is the chain of panel kernels.
+    // its row block of M^{-1}) on the fly.  The corrections below block k+1
+    // are split by distance.  Panels form batches of kBatch (256 columns);
+    // for panel q of batch b, with E_b = (kBatch (b + 2)) kNB:
+    //   narrow(q)  K = 64: columns [(q + 2) kNB, E_b) of A and the same row
+    //              blocks of M^{-1}, right after panel q; panel q + 2 waits
+    //              for it;
+    //   band(b)    K = 256, after the batch's last panel, on the narrow
+    //              streams: the batch's correction of columns (row blocks of
+    //              M^{-1}) [E_b, E_b + 256), which narrow(q') of the next
+    //              batch writes as well, so it goes first;
+    //   far(b)     K = 256: everything from E_b + 256 on, on streams of its
+    //              own, overlapping the next panels: first the head (the
+    //              256 columns band(b + 1) writes as well, so band(b + 1)
+    //              waits for it), then the tail, which band(b + 2) meets only
+    //              behind far(b + 1)'s head on the same stream.
+    // Every region thus receives its corrections in one fixed order (the
+    // factorisation is bitwise reproducible), and the bulk of the trailing
+    // work runs as K = 256 products: a quarter of the HBM traffic of
+    // rank-64 updates, which bound the factorisation at d = 11008.  The
+    // critical path is the chain of panel kernels (stream sp).  The far
+    // products run one CTA per tile at the lowest priority: they fill the
+    // SMs the chain leaves and give them back tile by tile.
+    constexpr int kBatch = 8;
+    constexpr int kBW = kBatch * kNB;
+    constexpr int kBatchMinDim = 7168;
     const int n_panels = (d + kNB - 1) / kNB;
     {
         static bool attr_panel[64] = {};
@@ -782,6 +816,13 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
             attr_panel[dev] = true;
         }
     }
+    // CTA caps of a pair of products (A, M^{-1}) sharing `sms` SMs in
+    // proportion to their flops
+    auto split = [](int sms, double f_a, double f_inv, int* c_a, int* c_inv) {
+        const double t = f_a + f_inv;
+        *c_a = std::max(8, static_cast<int>(sms * (t > 0 ? f_a / t : 0.5) + 0.5));
+        *c_inv = std::max(8, sms - *c_a);
+    };
     for (int p = 0; p < n_panels; ++p) {
         const int k0 = p * kNB;
         const int kb = std::min(kNB, d - k0);
@@ -790,45 +831,92 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
         // CTA 0 writes L_kk^{-1}; the others share the panel's work items, at
         // most kPanelMaxCtas of them so the side products keep enough SMs
         const int n_cta = std::min(1 + n_trsm + p, kPanelMaxCtas);
-        // SMs the side products may hold: the rest after this panel's CTAs,
-        // split between the two side streams in proportion to their flops
-        // (rest2^2 / 2 for the symmetric update, rest2 (k0 + kb) for M^{-1})
         const int free_sm = std::max(16, nsm - n_cta);
-        const double f_sym = 0.5 * std::max(rest - kNB, 0);
-        const double f_inv = static_cast<double>(k0 + kb);
-        const int ctas_sym = std::max(8, static_cast<int>(free_sm * f_sym / (f_sym + f_inv) + 0.5));
-        const int ctas_inv = std::max(8, free_sm - ctas_sym);
         if (p >= 2) {
-            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev[(p - 2) % SideStream::kRing], 0));
-            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->ev2[(p - 2) % SideStream::kRing], 0));
+            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->sp, side->ev[(p - 2) % SideStream::kRing], 0));
+            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->sp, side->ev2[(p - 2) % SideStream::kRing], 0));
         }
-        chol_panel_kernel<<<n_cta, 256, kPanelSmem, stream>>>(A, d, k0, kb, p > 0 ? k0 - kNB : -1,
-                                                              Minv, hdr);
+        chol_panel_kernel<<<n_cta, 256, kPanelSmem, side->sp>>>(A, d, k0, kb, p > 0 ? k0 - kNB : -1,
+                                                                Minv, hdr);
         GPTQ_LAUNCH_CHECK();
-        GPTQ_CUDA_CHECK(cudaEventRecord(side->done_panel, stream));
-        const int rest2 = rest - kNB;   // rows/columns below block k+1
-        if (rest2 > 0) {
-            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->done_panel, 0));
-            GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->done_panel, 0));
-            float* P = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0;
-            float* C = A + static_cast<int64_t>(k0 + kb + kNB) * d + k0 + kb + kNB;
-            rc = launch_sgemm(true, rest2, rest2, kb, -1.f, P, d, 0, P, d, 0, 1.f, C, d, 0, 1,
-                              kGemmLowerC, side->s, ctas_sym);
+        GPTQ_CUDA_CHECK(cudaEventRecord(side->done_panel, side->sp));
+        GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->done_panel, 0));
+        GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->done_panel, 0));
+        const int b = p / kBatch;
+        // below kBatchMinDim every correction is narrow: columns [r0, d)
+        const int64_t e_b = d >= kBatchMinDim ? static_cast<int64_t>(kBatch) * (b + 2) * kNB : d;
+        const bool batch_end = p % kBatch == kBatch - 1 && e_b < d;
+        const bool has_far = batch_end && e_b + kBW < d;
+        const int r0 = k0 + kb + kNB;   // first row/column below block k+1
+        const int c1 = static_cast<int>(std::min<int64_t>(e_b, d));
+        if (r0 < c1) {
+            const int m = d - r0, n = c1 - r0;
+            int ca = 0, ci = 0;
+            split(free_sm, 0.5 * n * n + double(m - n) * n, double(n) * (k0 + kb), &ca, &ci);
+            float* P = A + static_cast<int64_t>(r0) * d + k0;
+            rc = launch_sgemm(true, m, n, kb, -1.f, P, d, 0, P, d, 0, 1.f,
+                              A + static_cast<int64_t>(r0) * d + r0, d, 0, 1, kGemmLowerC, side->s, ca);
             if (rc) return rc;
-            // (M^{-1})[below k+1][0 : k0+kb] -= M[below k+1][k] (M^{-1})_k
-            rc = launch_sgemm(false, rest2, k0 + kb, kb, -1.f, P, d, 0,
-                              Minv + static_cast<int64_t>(k0) * d, d, 0, 1.f,
-                              Minv + static_cast<int64_t>(k0 + kb + kNB) * d, d, 0, 1, 0, side->s2,
-                              ctas_inv);
+            // (M^{-1})[r0 : c1][0 : k0+kb] -= M[r0 : c1][k] (M^{-1})_k
+            rc = launch_sgemm(false, n, k0 + kb, kb, -1.f, P, d, 0, Minv + static_cast<int64_t>(k0) * d, d,
+                              0, 1.f, Minv + static_cast<int64_t>(r0) * d, d, 0, 1, 0, side->s2, ci);
             if (rc) return rc;
+        }
+        if (batch_end) {
+            const int c0 = (p + 1) * kNB - kBW;   // first column of the batch
+            const int e = static_cast<int>(e_b);
+            const int m = d - e, n = std::min(kBW, d - e);
+            float* P = A + static_cast<int64_t>(e) * d + c0;
+            int ca = 0, ci = 0;
+            split(free_sm, 0.5 * n * n + double(m - n) * n, double(n) * (c0 + kBW), &ca, &ci);
+            if (b >= 1) {   // far(b - 1) wrote these columns / row blocks
+                GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s, side->far[(b - 1) % SideStream::kRing], 0));
+                GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s2, side->far2[(b - 1) % SideStream::kRing], 0));
+            }
+            rc = launch_sgemm(true, m, n, kBW, -1.f, P, d, 0, P, d, 0, 1.f,
+                              A + static_cast<int64_t>(e) * d + e, d, 0, 1, kGemmLowerC, side->s, ca);
+            if (rc) return rc;
+            rc = launch_sgemm(false, n, c0 + kBW, kBW, -1.f, P, d, 0, Minv + static_cast<int64_t>(c0) * d, d,
+                              0, 1.f, Minv + static_cast<int64_t>(e) * d, d, 0, 1, 0, side->s2, ci);
+            if (rc) return rc;
+            if (has_far) {
+                // head: the 256 columns band(b + 1) writes next, then the tail
+                const int f = e + kBW, mf = d - f, hb = std::min(kBW, mf);
+                GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s3, side->done_panel, 0));
+                GPTQ_CUDA_CHECK(cudaStreamWaitEvent(side->s4, side->done_panel, 0));
+                for (int part = 0; part < 2; ++part) {
+                    const int g0 = part == 0 ? f : f + hb;   // first row/column of the part
+                    const int mg = d - g0, ng = part == 0 ? hb : mg;
+                    if (mg <= 0) break;
+                    float* Pf = A + static_cast<int64_t>(g0) * d + c0;
+                    rc = launch_sgemm(true, mg, ng, kBW, -1.f, Pf, d, 0, Pf, d, 0, 1.f,
+                                      A + static_cast<int64_t>(g0) * d + g0, d, 0, 1, kGemmLowerC,
+                                      side->s3, -1);
+                    if (rc) return rc;
+                    rc = launch_sgemm(false, ng, c0 + kBW, kBW, -1.f, Pf, d, 0,
+                                      Minv + static_cast<int64_t>(c0) * d, d, 0, 1.f,
+                                      Minv + static_cast<int64_t>(g0) * d, d, 0, 1, 0, side->s4, -1);
+                    if (rc) return rc;
+                    if (part == 0) {
+                        GPTQ_CUDA_CHECK(cudaEventRecord(side->far[b % SideStream::kRing], side->s3));
+                        GPTQ_CUDA_CHECK(cudaEventRecord(side->far2[b % SideStream::kRing], side->s4));
+                    }
+                }
+            }
         }
         GPTQ_CUDA_CHECK(cudaEventRecord(side->ev[p % SideStream::kRing], side->s));
         GPTQ_CUDA_CHECK(cudaEventRecord(side->ev2[p % SideStream::kRing], side->s2));
     }
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->join_p, side->sp));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join_p, 0));
     GPTQ_CUDA_CHECK(cudaEventRecord(side->join, side->s));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join, 0));
     GPTQ_CUDA_CHECK(cudaEventRecord(side->join2, side->s2));
     GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join2, 0));
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->join3, side->s3));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join3, 0));
+    GPTQ_CUDA_CHECK(cudaEventRecord(side->join4, side->s4));
+    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(stream, side->join4, 0));
 
     reverse_upper_kernel<<<nsm * 8, 256, 0, stream>>>(Minv, d, U);
     GPTQ_LAUNCH_CHECK();

@@ -96,6 +96,24 @@ def test_prepare_matches_checker(d, act_order):
     assert np.abs(I - np.eye(d)).max() < 1e-3
 
 
+@pytest.mark.parametrize("act_order", [False, True])
+def test_prepare_batched_trailing_updates_match_checker(act_order):
+    """From d_in = 7168 on, the factorisation applies most trailing
+    corrections in batches of 512 columns (band and far products on streams
+    of their own).  d = 7232: 113 panels of 64, a ragged last batch; against
+    the float64 checker, and bitwise equal on a second run."""
+    d = 7232
+    xb = _rand_x(d + 5, 2 * d, d, outliers=d // 64)
+    Hg = _gpu_hessian(xb)
+    perm_g, Ug = _gpu_prepare(Hg, act_order)
+    perm_r, Ur, Hp, _ = oracle.prepare(Hg.astype(np.float64), 0.01, act_order)
+    np.testing.assert_array_equal(perm_g, perm_r)
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert P.rel_fro(Ug, Ur) <= P.U_RTOL, P.rel_fro(Ug, Ur)
+    perm_2, U2 = _gpu_prepare(Hg, act_order)
+    assert np.array_equal(perm_2, perm_g) and np.array_equal(U2, Ug)
+
+
 def test_prepare_rejects_singular_and_nonfinite():
     d = 64
     with pytest.raises(B.GptqError) as e:
