@@ -185,6 +185,29 @@ int gptq_prepare(const float *H, int64_t d_in, float damp, int act_order, int32_
                  float *Hinv_chol, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * gptq_prepare without the wait: the same work, enqueued on `stream` (the
+ * same cached graph), and the factorisation status (0, GPTQ_ERR_NOT_PD or
+ * GPTQ_ERR_NONFINITE, as gptq_prepare returns it) written to *status when
+ * the stream reaches the end of the call.  Returns as soon as the work is
+ * enqueued, so the host can enqueue the column loop while the factorisation
+ * runs.  The caller reads *status after synchronising the stream; U and perm
+ * are meaningful only when it is 0.
+ *   status   int32, device memory or pinned host memory, 4-byte aligned,
+ *            owned by the caller; must stay valid until the stream passes
+ *            the call.
+ * Returns GPTQ_ERR_INVALID_ARG / GPTQ_ERR_WORKSPACE for bad arguments (before
+ * any launch), else GPTQ_OK.  Concurrent calls are safe: the enqueue is
+ * serialised per device and each call replays its own cached graph (two
+ * calls with the same buffers replay the same graph, one after the other).
+ * With graphs switched off (GPTQ_GRAPHS=0) the call waits for the stream like
+ * gptq_prepare, since direct launches use the device's shared side streams;
+ * inside a stream capture it only enqueues.
+ */
+int gptq_prepare_async(const float *H, int64_t d_in, float damp, int act_order, int32_t *perm,
+                       float *Hinv_chol, void *workspace, size_t ws_bytes, int *status,
+                       void *stream);
+
+/*
  * GPTQ column loop ("Jak działa"): for columns c in processing order, with a
  * new per-row (scale, zero) at each group start taken from the row's current
  * values of the group's columns (range including 0; an all-zero range is

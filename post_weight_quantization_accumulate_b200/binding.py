@@ -37,6 +37,7 @@ SIGNATURES = [
     ("gptq_hessian_f32_workspace_bytes", _SZ, [_I64, _I64]),
     ("gptq_hessian_accumulate_f32", _I, [_P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     ("gptq_prepare", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P]),
+    ("gptq_prepare_async", _I, [_P, _I64, _F, _I, _P, _P, _P, _SZ, _P, _P]),
     ("gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     ("gptq_quantize_q4k", _I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                _SZ, _P]),
@@ -192,6 +193,24 @@ def gptq_prepare(H: torch.Tensor, damp: float, act_order: bool, perm: torch.Tens
     _check("gptq_prepare",
            lib().gptq_prepare(_ptr(H), d, float(damp), int(bool(act_order)), _ptr(perm),
                               _ptr(Hinv_chol), _ptr(ws), ws.numel(), _stream(H, stream)))
+
+
+def gptq_prepare_async(H: torch.Tensor, damp: float, act_order: bool, perm: torch.Tensor,
+                       Hinv_chol: torch.Tensor, ws: torch.Tensor, status: torch.Tensor, stream=None):
+    """gptq_prepare without waiting: the factorisation status lands in
+    status (int32, one element, on the device or in pinned host memory) when
+    the stream reaches it; read it after synchronising."""
+    _need(H, torch.float32, "H")
+    _need(perm, torch.int32, "perm")
+    _need(Hinv_chol, torch.float32, "Hinv_chol")
+    _need(status, torch.int32, "status")
+    if status.numel() < 1 or not (status.is_cuda or status.is_pinned()):
+        raise ValueError("status must be an int32 device tensor or pinned host tensor")
+    d = H.shape[0]
+    _check("gptq_prepare_async",
+           lib().gptq_prepare_async(_ptr(H), d, float(damp), int(bool(act_order)), _ptr(perm),
+                                    _ptr(Hinv_chol), _ptr(ws), ws.numel(), _ptr(status),
+                                    _stream(H, stream)))
 
 
 def gptq_quantize(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Tensor | None, bits: int,

@@ -16,7 +16,7 @@ size_t prepare_workspace_bytes(int64_t d);
 size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in);
 size_t quantize_workspace_min_bytes(int64_t d_out, int64_t d_in);
 int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* perm, float* U,
-                void* ws, cudaStream_t s, int* host_status, bool graphed);
+                void* ws, cudaStream_t s, int* host_status, bool graphed, int* async_status = nullptr);
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in,
                  int bits, int gs, int block, uint8_t* codes, float* scales, float* zeros,
                  uint8_t* packed, int32_t* g_idx, float* err_sq, void* ws, size_t ws_bytes,
@@ -350,6 +350,20 @@ int gptq_prepare(const float* H, int64_t d_in, float damp, int act_order, int32_
                      static_cast<cudaStream_t>(stream), &st, true);
     if (rc) return rc;
     return st;
+}
+
+int gptq_prepare_async(const float* H, int64_t d_in, float damp, int act_order, int32_t* perm,
+                       float* Hinv_chol, void* workspace, size_t ws_bytes, int* status, void* stream)
+{
+    if (!H || !perm || !Hinv_chol || !status || d_in <= 0 || d_in > kMaxDim || !(damp >= 0.f) ||
+        !(damp < 1e30f) || !aligned(status, 4))
+        return GPTQ_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < prepare_workspace_bytes(d_in))
+        return GPTQ_ERR_WORKSPACE;
+    int rc = check_device();
+    if (rc) return rc;
+    return run_prepare(H, d_in, damp, act_order ? 1 : 0, perm, Hinv_chol, workspace,
+                       static_cast<cudaStream_t>(stream), nullptr, true, status);
 }
 
 int gptq_quantize(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,

@@ -25,6 +25,8 @@ uint64_t launch_count();            // launches recorded by the calling thread
 // graph captured from it for the same `key` (every argument that shapes the
 // launch sequence).  With want_status, *status_out is a pinned word that holds
 // the run's status after `stream` is synchronised.
+// false when GPTQ_GRAPHS=0 asks for direct launches instead of cached graphs
+bool graphs_enabled();
 int run_graphed(const std::vector<uint64_t>& key, bool want_status,
                 const std::function<int(cudaStream_t, int*)>& enqueue, cudaStream_t stream,
                 int** status_out);

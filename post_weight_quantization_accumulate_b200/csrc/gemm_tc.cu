@@ -71,6 +71,7 @@ constexpr size_t gemm_smem_bytes()
 }
 static_assert(gemm_smem_bytes<128, false>() <= 227 * 1024, "one CTA per SM");
 static_assert(gemm_smem_bytes<256, true>() <= 227 * 1024, "one CTA per SM");
+static_assert(gemm_smem_bytes<128, true>() <= 227 * 1024, "one CTA per SM");
 
 enum CMode : int { kCPlain = 0, kCStore = 1, kCReduce = 2 };
 
@@ -551,8 +552,14 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
 {
     if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
     const bool prelo = A_lo && B_lo;
-    const int tn = prelo ? 256 : 128;
-    int rc = prelo ? set_smem_attr<256, true>() : set_smem_attr<128, false>();
+    // 128 x 256 tiles with supplied low parts, unless they would not fill one
+    // wave of the SMs: then 128 x 128 tiles, twice as many CTAs with half the
+    // MMA work each
+    int tn = prelo ? 256 : 128;
+    if (prelo && static_cast<int64_t>((M + TBM - 1) / TBM) * ((N + 255) / 256) * batch < sm_count())
+        tn = 128;
+    int rc = prelo ? (tn == 256 ? set_smem_attr<256, true>() : set_smem_attr<128, true>())
+                   : set_smem_attr<128, false>();
     if (rc) return rc;
     const int Kp = K > 0 ? K : 1;
     CUtensorMap mA, mB, mAlo, mBlo, mC;
@@ -602,9 +609,12 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;
     if (max_ctas < 0) cap = units;   // one CTA per tile
     const int grid = static_cast<int>(units < cap ? units : cap);
-    if (prelo)
+    if (prelo && tn == 256)
         GPTQ_CUDA_CHECK(launch_k(gemm_tc_kernel<256, true>, dim3(grid), dim3(TTHREADS),
                                  gemm_smem_bytes<256, true>(), stream, pdl, mA, mB, mAlo, mBlo, mC, g));
+    else if (prelo)
+        GPTQ_CUDA_CHECK(launch_k(gemm_tc_kernel<128, true>, dim3(grid), dim3(TTHREADS),
+                                 gemm_smem_bytes<128, true>(), stream, pdl, mA, mB, mAlo, mBlo, mC, g));
     else
         GPTQ_CUDA_CHECK(launch_k(gemm_tc_kernel<128, false>, dim3(grid), dim3(TTHREADS),
                                  gemm_smem_bytes<128, false>(), stream, pdl, mA, mB, mAlo, mBlo, mC, g));

@@ -29,6 +29,14 @@ std::mutex g_mu;
 std::list<Entry> g_cache;   // most recently used first
 cudaStream_t g_capture[64] = {};
 
+void drop(Entry& e)
+{
+    cudaGraphExecDestroy(e.exec);
+    if (e.status_host) cudaFreeHost(e.status_host);
+}
+
+}  // namespace
+
 bool graphs_enabled()
 {
     static const bool on = [] {
@@ -37,14 +45,6 @@ bool graphs_enabled()
     }();
     return on;
 }
-
-void drop(Entry& e)
-{
-    cudaGraphExecDestroy(e.exec);
-    if (e.status_host) cudaFreeHost(e.status_host);
-}
-
-}  // namespace
 
 // Runs enqueue(stream, status_host) either directly on `stream` or through a
 // cached graph.  status_host (when want_status) receives the device status

@@ -938,8 +938,12 @@ static std::mutex& prepare_mutex()
     return mu[dev];
 }
 
+// host_status != nullptr: synchronises the stream and stores the status there.
+// Otherwise the status word is copied to async_status in stream order and the
+// call returns without waiting.
 int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* perm, float* U,
-                void* workspace, cudaStream_t stream, int* host_status, bool graphed)
+                void* workspace, cudaStream_t stream, int* host_status, bool graphed,
+                int* async_status)
 {
     std::lock_guard<std::mutex> one_in_flight(prepare_mutex());
     uint32_t damp_bits = 0;
@@ -965,6 +969,19 @@ int run_prepare(const float* H, int64_t d, float damp, int act_order, int32_t* p
         rc = enq(stream, st);
     }
     if (rc) return rc;
+    if (!host_status) {
+        const PrepHeader* hdr = reinterpret_cast<const PrepHeader*>(workspace);
+        GPTQ_CUDA_CHECK(cudaMemcpyAsync(async_status, &hdr->status, sizeof(int), cudaMemcpyDefault, stream));
+        // launched directly (no graph) on the shared side streams: they must be
+        // idle before the next call of the device may use them
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        GPTQ_CUDA_CHECK(cudaStreamIsCapturing(stream, &cs));
+        int dev = 0;
+        GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
+        const bool direct = !graphed || !graphs_enabled() || dev < 0 || dev >= 64;
+        if (direct && cs == cudaStreamCaptureStatusNone) GPTQ_CUDA_CHECK(cudaStreamSynchronize(stream));
+        return GPTQ_OK;
+    }
     GPTQ_CUDA_CHECK(cudaStreamSynchronize(stream));
     *host_status = *st;
     return GPTQ_OK;

@@ -139,9 +139,10 @@ def calibrate(X_attn: torch.Tensor, W: dict, shape: DecoderShape, bits: int = 4,
         ev[0].record()
         q.reset()
         q.add_batch(X)
-        q.prepare()
+        q.prepare(wait=False)
         for name in names:
             res.layers[name] = _copy(q.quantize(W[name]))
+        q.check()
         ev[1].record()
         if keep_state:
             res.H[group], res.U[group], res.perm[group] = q.H.clone(), q.U.clone(), q.perm.clone()

@@ -52,6 +52,8 @@ class LayerQuantizer:
         self.ws = B.workspace(d_out, d_in, block_size, device=dev)
         self.staging = None
         self.n_tokens = 0
+        self._status = None      # pinned status word of a prepare(wait=False)
+        self._pending = False
 
     # -- step 1: Hessian ------------------------------------------------------
     def reset(self):
@@ -83,8 +85,33 @@ class LayerQuantizer:
         self.n_tokens += X.shape[0]
 
     # -- steps 2-5 ----------------------------------------------------------------
-    def prepare(self):
-        B.gptq_prepare(self.H, self.damp, self.act_order, self.perm, self.U, self.ws)
+    def prepare(self, wait: bool = True):
+        """Damping, activation order and U.  wait=False enqueues the
+        factorisation without synchronising the stream (the host can enqueue
+        quantize meanwhile); its status is checked by check(), which the next
+        prepare also calls."""
+        self.check()
+        if wait:
+            B.gptq_prepare(self.H, self.damp, self.act_order, self.perm, self.U, self.ws)
+            return
+        if self._status is None:
+            self._status = torch.zeros(1, dtype=torch.int32).pin_memory()
+            self._done = torch.cuda.Event()
+        B.gptq_prepare_async(self.H, self.damp, self.act_order, self.perm, self.U, self.ws,
+                             self._status)
+        self._done.record(torch.cuda.current_stream(self.device))
+        self._pending = True
+
+    def check(self):
+        """Raises GptqError if a prepare(wait=False) failed.  Waits only for
+        that factorisation (an event after it), not for later work."""
+        if not self._pending:
+            return
+        self._done.synchronize()
+        self._pending = False
+        st = int(self._status[0])
+        if st != 0:
+            raise B.GptqError("gptq_prepare_async", st)
 
     def quantize(self, W: torch.Tensor) -> QuantizedLayer:
         """W [d_out, d_in] bf16 or float32 on the device (not modified)."""
@@ -140,5 +167,10 @@ class LayerQuantizer:
                                      err_sq=self.err_sq)
 
     def run(self, W: torch.Tensor) -> QuantizedLayer:
-        self.prepare()
-        return self.quantize(W)
+        """prepare + quantize.  The column loop is enqueued before the host
+        waits for the factorisation's status, so the GPU goes from one to the
+        other without a host round trip in between."""
+        self.prepare(wait=False)
+        out = self.quantize(W)
+        self.check()
+        return out

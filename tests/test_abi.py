@@ -75,6 +75,12 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.gptq_prepare(fake, 64, ctypes.c_float(0.01), 0, None, fake, fake, 1 << 30, None) == 1
     assert lib.gptq_prepare(fake, 64, ctypes.c_float(0.01), 0, fake, fake, None, 0, None) == 6
     assert lib.gptq_prepare(fake, 64, ctypes.c_float(0.01), 0, fake, fake, fake, 10, None) == 6
+    # prepare_async: the same refusals, plus a missing or misaligned status word
+    pa = lib.gptq_prepare_async
+    assert pa(fake, 64, ctypes.c_float(-1.0), 0, fake, fake, fake, 1 << 30, fake, None) == 1
+    assert pa(fake, 64, ctypes.c_float(0.01), 0, fake, fake, fake, 1 << 30, None, None) == 1
+    assert pa(fake, 64, ctypes.c_float(0.01), 0, fake, fake, fake, 1 << 30, P((1 << 20) + 2), None) == 1
+    assert pa(fake, 64, ctypes.c_float(0.01), 0, fake, fake, None, 0, fake, None) == 6
 
     def q(bits=4, gs=128, block=128, d_in=256, packed=None, ws=fake, ws_bytes=1 << 40):
         return lib.gptq_quantize(fake, fake, None, 64, d_in, bits, gs, block, None, fake, fake,

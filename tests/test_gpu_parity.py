@@ -132,6 +132,39 @@ def test_prepare_rejects_singular_and_nonfinite():
     assert e.value.status == 2
 
 
+def test_prepare_async_matches_prepare_and_reports_status():
+    """gptq_prepare_async: the same U and perm bits as gptq_prepare, the
+    status in a device word or a pinned host word once the stream passes the
+    call, and LayerQuantizer.run raising on a failed factorisation."""
+    d = 392
+    xb = _rand_x(17, 4 * d, d, outliers=3)
+    Hg = _gpu_hessian(xb)
+    perm_s, U_s = _gpu_prepare(Hg, True)
+    H = torch.from_numpy(Hg).to(DEV)
+    U = torch.empty(d, d, device=DEV)
+    perm = torch.empty(d, dtype=torch.int32, device=DEV)
+    ws = B.workspace(1, d, 128)
+    st = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    B.gptq_prepare_async(H, 0.01, True, perm, U, ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(U.cpu().numpy(), U_s) and np.array_equal(perm.cpu().numpy(), perm_s)
+    sp = torch.full((1,), -7, dtype=torch.int32).pin_memory()
+    B.gptq_prepare_async(torch.zeros(d, d, device=DEV), 0.01, False, perm, U, ws, sp)
+    torch.cuda.synchronize()
+    assert int(sp[0]) == 2                      # GPTQ_ERR_NOT_PD
+    Hn = torch.eye(d, device=DEV)
+    Hn[3, 3] = float("nan")
+    B.gptq_prepare_async(Hn, 0.01, False, perm, U, ws, sp)
+    torch.cuda.synchronize()
+    assert int(sp[0]) == 3                      # GPTQ_ERR_NONFINITE
+    q = LayerQuantizer(64, 384, 4, 128, 128, 0.01, False)
+    q.reset()                                   # H = 0: not positive definite
+    with pytest.raises(B.GptqError) as e:
+        q.run(torch.zeros(64, 384, device=DEV))
+    assert e.value.status == 2
+
+
 # ------------------------------------------------------------------ column loop
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])
