@@ -511,8 +511,15 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
                     kq[h][cl % 2] = q;
                     if (kGroupsInStep) kw[h][cl % 2] = what;
                 }
+                // the row's 16 columns, two per instruction (each lane of the
+                // pair is fmaf(-e, u, w): the same bits as the scalar form)
+                const float2 ne = make_float2(-e, -e);
 #pragma unroll
-                for (int k = 0; k < QCPT; ++k) w[h][k] = fmaf(-e, u[k], w[h][k]);
+                for (int k = 0; k < QCPT; k += 2) {
+                    const float2 r2 = __ffma2_rn(ne, make_float2(u[k], u[k + 1]), make_float2(w[h][k], w[h][k + 1]));
+                    w[h][k] = r2.x;
+                    w[h][k + 1] = r2.y;
+                }
             }
         }
         // this lane's two columns of the sub-block: e, w^ and the codes
