@@ -175,9 +175,11 @@ def lazy_flops(spec) -> float:
 
 
 def lazy_batch_line(spec, stage):
-    """All lazy-batch products of the column loop (events between launches,
-    gptq_quantize_timed) against the measured tf32 peak: `frac` against the
-    burst figure (the products run as short bursts inside the column loop),
+    """All lazy-batch products of the column loop against the measured tf32
+    peak: `ms` is the sum of the products' own spans in the production launch
+    sequence (gptq_quantize_timed: device clock from each product's first CTA
+    past its dependency wait to its last CTA's end); `frac` against the burst
+    figure (the products run as short bursts inside the column loop),
     `frac_sustained` against the power-capped one."""
     if not stage or not stage.get("lazy_batch_ms"):
         return None
@@ -188,8 +190,8 @@ def lazy_batch_line(spec, stage):
             "tf32_rate_tflops": 3 * rate, "peak": pk["burst"], "peak_sustained": pk["sustained"],
             "unit": "TFLOP/s", "frac": (3 * rate / pk["burst"]) if pk["burst"] else None,
             "frac_sustained": (3 * rate / pk["sustained"]) if pk["sustained"] else None,
-            "note": "3xTF32: three tf32 MMAs per fp32-accurate product; peaks = measured cuBLAS tf32 "
-                    "(profiles/tf32_peak_cublas.md)"}
+            "note": "3xTF32: three tf32 MMAs per fp32-accurate product; ms = summed in-schedule "
+                    "kernel spans (globaltimer); peaks = measured cuBLAS tf32 (profiles/tf32_peak_cublas.md)"}
 
 
 def layer_roofline(spec, ms, reg, peaks):
@@ -559,7 +561,7 @@ def _timed_layer(q, X, Wd, stream, steps, warmup, barrier, clock_gpu):
 
 def _stages(q, X, Wd, stream):
     """One step broken down by stage (after the timed region), and the column
-    loop split into its kernel classes (events between launches)."""
+    loop split into its kernel classes (in-schedule kernel spans)."""
     import torch
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     evs[0].record(stream)

@@ -319,11 +319,15 @@ int gptq_quantize_static_scratch(float *W, const float *Hinv_chol, const int32_t
                                  void *stream);
 
 /* Diagnostic: gptq_quantize (same arguments, rules and results) enqueued
- * directly on `stream` with a CUDA event after every launch; synchronises
- * the stream and returns the summed device time of the column-loop kernels
- * (*loop_ms), of the lazy-batch products (*update_ms) and of everything else
- * (*other_ms: layout, gathers, unpermute/packing).  For measurement only:
- * the events add small gaps between launches. */
+ * directly on `stream` in its production launch sequence (programmatic
+ * dependent launches included); synchronises the stream.  The column-loop
+ * kernels and the tensor-core lazy-batch products record their own spans
+ * (device clock, ns): each launch from its first CTA passing its wait for the
+ * previous kernel to its last CTA's end.  Returns the summed spans of the
+ * column-loop kernels (*loop_ms) and of the lazy-batch products (*update_ms),
+ * and the rest of the call's device time (*other_ms: layout, gathers,
+ * unpermute/packing and launch gaps).  One timed call runs at a time in a
+ * process (the spans live in one static device array). */
 int gptq_quantize_timed(float* W, const float* Hinv_chol, const int32_t* perm, int64_t d_out,
                         int64_t d_in, int bits, int group_size, int block_size, uint8_t* codes,
                         float* scales, float* zeros, uint8_t* packed_int4, int32_t* g_idx,

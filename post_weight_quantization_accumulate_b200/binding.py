@@ -234,7 +234,9 @@ def gptq_quantize_timed(W: torch.Tensor, Hinv_chol: torch.Tensor, perm: torch.Te
                         packed_int4: torch.Tensor | None = None, g_idx: torch.Tensor | None = None,
                         err_sq: torch.Tensor | None = None, stream=None):
     """gptq_quantize with per-class device times: returns (column-loop ms,
-    lazy-batch product ms, other ms) of this call (synchronises the stream)."""
+    lazy-batch product ms, other ms) of this call (synchronises the stream).
+    The first two are the kernels' own spans in the production launch
+    sequence; other is the rest of the call's device time."""
     _need(W, torch.float32, "W")
     d_out, d_in = W.shape
     out = [ctypes.c_float(0.0) for _ in range(3)]

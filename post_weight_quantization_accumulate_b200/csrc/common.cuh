@@ -188,6 +188,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
 // once for a kernel launched without the attribute).  pdl_trigger: this CTA
 // lets the next kernel start; the next kernel's CTAs may occupy free SMs and
 // run their prologue while this grid still runs.
+// Device-wide nanosecond clock (the same on every SM), for the spans the
+// timing entry points record.
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

@@ -29,11 +29,15 @@ enum GemmFlags : int {
 // tensor-core path skips its conversion pass and uses 128 x 256 tiles.
 // pdl: launch the tensor-core product as a programmatic dependent launch (its
 // prologue overlaps the previous kernel on the stream; see launch_k).
+// stamp (optional, device, two words preset to ~0 and 0): the tensor-core
+// product records its span there, atomicMin of the time its first CTA passes
+// the dependency wait and atomicMax of the time its last CTA ends
+// (globaltimer, ns).  The SIMT path records nothing.
 int launch_sgemm(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                  int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                  int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream,
                  int max_ctas = 0, const float* A_lo = nullptr, const float* B_lo = nullptr,
-                 bool pdl = false);
+                 bool pdl = false, unsigned long long* stamp = nullptr);
 
 int launch_sgemm_simt(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                       int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
@@ -42,7 +46,7 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
                    int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                    int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream,
                    int max_ctas = 0, const float* A_lo = nullptr, const float* B_lo = nullptr,
-                   bool pdl = false);
+                   bool pdl = false, unsigned long long* stamp = nullptr);
 bool gemm_tc_supported(const float* A, int64_t lda, int64_t sA, const float* B, int64_t ldb,
                        int64_t sB, int batch);
 

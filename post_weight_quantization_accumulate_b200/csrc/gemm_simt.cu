@@ -119,14 +119,14 @@ __global__ void __launch_bounds__(256)
 int launch_sgemm(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                  int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                  int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream, int max_ctas,
-                 const float* A_lo, const float* B_lo, bool pdl)
+                 const float* A_lo, const float* B_lo, bool pdl, unsigned long long* stamp)
 {
     if (gemm_tc_supported(A, lda, sA, B, ldb, sB, batch)) {
         // the low parts are used only when they obey the same TMA rules
         const bool lo_ok = A_lo && B_lo && gemm_tc_supported(A_lo, lda, sA, B_lo, ldb, sB, batch);
         return launch_gemm_tc(trans_b, M, N, K, alpha, A, lda, sA, B, ldb, sB, beta, C, ldc, sC,
                               batch, flags, stream, max_ctas, lo_ok ? A_lo : nullptr,
-                              lo_ok ? B_lo : nullptr, pdl);
+                              lo_ok ? B_lo : nullptr, pdl, stamp);
     }
     // the SIMT kernel is launched plainly (it waits for the previous kernel)
     return launch_sgemm_simt(trans_b, M, N, K, alpha, A, lda, sA, B, ldb, sB, beta, C, ldc, sC,

@@ -82,6 +82,7 @@ struct GemmArgs {
     int64_t ldc, sC;
     int n_mt, n_nt;
     int* status;
+    unsigned long long* stamp;   // span of this launch (see launch_sgemm) or null
 };
 
 // Low part of x below its tf32 truncation (exact in float32).
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
     // after this wait.  The next kernel may then start its own set-up.
     pdl_wait();
     pdl_trigger();
+    if (g.stamp && threadIdx.x == 0) atomicMin(g.stamp, globaltimer_ns());
     const uint32_t tbase = S.tmem_base;
     volatile int* abort = &S.abort;
     int* status = g.status;
@@ -473,6 +475,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (g.stamp && threadIdx.x == 0) atomicMax(g.stamp + 1, globaltimer_ns());
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, Cfg::TMEM_COLS);
@@ -548,7 +551,7 @@ static int set_smem_attr()
 int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* A, int64_t lda,
                    int64_t sA, const float* B, int64_t ldb, int64_t sB, float beta, float* C,
                    int64_t ldc, int64_t sC, int batch, int flags, cudaStream_t stream, int max_ctas,
-                   const float* A_lo, const float* B_lo, bool pdl)
+                   const float* A_lo, const float* B_lo, bool pdl, unsigned long long* stamp)
 {
     if (M <= 0 || N <= 0 || batch <= 0) return GPTQ_OK;
     const bool prelo = A_lo && B_lo;
@@ -604,6 +607,7 @@ int launch_gemm_tc(bool trans_b, int M, int N, int K, float alpha, const float* 
     g.n_mt = (M + TBM - 1) / TBM;
     g.n_nt = (N + tn - 1) / tn;
     g.status = device_status_ptr();
+    g.stamp = stamp;
     const int64_t units = static_cast<int64_t>(g.n_mt) * g.n_nt * batch;
     int64_t cap = sm_count();
     if (max_ctas > 0 && max_ctas < cap) cap = max_ctas;

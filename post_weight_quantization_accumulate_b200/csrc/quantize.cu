@@ -23,6 +23,8 @@
 #include "common.cuh"
 #include "gemm.cuh"
 
+#include <algorithm>
+#include <mutex>
 #include <vector>
 
 namespace gptq {
@@ -75,6 +77,10 @@ struct QArgs {
     uint8_t* m6;
     float* dsup;
     float* dmin;
+    // span of this launch (two words preset to ~0 and 0; null when not timed):
+    // atomicMin of the time the first CTA passes the dependency wait,
+    // atomicMax of the time the last CTA ends (globaltimer, ns)
+    unsigned long long* stamp;
 };
 
 // Sub-block layout of U's diagonal blocks: chunk (b, S) covers rows
@@ -284,6 +290,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
     // only after it completes.  The next product may start its set-up now.
     pdl_wait();
     pdl_trigger();
+    if (a.stamp && tid == 0) atomicMin(a.stamp, globaltimer_ns());
 
     const int pair = tid / QTPR, part = tid % QTPR;
     const int lane = tid & 31;
@@ -550,6 +557,10 @@ __global__ void __launch_bounds__(QTHREADS, 1) gptq_block_kernel(QArgs a)
 #pragma unroll
     for (int h = 0; h < 2; ++h)
         if (valid[h] && a.err_sq && part == 0) a.err_sq[r[h]] += errsum[h];
+    if (a.stamp) {
+        __syncthreads();
+        if (tid == 0) atomicMax(a.stamp + 1, globaltimer_ns());
+    }
 }
 
 // One (scale, zero) per row from the whole original row (group_size = -1).
@@ -840,24 +851,30 @@ size_t quantize_workspace_bytes(int64_t d_out, int64_t d_in)
            up256(static_cast<size_t>(d_in) * static_cast<size_t>(d_in) * sizeof(float));
 }
 
-// Optional CUDA-event marks between the launches of one enqueue (the
-// diagnostic entry point): an event after every launch, tagged with the class
-// of the launch it ends (0 = other, 1 = column loop, 2 = lazy-batch product).
-struct QuantizeMarks {
-    std::vector<cudaEvent_t> ev;
-    std::vector<int> cls;
-    int mark(cudaStream_t s, int c)
-    {
-        cudaEvent_t e = nullptr;
-        GPTQ_CUDA_CHECK(cudaEventCreate(&e));
-        ev.push_back(e);
-        cls.push_back(c);
-        GPTQ_CUDA_CHECK(cudaEventRecord(e, s));
-        return GPTQ_OK;
+// Timing of one enqueue (the diagnostic entry point): the column-loop
+// kernels and the tensor-core lazy-batch products record their spans in a
+// static device array, one pair of words per launch, tagged on the host with
+// the launch's class (1 = column loop, 2 = lazy-batch product).  The launch
+// sequence is the production one (programmatic dependent launches included).
+constexpr int kMaxStamped = 8192;
+__device__ unsigned long long g_stamps[2 * kMaxStamped];
+
+__global__ void stamps_init_kernel(unsigned long long* st, int n)
+{
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        st[2 * i] = ~0ull;
+        st[2 * i + 1] = 0ull;
     }
-    ~QuantizeMarks()
+}
+
+struct QuantizeMarks {
+    unsigned long long* stamps = nullptr;   // g_stamps
+    std::vector<int> cls;
+    unsigned long long* slot(int c)
     {
-        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+        if (cls.size() >= static_cast<size_t>(kMaxStamped)) return nullptr;
+        cls.push_back(c);
+        return stamps + 2 * (cls.size() - 1);
     }
 };
 
@@ -867,12 +884,11 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
                             float* err_sq, void* workspace, bool with_low_parts, cudaStream_t stream,
                             QuantizeMarks* marks = nullptr, const Q4KOut* q4k = nullptr)
 {
-    auto mark = [&](int c) { return marks ? marks->mark(stream, c) : GPTQ_OK; };
-    if (int rc = mark(0)) return rc;
+    auto slot = [&](int c) { return marks ? marks->slot(c) : nullptr; };
     // The column-loop kernels and the lazy-batch products alternate on the
     // stream as programmatic dependent launches, each one's set-up overlapping
-    // the previous one's tail -- except when events are recorded between them.
-    const bool pdl = marks == nullptr;
+    // the previous one's tail.
+    const bool pdl = true;
     const int d_out = static_cast<int>(d_out64), d_in = static_cast<int>(d_in64);
     const size_t n = static_cast<size_t>(d_out) * d_in;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -972,22 +988,19 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
             QArgs a{work, Ul, d_out, d_in, j0, bw, block, bits, gs, n_groups, scales, zeros,
                     codes_p, E, E_lo, j0 - J0, err_sq, status,
                     q4k ? q4k->sc6 : nullptr, q4k ? q4k->m6 : nullptr,
-                    q4k ? q4k->dsup : nullptr, q4k ? q4k->dmin : nullptr};
-            if (int rc = mark(0)) return rc;
+                    q4k ? q4k->dsup : nullptr, q4k ? q4k->dmin : nullptr, slot(1)};
             auto kern = q4k ? gptq_block_kernel<false, true>
                             : (groups_in_step ? gptq_block_kernel<true, false> : gptq_block_kernel<false, false>);
             GPTQ_CUDA_CHECK(launch_k(kern, dim3(grid), dim3(QTHREADS), block_smem, stream, pdl, a));
             GPTQ_LAUNCH_CHECK();
-            if (int rc = mark(1)) return rc;
             const int rest_in = J1 - j0 - bw;
             if (rest_in > 0) {
                 const int64_t uo = static_cast<int64_t>(j0) * d_in + j0 + bw;
                 int rc = launch_sgemm(false, d_out, rest_in, bw, -1.f, E + (j0 - J0), kOuterMax, 0,
                                       U + uo, d_in, 0, 1.f, work + j0 + bw, d_in, 0, 1, 0, stream, 0,
                                       E_lo ? E_lo + (j0 - J0) : nullptr, U_lo ? U_lo + uo : nullptr,
-                                      pdl);
+                                      pdl, slot(2));
                 if (rc) return rc;
-                if ((rc = mark(2))) return rc;
             }
         }
         const int rest = d_in - J1;
@@ -995,9 +1008,8 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
             const int64_t uo = static_cast<int64_t>(J0) * d_in + J1;
             int rc = launch_sgemm(false, d_out, rest, J1 - J0, -1.f, E, kOuterMax, 0, U + uo, d_in, 0,
                                   1.f, work + J1, d_in, 0, 1, 0, stream, 0, E_lo,
-                                  U_lo ? U_lo + uo : nullptr, pdl);
+                                  U_lo ? U_lo + uo : nullptr, pdl, slot(2));
             if (rc) return rc;
-            if ((rc = mark(2))) return rc;
         }
     }
     if (codes || packed || perm) {
@@ -1018,7 +1030,7 @@ static int enqueue_quantize(float* W, const float* U, const int32_t* perm, int64
         g_idx_kernel<<<(d_in + 255) / 256, 256, 0, stream>>>(perm, d_in, gs, g_idx);
         GPTQ_LAUNCH_CHECK();
     }
-    return mark(0);
+    return GPTQ_OK;
 }
 
 int run_quantize(float* W, const float* U, const int32_t* perm, int64_t d_out, int64_t d_in, int bits,
@@ -1049,18 +1061,39 @@ int run_quantize_timed(float* W, const float* U, const int32_t* perm, int64_t d_
                        uint8_t* packed, int32_t* g_idx, float* err_sq, void* workspace,
                        size_t ws_bytes, cudaStream_t stream, float* ms_by_class)
 {
+    static std::mutex mu;   // one timed call at a time: they share g_stamps
+    std::lock_guard<std::mutex> lk(mu);
     QuantizeMarks marks;
+    void* p = nullptr;
+    GPTQ_CUDA_CHECK(cudaGetSymbolAddress(&p, g_stamps));
+    marks.stamps = static_cast<unsigned long long*>(p);
+    stamps_init_kernel<<<(kMaxStamped + 255) / 256, 256, 0, stream>>>(marks.stamps, kMaxStamped);
+    GPTQ_LAUNCH_CHECK();
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    GPTQ_CUDA_CHECK(cudaEventCreate(&e0));
+    GPTQ_CUDA_CHECK(cudaEventCreate(&e1));
     const bool low = ws_bytes >= quantize_workspace_bytes(d_out, d_in);
-    int rc = enqueue_quantize(W, U, perm, d_out, d_in, bits, gs, block, codes, scales, zeros, packed,
+    int rc = GPTQ_OK;
+    if (cudaEventRecord(e0, stream) != cudaSuccess) rc = cuda_fail(cudaGetLastError());
+    if (!rc)
+        rc = enqueue_quantize(W, U, perm, d_out, d_in, bits, gs, block, codes, scales, zeros, packed,
                               g_idx, err_sq, workspace, low, stream, &marks);
+    if (!rc && cudaEventRecord(e1, stream) != cudaSuccess) rc = cuda_fail(cudaGetLastError());
+    if (!rc && cudaStreamSynchronize(stream) != cudaSuccess) rc = cuda_fail(cudaGetLastError());
+    float total = 0.f;
+    if (!rc && cudaEventElapsedTime(&total, e0, e1) != cudaSuccess) rc = cuda_fail(cudaGetLastError());
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
     if (rc) return rc;
-    GPTQ_CUDA_CHECK(cudaStreamSynchronize(stream));
-    for (int c = 0; c < 3; ++c) ms_by_class[c] = 0.f;
-    for (size_t i = 1; i < marks.ev.size(); ++i) {
-        float ms = 0.f;
-        GPTQ_CUDA_CHECK(cudaEventElapsedTime(&ms, marks.ev[i - 1], marks.ev[i]));
-        ms_by_class[marks.cls[i]] += ms;
-    }
+    std::vector<unsigned long long> h(2 * marks.cls.size());
+    if (!h.empty())
+        GPTQ_CUDA_CHECK(cudaMemcpyFromSymbol(h.data(), g_stamps, h.size() * sizeof(unsigned long long)));
+    double by[3] = {0.0, 0.0, 0.0};
+    for (size_t i = 0; i < marks.cls.size(); ++i)
+        if (h[2 * i] != ~0ull && h[2 * i + 1] > h[2 * i]) by[marks.cls[i]] += 1e-6 * (h[2 * i + 1] - h[2 * i]);
+    ms_by_class[1] = static_cast<float>(by[1]);
+    ms_by_class[2] = static_cast<float>(by[2]);
+    ms_by_class[0] = std::max(0.f, total - ms_by_class[1] - ms_by_class[2]);
     return GPTQ_OK;
 }
 
