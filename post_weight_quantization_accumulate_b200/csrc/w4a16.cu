@@ -38,6 +38,10 @@
 //   * K is split over a cluster of up to 8 CTAs; the partial sums meet in
 //     distributed shared memory and each CTA of the cluster adds a slice of
 //     the tile in a fixed rank order (deterministic) and writes Y.
+// Decode path (at most 4 activation rows, groups contiguous along K): the
+// weights streamed once with 16-byte loads straight into registers, four
+// weight rows per block sharing each read of the activations, (q - z) x in
+// bf16 pairs and mixed-precision FMAs (see the kernel below).
 // General path (g_idx given, or a group size or K the tiles do not fit): one
 // warp per weight row on the SIMT pipes, W^ = s (q - z) in fp32.
 #include "common.cuh"
