@@ -867,7 +867,7 @@ __global__ void stamps_init_kernel(unsigned long long* st, int n)
     }
 }
 
-struct QuantizeMarks {
+struct QuantizeMarks {   // the launches of one timed enqueue and their span slots
     unsigned long long* stamps = nullptr;   // g_stamps
     std::vector<int> cls;
     unsigned long long* slot(int c)

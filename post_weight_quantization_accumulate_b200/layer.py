@@ -155,8 +155,9 @@ class LayerQuantizer:
         return out
 
     def quantize_timed(self, W: torch.Tensor):
-        """As quantize, enqueued directly with CUDA events between launches;
-        returns (column-loop ms, lazy-batch product ms, other ms)."""
+        """As quantize, enqueued directly (the production launch sequence)
+        with the kernels recording their spans; returns (column-loop ms,
+        lazy-batch product ms, other ms)."""
         if W.dtype == torch.bfloat16:
             B.gptq_bf16_to_f32(self.W, W)
         else:
