@@ -823,12 +823,26 @@ def main():
         zeros_h = torch.empty_like(q.zeros, device="cpu").pin_memory()
         gidx_h = torch.empty_like(q.g_idx, device="cpu").pin_memory()
         Wd2 = torch.empty_like(Wd)
+        w_stream = torch.cuda.Stream(dev)
+        ev_w, ev_w_free = torch.cuda.Event(), torch.cuda.Event()
 
         def e2e_step():
+            # X's chunks go up on the library's copy stream as soon as the
+            # previous step's accumulations have freed the staging buffers, and
+            # W on a stream of its own once the previous step has consumed it:
+            # both uploads overlap the previous step's factorisation and
+            # column loop.  The factorisation's status is checked by the next
+            # prepare (and after the loop).
             q.reset()
             q.add_batch_host(X_host, chunk_tokens=16384)
-            Wd2.copy_(W_host, non_blocking=True)
-            res = q.run(Wd2)
+            w_stream.wait_event(ev_w_free)
+            with torch.cuda.stream(w_stream):
+                Wd2.copy_(W_host, non_blocking=True)
+                ev_w.record(w_stream)
+            stream.wait_event(ev_w)
+            q.prepare(wait=False)
+            res = q.quantize(Wd2)
+            ev_w_free.record(stream)
             packed_h.copy_(res.packed, non_blocking=True)
             scales_h.copy_(res.scales, non_blocking=True)
             zeros_h.copy_(res.zeros, non_blocking=True)
@@ -844,6 +858,7 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
+        q.check()
         e2e_ms = a.elapsed_time(b) / args.steps
         e2e_ms = ranks.max_over_ranks([e2e_ms], device=dev)[0]
         h2d = X_host.numel() * 2 + W_host.numel() * W_host.element_size()

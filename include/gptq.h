@@ -117,11 +117,18 @@ int gptq_hessian_accumulate(float *H, const uint16_t *X, int64_t n_tokens, int64
  * in chunks of `chunk_tokens` through two caller-owned device staging buffers
  * while earlier chunks are accumulated, so the copy overlaps the tensor-core
  * work.  X_host should be page-locked for the copies to be asynchronous.
+ * The copies run on a copy stream of the library and wait only for the
+ * accumulations of this function's earlier calls on the device (the last
+ * readers of staging buffers), not for all earlier work on `stream`: the
+ * uploads of one layer's activations overlap the previous layer's
+ * factorisation and column loop.  The accumulations into H stay in the order
+ * of `stream`.  (Inside a stream capture the copies wait for the capture's
+ * earlier work instead.)
  *
  *   X_host        host bf16 bit patterns [n_tokens, d_in].
  *   staging       device buffer of 2 * chunk_tokens * d_in uint16, 16-byte
- *                 aligned, not used by anything else until the stream reaches
- *                 the end of this call's work.
+ *                 aligned, used by nothing but this function while any of
+ *                 its calls may be in flight.
  *   chunk_tokens  > 0.
  * Returns after all copies and kernels are enqueued; the host buffer must stay
  * valid until `stream` has finished them.

@@ -313,9 +313,17 @@ int gptq_hessian_accumulate_host(float* H, const uint16_t* X_host, int64_t n_tok
         }
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the staging buffers may still be read by earlier work on `stream`
-    GPTQ_CUDA_CHECK(cudaEventRecord(sp.ev_start, s));
-    GPTQ_CUDA_CHECK(cudaStreamWaitEvent(sp.copy, sp.ev_start, 0));
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    GPTQ_CUDA_CHECK(cudaStreamIsCapturing(s, &cs));
+    if (cs != cudaStreamCaptureStatusNone) {
+        // captured: the copy stream joins the capture through `stream`
+        GPTQ_CUDA_CHECK(cudaEventRecord(sp.ev_start, s));
+        GPTQ_CUDA_CHECK(cudaStreamWaitEvent(sp.copy, sp.ev_start, 0));
+    } else {
+        // the staging buffers' last readers are the accumulations of earlier
+        // calls (an event never recorded is no wait)
+        for (int i = 0; i < 2; ++i) GPTQ_CUDA_CHECK(cudaStreamWaitEvent(sp.copy, sp.ev_done[i], 0));
+    }
     const size_t chunk_elems = static_cast<size_t>(chunk_tokens) * static_cast<size_t>(d_in);
     int64_t c = 0;
     for (int64_t t = 0; t < n_tokens; t += chunk_tokens, ++c) {

@@ -70,6 +70,35 @@ def test_hessian_host_streaming_matches_device():
     assert P.rel_fro(Hh, oracle.hessian(xb)) <= P.H_RTOL
 
 
+def test_hessian_host_streaming_back_to_back_calls():
+    """Calls that share the staging buffers, enqueued without a synchronise in
+    between (the second call's uploads wait only for the first call's
+    accumulations): each H equals the device-resident result bit for bit, and
+    a kernel queued on the stream between the calls does not hold them up."""
+    xa, xc = _rand_x(6, 3000, 256, 2), _rand_x(7, 4100, 256, 3)
+    staging = torch.empty(2 * 512 * 256, dtype=torch.bfloat16, device=DEV)
+    Ha = torch.zeros(256, 256, dtype=torch.float32, device=DEV)
+    Hc = torch.zeros(256, 256, dtype=torch.float32, device=DEV)
+    Xa = torch.from_numpy(xa.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Xc = torch.from_numpy(xc.view(np.int16)).view(torch.bfloat16).pin_memory()
+    # references: one call at a time, the same chunks
+    B.gptq_hessian_accumulate_host(Ha, Xa, staging, 512)
+    torch.cuda.synchronize()
+    B.gptq_hessian_accumulate_host(Hc, Xc, staging, 512)
+    torch.cuda.synchronize()
+    Ha_ref, Hc_ref = Ha.cpu().numpy(), Hc.cpu().numpy()
+    assert P.rel_fro(Ha_ref, _gpu_hessian(xa)) <= 1e-6 and P.rel_fro(Hc_ref, _gpu_hessian(xc)) <= 1e-6
+    for _ in range(2):
+        Ha.zero_()
+        Hc.zero_()
+        B.gptq_hessian_accumulate_host(Ha, Xa, staging, 512)
+        torch.cuda._sleep(1000000)            # ~1 ms of other work on the stream
+        B.gptq_hessian_accumulate_host(Hc, Xc, staging, 512)
+        torch.cuda.synchronize()
+        assert np.array_equal(Ha.cpu().numpy(), Ha_ref)
+        assert np.array_equal(Hc.cpu().numpy(), Hc_ref)
+
+
 def test_hessian_zero_tokens_is_noop():
     H = torch.ones(64, 64, dtype=torch.float32, device=DEV)
     X = torch.empty(0, 64, dtype=torch.bfloat16, device=DEV)
