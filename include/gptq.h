@@ -117,13 +117,13 @@ int gptq_hessian_accumulate(float *H, const uint16_t *X, int64_t n_tokens, int64
  * in chunks of `chunk_tokens` through two caller-owned device staging buffers
  * while earlier chunks are accumulated, so the copy overlaps the tensor-core
  * work.  X_host should be page-locked for the copies to be asynchronous.
- * The copies run on a copy stream of the library and wait only for the
- * accumulations of this function's earlier calls on the device (the last
- * readers of staging buffers), not for all earlier work on `stream`: the
- * uploads of one layer's activations overlap the previous layer's
- * factorisation and column loop.  The accumulations into H stay in the order
- * of `stream`.  (Inside a stream capture the copies wait for the capture's
- * earlier work instead.)
+ * The copies run on a copy stream of the library.  When `staging` is the
+ * buffer the previous call on the device used, they wait only for that
+ * call's accumulations (the buffer's last readers), not for all earlier work
+ * on `stream`: the uploads of one layer's activations overlap the previous
+ * layer's factorisation and column loop.  With another buffer, or inside a
+ * stream capture, they wait for the earlier work on `stream`.  The
+ * accumulations into H stay in the order of `stream`.
  *
  *   X_host        host bf16 bit patterns [n_tokens, d_in].
  *   staging       device buffer of 2 * chunk_tokens * d_in uint16, 16-byte

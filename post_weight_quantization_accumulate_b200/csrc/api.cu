@@ -57,6 +57,8 @@ struct StreamPair {
     cudaEvent_t ev_ready[2] = {nullptr, nullptr};
     cudaEvent_t ev_done[2] = {nullptr, nullptr};
     cudaEvent_t ev_start = nullptr;
+    const void* last_staging = nullptr;   // staging buffer of the previous call
+    size_t last_bytes = 0;
 };
 StreamPair g_streams[kMaxDevices];
 }  // namespace
@@ -315,15 +317,21 @@ int gptq_hessian_accumulate_host(float* H, const uint16_t* X_host, int64_t n_tok
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     GPTQ_CUDA_CHECK(cudaStreamIsCapturing(s, &cs));
-    if (cs != cudaStreamCaptureStatusNone) {
-        // captured: the copy stream joins the capture through `stream`
+    const size_t staging_bytes = 2 * static_cast<size_t>(chunk_tokens) * static_cast<size_t>(d_in) * 2;
+    const bool same_staging = sp.last_staging == staging && sp.last_bytes == staging_bytes;
+    if (cs != cudaStreamCaptureStatusNone || !same_staging) {
+        // captured (the copy stream joins the capture through `stream`), or a
+        // staging buffer this function has not used last (it may hold memory
+        // that earlier work on `stream` still reads): wait for that work
         GPTQ_CUDA_CHECK(cudaEventRecord(sp.ev_start, s));
         GPTQ_CUDA_CHECK(cudaStreamWaitEvent(sp.copy, sp.ev_start, 0));
     } else {
-        // the staging buffers' last readers are the accumulations of earlier
-        // calls (an event never recorded is no wait)
+        // the same buffers as the previous call: their last readers are that
+        // call's accumulations
         for (int i = 0; i < 2; ++i) GPTQ_CUDA_CHECK(cudaStreamWaitEvent(sp.copy, sp.ev_done[i], 0));
     }
+    sp.last_staging = staging;
+    sp.last_bytes = staging_bytes;
     const size_t chunk_elems = static_cast<size_t>(chunk_tokens) * static_cast<size_t>(d_in);
     int64_t c = 0;
     for (int64_t t = 0; t < n_tokens; t += chunk_tokens, ++c) {
