@@ -139,6 +139,28 @@ __global__ void gather_rev_direct_kernel(const float* __restrict__ H, int d,
     }
 }
 
+// Without a reordering (perm = identity) the gather is a reversed copy:
+// A[a][b] = H[d-1-a][d-1-b] (+ delta on the diagonal), four columns per
+// thread with 16-byte loads and stores (d % 4 == 0, H and A 16-byte aligned).
+__global__ void reverse_copy_kernel(const float* __restrict__ H, int d, const PrepHeader* hdr,
+                                    float* __restrict__ A)
+{
+    const float delta = hdr->delta;
+    const int q = d / 4;
+    const int64_t n = static_cast<int64_t>(d) * q;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int a = static_cast<int>(idx / q), b = 4 * static_cast<int>(idx % q);
+        const float4 h = *reinterpret_cast<const float4*>(H + static_cast<int64_t>(d - 1 - a) * d + (d - 4 - b));
+        float4 v = make_float4(h.w, h.z, h.y, h.x);   // columns b .. b+3 of A
+        if (a == b) v.x += delta;
+        if (a == b + 1) v.y += delta;
+        if (a == b + 2) v.z += delta;
+        if (a == b + 3) v.w += delta;
+        *reinterpret_cast<float4*>(A + static_cast<int64_t>(a) * d + b) = v;
+    }
+}
+
 // One panel step of the blocked Cholesky, fused:
 //   every CTA factors the kb x kb diagonal block at (k0, k0) (redundantly, so
 //   no other launch has to wait for it) and inverts the factor; CTA 0 writes
@@ -756,7 +778,11 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
     GPTQ_LAUNCH_CHECK();
     act_order_kernel<<<(d + 255) / 256, 256, 0, stream>>>(H, d, act_order, perm);
     GPTQ_LAUNCH_CHECK();
-    if (d <= kGatherSmemMax) {
+    if (!act_order && d % 4 == 0 && (reinterpret_cast<uintptr_t>(H) & 15) == 0) {
+        const int64_t n4 = static_cast<int64_t>(d) * (d / 4);
+        reverse_copy_kernel<<<static_cast<int>(std::min<int64_t>((n4 + 255) / 256, nsm * 8)), 256, 0,
+                              stream>>>(H, d, hdr, A);
+    } else if (d <= kGatherSmemMax) {
         const size_t sm = static_cast<size_t>(d) * sizeof(float);
         static bool attr[64] = {};   // per device: the attribute is set per context
         int dev = 0;
