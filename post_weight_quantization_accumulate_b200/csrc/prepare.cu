@@ -100,26 +100,48 @@ __global__ void act_order_kernel(const float* __restrict__ H, int d, int act_ord
     if (i < d) perm[rank] = i;
 }
 
-// A[a][b] = H[q(a)][q(b)] + (a == b ? delta : 0), q(a) = perm[d-1-a]; one
-// row of H staged in shared memory per CTA (d <= kGatherSmemMax).
+// A[a][b] = H[q(a)][q(b)] + (a == b ? delta : 0), q(a) = perm[d-1-a]; the
+// reversed order q staged once per CTA and one row of H at a time, both in
+// shared memory (2 d floats, d <= kGatherSmemMax); rows read and written with
+// 16-byte accesses when d % 4 == 0 and H is 16-byte aligned.
 constexpr int kGatherSmemMax = 16384;
 __global__ void gather_rev_kernel(const float* __restrict__ H, int d,
                                   const int32_t* __restrict__ perm, const PrepHeader* hdr,
                                   float* __restrict__ A)
 {
-    extern __shared__ float rowbuf[];
+    extern __shared__ float gsm[];
+    float* rowbuf = gsm;
+    int* q = reinterpret_cast<int*>(gsm + d);
     const float delta = hdr->delta;
+    const bool vec = (d % 4) == 0 && (reinterpret_cast<uintptr_t>(H) & 15) == 0;
+    for (int b = threadIdx.x; b < d; b += blockDim.x) q[b] = perm[d - 1 - b];
     for (int a = blockIdx.x; a < d; a += gridDim.x) {
-        const int qa = perm[d - 1 - a];
-        __syncthreads();
-        const float* src = H + static_cast<int64_t>(qa) * d;
-        for (int j = threadIdx.x; j < d; j += blockDim.x) rowbuf[j] = src[j];
+        __syncthreads();   // q staged; the previous row's reads of rowbuf done
+        const float* src = H + static_cast<int64_t>(q[a]) * d;
+        if (vec) {
+            for (int j = threadIdx.x; j < d / 4; j += blockDim.x)
+                reinterpret_cast<float4*>(rowbuf)[j] = reinterpret_cast<const float4*>(src)[j];
+        } else {
+            for (int j = threadIdx.x; j < d; j += blockDim.x) rowbuf[j] = src[j];
+        }
         __syncthreads();
         float* dst = A + static_cast<int64_t>(a) * d;
-        for (int b = threadIdx.x; b < d; b += blockDim.x) {
-            float v = rowbuf[perm[d - 1 - b]];
-            if (b == a) v += delta;
-            dst[b] = v;
+        if (vec) {
+            for (int j = threadIdx.x; j < d / 4; j += blockDim.x) {
+                const int b = 4 * j;
+                float4 v = make_float4(rowbuf[q[b]], rowbuf[q[b + 1]], rowbuf[q[b + 2]], rowbuf[q[b + 3]]);
+                if (a == b) v.x += delta;
+                if (a == b + 1) v.y += delta;
+                if (a == b + 2) v.z += delta;
+                if (a == b + 3) v.w += delta;
+                reinterpret_cast<float4*>(dst)[j] = v;
+            }
+        } else {
+            for (int b = threadIdx.x; b < d; b += blockDim.x) {
+                float v = rowbuf[q[b]];
+                if (b == a) v += delta;
+                dst[b] = v;
+            }
         }
     }
 }
@@ -783,7 +805,7 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
         reverse_copy_kernel<<<static_cast<int>(std::min<int64_t>((n4 + 255) / 256, nsm * 8)), 256, 0,
                               stream>>>(H, d, hdr, A);
     } else if (d <= kGatherSmemMax) {
-        const size_t sm = static_cast<size_t>(d) * sizeof(float);
+        const size_t sm = 2 * static_cast<size_t>(d) * sizeof(float);
         static bool attr[64] = {};   // per device: the attribute is set per context
         int dev = 0;
         GPTQ_CUDA_CHECK(cudaGetDevice(&dev));
@@ -791,10 +813,12 @@ static int enqueue_prepare(const float* H, int64_t d64, float damp, int act_orde
         if (!attr[dev]) {
             GPTQ_CUDA_CHECK(cudaFuncSetAttribute(gather_rev_kernel,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kGatherSmemMax * static_cast<int>(sizeof(float))));
+                                                 2 * kGatherSmemMax * static_cast<int>(sizeof(float))));
             attr[dev] = true;
         }
-        gather_rev_kernel<<<std::min(d, nsm * 8), 256, sm, stream>>>(H, d, perm, hdr, A);
+        // CTAs per SM that fit next to each other, about two rows each
+        const int per_sm = std::max(1, static_cast<int>((220u * 1024u) / (sm + 1024)));
+        gather_rev_kernel<<<std::min(d, nsm * per_sm), 256, sm, stream>>>(H, d, perm, hdr, A);
     } else {
         gather_rev_direct_kernel<<<nsm * 8, 256, 0, stream>>>(H, d, perm, hdr, A);
     }
