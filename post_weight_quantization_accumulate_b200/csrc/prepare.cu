@@ -185,8 +185,8 @@ __global__ void reverse_copy_kernel(const float* __restrict__ H, int d, const Pr
 
 // One panel step of the blocked Cholesky, fused:
 //   every CTA factors the kb x kb diagonal block at (k0, k0) (redundantly, so
-//   no other launch has to wait for it) and inverts the factor; CTA 0 writes
-//   L_kk^{-1} into M^{-1}; CTA b in 1..n_trsm solves the panel rows
+//   no other launch has to wait for it); CTA 0 writes L_kk^{-1} (the solve
+//   with the identity) into M^{-1}; CTA b in 1..n_trsm solves the panel rows
 //   k0+kb+64(b-1) .. +63:  L[r][k0:k0+kb] = A[r][k0:k0+kb] L_kk^{-T};
 //   CTA n_trsm+1+c finishes column block c < k0/64 of row block k of M^{-1}:
 //   Y_k = L_kk^{-1} (Y~_k - L_k,k-1 Y_{k-1}), Y~_k holding the updates of the
@@ -197,11 +197,10 @@ __global__ void reverse_copy_kernel(const float* __restrict__ H, int d, const Pr
 // lower triangle (thread (ty, tx) owns the 4 x 4 tile rows 4ty.., cols 4tx..).
 // The factor is then used through triangular solves, never inverted as a
 // whole: the panel rows P solve P L^T = T and the row block of M^{-1} solves
-// L X = T, by substitution -- one thread per row (or column) of the 64 x 64
-// right-hand side, holding it in registers; at step s it divides entry s by
-// L[s][s] and subtracts the multiple of L's column s (read from a transposed
-// copy with 16-byte loads) from the later entries.  The diagonal block of
-// M^{-1} is the solve with T = I.
+// L X = T (as X^T L^T = T^T), by blocked substitution (solve_rows: 16 columns
+// at a time by one thread per row, then the block's product subtracted from
+// the later columns by all threads).  The diagonal block of M^{-1} is the
+// solve with T = I.
 // The previous panel's rows enter every product of the kernel as its k index
 // (the 64 columns of that panel), so they are kept k-major: KTile[k][r] with
 // 16-byte aligned rows, read four rows (or columns) of the product at a time.
