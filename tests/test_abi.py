@@ -168,3 +168,31 @@ def test_q4k_arguments_rejected_on_host(lib):
     assert q(sc6=None) == 1
     assert q(ws=None) == 6
     assert q(ws_bytes=100) == 6
+
+
+def test_a_c_program_links_and_calls_the_library(tmp_path):
+    """The boundary is plain C: a C99 program includes gptq.h, links
+    libgptq.so and calls the host-only entry points (no GPU needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "post_weight_quantization_accumulate_b200")
+    src = tmp_path / "t.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "gptq.h"\n'
+        "int main(void) {\n"
+        "  size_t ws = gptq_workspace_bytes(4096, 4096, 128);\n"
+        "  size_t bad = gptq_workspace_bytes(4096, -5, 128);\n"
+        '  printf("%d %zu %zu %s\\n", gptq_version(), ws, bad, gptq_status_string(1));\n'
+        "  return (gptq_version() > 0 && ws > 0 && bad == 0) ? 0 : 1;\n}\n")
+    exe = tmp_path / "t"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        str(src), "-L", pkg, "-lgptq", f"-Wl,-rpath,{pkg}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    version, ws, bad = r.stdout.split()[:3]
+    assert int(version) == B.gptq_version() and int(ws) == B.gptq_workspace_bytes(4096, 4096, 128)
